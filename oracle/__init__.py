@@ -1,0 +1,178 @@
+"""Oracle for per-RoPE-wavelength windowed causal attention (test infrastructure).
+
+Only the tests, the package's ``smoke()`` check and the CPU-baseline leg of
+``bench.py`` may import this module.  The product path (the CUDA library and
+its Python binding) never does, and the two share no code.
+
+The arithmetic lives in ``oracle.c`` (plain C, double precision, one thread);
+this module compiles it with the host C compiler on first use and exposes
+numpy-friendly wrappers.  Each wrapper names the passage it follows; see the
+header of ``oracle.c`` for the readings taken where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+T_INF = (1 << 63) - 1
+
+
+def build() -> str:
+    """Compile oracle.c into a shared object (idempotent)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if (not os.path.exists(_LIB_PATH)
+            or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            i64p = ctypes.POINTER(ctypes.c_int64)
+            u64p = ctypes.POINTER(ctypes.c_uint64)
+            dp = ctypes.POINTER(ctypes.c_double)
+            vp = ctypes.c_void_p
+            lib.oracle_thresholds.argtypes = [ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                              ctypes.c_int, i64p, dp]
+            lib.oracle_attention_rows.argtypes = [
+                vp, vp, vp, vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                ctypes.c_double, ctypes.c_int, ctypes.c_double, ctypes.c_int64, vp, vp, vp]
+            lib.oracle_scores.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
+                                          ctypes.c_int64, ctypes.c_double, ctypes.c_double,
+                                          ctypes.c_int, vp]
+            for name in ("oracle_count_bruteforce", "oracle_count_rows"):
+                getattr(lib, name).argtypes = [ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                               ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                               ctypes.c_int64, ctypes.c_int64, u64p, u64p]
+            _lib = lib
+    return _lib
+
+
+def _u16(a: np.ndarray) -> np.ndarray:
+    """bf16 payload as a contiguous uint16 array (accepts uint16 or torch bf16 bits)."""
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("oracle inputs are raw bf16 bit patterns (uint16)")
+    return a
+
+
+def thresholds(D: int, base: float, alpha: float, g: int):
+    """T_eff[p] per pair and the smallest distance of alpha*lambda_p to an integer.
+
+    ATFlash Abstract ("wavelength-proportional distance"), WavePrune Original
+    abstract (first rotation period at alpha = 1, 16-dim blocks for g = 8).
+    """
+    lib = _load()
+    T = np.zeros(D // 2, dtype=np.int64)
+    margin = ctypes.c_double(0.0)
+    rc = lib.oracle_thresholds(D, base, alpha, g,
+                               T.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                               ctypes.byref(margin))
+    if rc != 0:
+        raise ValueError("oracle_thresholds: bad arguments")
+    return T, margin.value
+
+
+def attention_rows(q, k, v, *, Hq, Hkv, q_pos0=0, k_pos0=0, base, alpha, g, scale,
+                   rows, kv_len=None):
+    """out [n, D] and lse [n] (float64) for the (b, h, t) triples in ``rows``.
+
+    q: uint16 [B, Nq, Hq, D]; k, v: uint16 [B, Nk, Hkv, D] (bf16 bit patterns).
+    ATFlash Abstract: windowed score, unchanged softmax.
+    """
+    lib = _load()
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    B, Nq, _, D = q.shape
+    Nk = k.shape[1]
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    n = rows.shape[0]
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros(n, dtype=np.float64)
+    kvl = None
+    if kv_len is not None:
+        kvl = np.ascontiguousarray(np.asarray(kv_len, dtype=np.int64))
+    rc = lib.oracle_attention_rows(
+        q.ctypes.data, k.ctypes.data, v.ctypes.data,
+        kvl.ctypes.data if kvl is not None else None,
+        B, Nq, Nk, Hq, Hkv, D, q_pos0, k_pos0, base, alpha, g, scale, n,
+        rows.ctypes.data, out.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_attention_rows failed ({rc})")
+    return out, lse
+
+
+def decode_rows(q, k_cache, v_cache, kv_len, *, Hq, Hkv, base, alpha, g, scale, rows=None):
+    """Decode: one new query per sequence at position kv_len[b]-1 over keys 0..kv_len[b]-1.
+
+    q: uint16 [B, Hq, D]; caches uint16 [B, Lmax, Hkv, D].  Same definition as
+    ``attention_rows`` with Nq = 1 and a per-sequence key count.
+    """
+    q = _u16(q)
+    B, _, D = q.shape
+    kv_len = np.asarray(kv_len, dtype=np.int64)
+    if rows is None:
+        rows = [(b, h) for b in range(B) for h in range(Hq)]
+    outs, lses = [], []
+    for (b, h) in rows:
+        # each sequence has its own query position, so rows go one at a time
+        qb = q[b:b + 1].reshape(1, 1, Hq, D)
+        o, l = attention_rows(qb, k_cache[b:b + 1], v_cache[b:b + 1], Hq=Hq, Hkv=Hkv,
+                              q_pos0=int(kv_len[b]) - 1, k_pos0=0, base=base, alpha=alpha,
+                              g=g, scale=scale, rows=[(0, h, 0)], kv_len=kv_len[b:b + 1])
+        outs.append(o[0])
+        lses.append(l[0])
+    return np.stack(outs), np.array(lses)
+
+
+def scores(qrow, keys, *, q_pos, k_pos0=0, base, alpha, g):
+    """Windowed scores (no scale) of one query row vs keys [n, D]; NaN = causal."""
+    lib = _load()
+    qrow, keys = _u16(qrow), _u16(keys)
+    n, D = keys.shape
+    s = np.zeros(n, dtype=np.float64)
+    rc = lib.oracle_scores(qrow.ctypes.data, keys.ctypes.data, n, D, q_pos, k_pos0,
+                           base, alpha, g, s.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_scores failed")
+    return s
+
+
+def _count(fn, D, base, alpha, g, Nq, Nk, q_pos0, k_pos0):
+    pr = ctypes.c_uint64(0)
+    tot = ctypes.c_uint64(0)
+    rc = fn(D, base, alpha, g, Nq, Nk, q_pos0, k_pos0, ctypes.byref(pr), ctypes.byref(tot))
+    if rc != 0:
+        raise ValueError("oracle count: bad arguments")
+    return pr.value, tot.value
+
+
+def count_bruteforce(D, base, alpha, g, Nq, Nk, q_pos0=0, k_pos0=0):
+    """(pruned, total) pair-terms per (batch, head) by full enumeration (tiny sizes)."""
+    return _count(_load().oracle_count_bruteforce, D, base, alpha, g, Nq, Nk, q_pos0, k_pos0)
+
+
+def count_rows(D, base, alpha, g, Nq, Nk, q_pos0=0, k_pos0=0):
+    """(pruned, total) pair-terms per (batch, head), one query row at a time.
+
+    ATFlash Abstract: the reduction rate is input-independent and has a
+    closed form in N.
+    """
+    return _count(_load().oracle_count_rows, D, base, alpha, g, Nq, Nk, q_pos0, k_pos0)

@@ -1,0 +1,162 @@
+"""Seeded synthetic inputs shared by the tests, the benchmark and the oracle checks.
+
+This module holds no part of the method's arithmetic: it only draws random
+tensors with the shapes and value distributions of the workloads.  The
+planted-key fixture scales one key so that its *longest-wavelength* pairs
+line up with a chosen query; which pairs those are is a fixed structural
+choice (the last ``PLANT_PAIRS`` pair indices), not a window computation.
+
+All tensors are bf16 in the layouts the library takes:
+  prefill  q [B, Nq, Hq, D], k/v [B, Nk, Hkv, D]
+  decode   q [B, Hq, D],     k/v cache [B, L, Hkv, D]
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+PLANT_PAIRS = 8  # pair indices P-8 .. P-1: the 8 longest RoPE wavelengths
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One synthetic workload: shapes, RoPE window parameters and input recipe."""
+    name: str
+    kind: str                      # "prefill" or "decode"
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    Nq: int                        # prefill queries (decode: 1)
+    Nk: int                        # prefill keys / decode cache length
+    base: float
+    alpha: float
+    g: int
+    q_pos0: int = 0
+    k_pos0: int = 0
+    pair_lognormal_sigma: float = 0.0   # >0: per-(head, pair) magnitudes for q and k
+    plant_key: bool = False
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+
+# Workloads of the pages' evaluation models, as single-layer attention shapes.
+WORKLOADS = {
+    "tiny": Workload("tiny", "prefill", 1, 1, 1, 64, 256, 256, 1e4, 1.0, 1),
+    "qwen2.5-0.5b-32k": Workload("qwen2.5-0.5b-32k", "prefill", 1, 14, 2, 64, 32768, 32768,
+                                 1e6, 1.0, 8, pair_lognormal_sigma=0.5),
+    "llama3.2-3b-128k-a1": Workload("llama3.2-3b-128k-a1", "prefill", 1, 24, 8, 128, 131072,
+                                    131072, 5e5, 1.0, 1, plant_key=True),
+    "llama3.2-3b-128k-a2": Workload("llama3.2-3b-128k-a2", "prefill", 1, 24, 8, 128, 131072,
+                                    131072, 5e5, 2.0, 1, plant_key=True),
+    "llama3.2-3b-decode-128k": Workload("llama3.2-3b-decode-128k", "decode", 16, 24, 8, 128, 1,
+                                        131072, 5e5, 1.0, 1),
+    "qwen2.5-7b-1m-prefill": Workload("qwen2.5-7b-1m-prefill", "prefill", 1, 28, 4, 128, 16384,
+                                      1048576, 1e7, 1.0, 8, q_pos0=1048576 - 16384),
+    "qwen2.5-7b-1m-decode": Workload("qwen2.5-7b-1m-decode", "decode", 1, 28, 4, 128, 1,
+                                     1048576, 1e7, 1.0, 8),
+}
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def randn_bf16(shape, seed: int, device="cpu") -> torch.Tensor:
+    """i.i.d. N(0, 1) rounded to bf16."""
+    x = torch.randn(shape, generator=_gen(seed, device), device=device, dtype=torch.float32)
+    return x.to(torch.bfloat16)
+
+
+def _pair_magnitudes(H: int, D: int, sigma: float, seed: int, device) -> torch.Tensor:
+    """[H, D] multipliers: one LogNormal(0, sigma) draw per (head, pair), shared by dims p, p+D/2."""
+    m = torch.exp(sigma * torch.randn((H, D // 2), generator=_gen(seed, device),
+                                      device=device, dtype=torch.float32))
+    return torch.cat([m, m], dim=1)
+
+
+def prefill_inputs(w: Workload, seed: int = 0, device="cpu"):
+    """(q, k, v, planted) for a prefill workload.
+
+    Generator seeds are 16*seed + {1: q, 2: k, 3: v, 4/5: q/k pair magnitudes, 6: planted key}.
+    """
+    s = seed * 16
+    shape_q = (w.B, w.Nq, w.Hq, w.D)
+    shape_k = (w.B, w.Nk, w.Hkv, w.D)
+    if w.pair_lognormal_sigma > 0:
+        q = torch.randn(shape_q, generator=_gen(s + 1, device), device=device)
+        k = torch.randn(shape_k, generator=_gen(s + 2, device), device=device)
+        q *= _pair_magnitudes(w.Hq, w.D, w.pair_lognormal_sigma, s + 4, device)
+        k *= _pair_magnitudes(w.Hkv, w.D, w.pair_lognormal_sigma, s + 5, device)
+        q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    else:
+        q = randn_bf16(shape_q, s + 1, device)
+        k = randn_bf16(shape_k, s + 2, device)
+    v = randn_bf16(shape_k, s + 3, device)
+    planted = []
+    if w.plant_key:
+        planted = plant_keys(q, k, Hq=w.Hq, Hkv=w.Hkv, scale=w.scale, seed=s + 6)
+    return q, k, v, planted
+
+
+def plant_keys(q: torch.Tensor, k: torch.Tensor, *, Hq: int, Hkv: int, scale: float, seed: int):
+    """Plant one aligned key per kv head (in place); returns [(b, hq, t, kvh, j*)].
+
+    For kv head kvh the probe query is the last row (t = Nq-1) of the group's
+    first query head.  A key index j* ~ U[0, Nk/2) is drawn; its last
+    ``PLANT_PAIRS`` pairs are set to c * (the query's same pairs), with c chosen
+    so that those pairs alone add ln(Nk) + 10 to the scaled score.  The other
+    pairs of the key stay random.  Values are rounded to bf16 afterwards.
+    """
+    B, Nq, _, D = q.shape
+    Nk = k.shape[1]
+    P = D // 2
+    G = Hq // Hkv
+    gen = _gen(seed, "cpu")
+    lo = list(range(P - PLANT_PAIRS, P)) + list(range(D - PLANT_PAIRS, D))
+    idx = torch.tensor(lo, device=q.device)
+    planted = []
+    for b in range(B):
+        for kvh in range(Hkv):
+            hq = kvh * G
+            t = Nq - 1
+            j = int(torch.randint(0, max(1, Nk // 2), (1,), generator=gen).item())
+            qv = q[b, t, hq].float()
+            qsel = qv[idx]
+            target = math.log(Nk) + 10.0
+            c = target / (scale * float((qsel * qsel).sum()))
+            row = k[b, j, kvh].float()
+            row[idx] = c * qsel
+            k[b, j, kvh] = row.to(torch.bfloat16)
+            planted.append((b, hq, t, kvh, j))
+    return planted
+
+
+def decode_inputs(w: Workload, seed: int = 0, device="cpu"):
+    """(q [B,Hq,D], k_cache, v_cache [B,L,Hkv,D], kv_len [B]) for a decode workload.
+
+    Every sequence is full (kv_len = L) unless ``w.extra['ragged']`` asks for
+    lengths drawn uniformly from [1, L].
+    """
+    s = seed * 16
+    q = randn_bf16((w.B, w.Hq, w.D), s + 7, device)
+    kc = randn_bf16((w.B, w.Nk, w.Hkv, w.D), s + 8, device)
+    vc = randn_bf16((w.B, w.Nk, w.Hkv, w.D), s + 9, device)
+    if w.extra.get("ragged"):
+        kv_len = torch.randint(1, w.Nk + 1, (w.B,), generator=_gen(s + 10, "cpu"),
+                               dtype=torch.int32)
+    else:
+        kv_len = torch.full((w.B,), w.Nk, dtype=torch.int32)
+    return q, kc, vc, kv_len
+
+
+def bits(t: torch.Tensor):
+    """bf16 tensor -> numpy uint16 bit patterns (CPU), the form the oracle reads."""
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view("uint16")

@@ -1,0 +1,280 @@
+"""Pins for the oracle: checks against facts other than the oracle itself.
+
+Each test names what it pins and where the fact comes from:
+hand-worked examples (tests/golden), a library routine the method reduces to
+(torch's scaled_dot_product_attention at alpha = inf), brute-force
+enumeration, closed forms of special cases, and invariants of the definition.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from rope_wavelength_sparsity_b200 import inputs
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16_bits(x: np.ndarray) -> np.ndarray:
+    return inputs.bits(torch.tensor(x, dtype=torch.float32).to(torch.bfloat16))
+
+
+def _rand(shape, seed):
+    return inputs.randn_bf16(shape, seed)
+
+
+# ---------------------------------------------------------------------------
+# hand-worked examples (ATFlash Abstract; WavePrune Original abstract)
+# ---------------------------------------------------------------------------
+
+def test_hand_two_pair_thresholds_scores_and_counts():
+    g = json.load(open(os.path.join(GOLD, "hand_two_pair.json")))
+    T, _ = oracle.thresholds(g["D"], g["base"], g["alpha"], g["g"])
+    assert T.tolist() == g["thresholds"]
+    q = _bf16_bits(np.array(g["q"]))
+    dmax = max(d for d, _ in g["score_by_distance"])
+    keys = _bf16_bits(np.tile(np.array(g["k"]), (dmax + 1, 1)))
+    # query at position dmax, key j at position j -> distance dmax - j
+    s = oracle.scores(q, keys, q_pos=dmax, base=g["base"], alpha=g["alpha"], g=g["g"])
+    for d, want in g["score_by_distance"]:
+        assert s[dmax - d] == want, (d, s[dmax - d], want)
+    for N, pruned, total in g["counts"]:
+        assert oracle.count_bruteforce(g["D"], g["base"], g["alpha"], g["g"], N, N) == (pruned, total)
+        assert oracle.count_rows(g["D"], g["base"], g["alpha"], g["g"], N, N) == (pruned, total)
+
+
+def test_threshold_values_by_hand():
+    cases = json.load(open(os.path.join(GOLD, "thresholds.json")))["cases"]
+    for c in cases:
+        T, margin = oracle.thresholds(c["D"], c["base"], c["alpha"], c["g"])
+        assert T[: len(c["first"])].tolist() == c["first"], c
+        assert margin > 1e-6
+
+
+def test_two_pair_softmax_by_hand():
+    """Query at position 7 over 8 keys (D = 4, base 100, alpha 1, T = (6, 62)).
+    Key 0 (d = 7) = (1,1,1,1): pair 0 pruned, s = 2 + 4 = 6.  Key 7 (d = 0) =
+    (0.5, 0, 0.25, 1): s = 0.5 + 0.75 + 4 = 5.25.  Keys 1..6 are zero: s = 0.
+    With scale 1 the weights are (e^6, 1, ..., 1, e^5.25) / Z."""
+    q = _bf16_bits(np.array([1.0, 2.0, 3.0, 4.0]).reshape(1, 1, 1, 4))
+    kk = np.zeros((1, 8, 1, 4))
+    vv = np.zeros((1, 8, 1, 4))
+    kk[0, 0, 0] = [1.0, 1.0, 1.0, 1.0]
+    kk[0, 7, 0] = [0.5, 0.0, 0.25, 1.0]
+    vv[0, 0, 0] = [1.0, 0.0, 0.0, 0.0]
+    vv[0, 7, 0] = [0.0, 1.0, 0.0, 0.0]
+    out, lse = oracle.attention_rows(q, _bf16_bits(kk), _bf16_bits(vv), Hq=1, Hkv=1,
+                                     q_pos0=7, k_pos0=0, base=100.0, alpha=1.0, g=1,
+                                     scale=1.0, rows=[(0, 0, 0)])
+    z = math.exp(6.0) + math.exp(5.25) + 6 * math.exp(0.0)
+    assert abs(out[0, 0] - math.exp(6.0) / z) < 1e-12
+    assert abs(out[0, 1] - math.exp(5.25) / z) < 1e-12
+    assert abs(lse[0] - math.log(z)) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# alpha = inf reduces to ordinary causal attention (a library routine)
+# ---------------------------------------------------------------------------
+
+def _sdpa_reference(q, k, v, Hq, Hkv, q_pos0, k_pos0, scale):
+    qf = q.double().permute(0, 2, 1, 3)                # B,Hq,Nq,D
+    kf = k.double().repeat_interleave(Hq // Hkv, dim=2).permute(0, 2, 1, 3)
+    vf = v.double().repeat_interleave(Hq // Hkv, dim=2).permute(0, 2, 1, 3)
+    Nq, Nk = q.shape[1], k.shape[1]
+    qp = q_pos0 + torch.arange(Nq)
+    kp = k_pos0 + torch.arange(Nk)
+    mask = kp[None, :] <= qp[:, None]
+    out = torch.nn.functional.scaled_dot_product_attention(qf, kf, vf, attn_mask=mask, scale=scale)
+    return out.permute(0, 2, 1, 3)
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,Nq,Nk,q0,k0", [
+    (16, 4, 2, 37, 37, 0, 0),
+    (64, 3, 1, 20, 45, 25, 0),
+    (8, 2, 2, 9, 30, 100, 80),
+])
+def test_alpha_inf_is_causal_sdpa(D, Hq, Hkv, Nq, Nk, q0, k0):
+    q = _rand((2, Nq, Hq, D), 11)
+    k = _rand((2, Nk, Hkv, D), 12)
+    v = _rand((2, Nk, Hkv, D), 13)
+    scale = 1.0 / math.sqrt(D)
+    ref = _sdpa_reference(q, k, v, Hq, Hkv, q0, k0, scale)
+    rows = [(b, h, t) for b in range(2) for h in range(Hq) for t in range(Nq)
+            if q0 + t >= k0]
+    out, lse = oracle.attention_rows(inputs.bits(q), inputs.bits(k), inputs.bits(v), Hq=Hq,
+                                     Hkv=Hkv, q_pos0=q0, k_pos0=k0, base=1e4,
+                                     alpha=float("inf"), g=1, scale=scale, rows=rows)
+    for n, (b, h, t) in enumerate(rows):
+        np.testing.assert_allclose(out[n], ref[b, t, h].numpy(), rtol=0, atol=1e-10)
+
+
+# ---------------------------------------------------------------------------
+# special cases with a closed form
+# ---------------------------------------------------------------------------
+
+def test_small_alpha_keeps_only_distance_zero():
+    """alpha * lambda_{P-1} < 1 (the longest wavelength): every T_p = 0, so a
+    key j < i scores exactly 0 and the row's softmax is
+    (e^{z_ii}, 1, ..., 1) / (e^{z_ii} + i)."""
+    D, N = 16, 24
+    alpha = 0.9 / (2 * math.pi * 1e4 ** (2 * 7 / 16))
+    T, _ = oracle.thresholds(D, 1e4, alpha, 1)
+    assert (T == 0).all()
+    q = _rand((1, N, 1, D), 21)
+    k = _rand((1, N, 1, D), 22)
+    v = _rand((1, N, 1, D), 23)
+    scale = 0.25
+    rows = [(0, 0, t) for t in range(N)]
+    out, lse = oracle.attention_rows(inputs.bits(q), inputs.bits(k), inputs.bits(v), Hq=1,
+                                     Hkv=1, base=1e4, alpha=alpha, g=1, scale=scale, rows=rows)
+    qd, kd, vd = q.double()[0, :, 0], k.double()[0, :, 0], v.double()[0, :, 0]
+    for t in range(N):
+        zt = scale * float(qd[t] @ kd[t])
+        w_self = math.exp(zt)
+        want = (w_self * vd[t] + vd[:t].sum(0)) / (w_self + t)
+        np.testing.assert_allclose(out[t], want.numpy(), atol=1e-12)
+        assert abs(lse[t] - math.log(w_self + t)) < 1e-12
+
+
+def test_distance_zero_keeps_every_pair():
+    """d = 0 keeps all pairs: the diagonal score is the full dot product."""
+    for D, base, alpha, g in [(64, 1e4, 1.0, 1), (128, 5e5, 0.01, 1), (64, 1e6, 0.001, 8)]:
+        q = _rand((1, D), 31)
+        k = _rand((1, D), 32)
+        s = oracle.scores(inputs.bits(q)[0], inputs.bits(k), q_pos=5, k_pos0=5, base=base,
+                          alpha=alpha, g=g)
+        assert abs(s[0] - float(q.double()[0] @ k.double()[0])) < 1e-12
+
+
+def test_half_split_pairing_not_interleaved():
+    """Pair p couples dims p and p + D/2: with only dims (0, D/2) nonzero in
+    q and k, the term survives exactly while pair 0 is kept (d <= T_0)."""
+    D = 8
+    T, _ = oracle.thresholds(D, 100.0, 1.0, 1)
+    qv = np.zeros(D); qv[0] = 1.0; qv[D // 2] = 2.0
+    kv = np.zeros(D); kv[0] = 3.0; kv[D // 2] = 5.0
+    n = int(T[0]) + 3
+    keys = _bf16_bits(np.tile(kv, (n, 1)))
+    s = oracle.scores(_bf16_bits(qv), keys, q_pos=n - 1, base=100.0, alpha=1.0, g=1)
+    for j in range(n):
+        d = n - 1 - j
+        assert s[j] == (13.0 if d <= T[0] else 0.0)
+
+
+def test_group_window_uses_longest_wavelength():
+    """g = 8: a group stays while its longest-wavelength member would; with a
+    single pair active in q (pair 0), the term survives to T_7, not T_0."""
+    D = 16
+    T1, _ = oracle.thresholds(D, 100.0, 1.0, 1)
+    T8, _ = oracle.thresholds(D, 100.0, 1.0, 8)
+    assert (T8 == T1[7]).all()
+    qv = np.zeros(D); qv[0] = 1.0
+    kv = np.zeros(D); kv[0] = 1.0
+    d_probe = int(T1[0]) + 1            # pruned with g = 1, kept with g = 8
+    keys = _bf16_bits(np.tile(kv, (d_probe + 1, 1)))
+    s1 = oracle.scores(_bf16_bits(qv), keys, q_pos=d_probe, base=100.0, alpha=1.0, g=1)
+    s8 = oracle.scores(_bf16_bits(qv), keys, q_pos=d_probe, base=100.0, alpha=1.0, g=8)
+    assert s1[0] == 0.0 and s8[0] == 1.0
+
+
+def test_empty_row_has_zero_output_and_minus_inf_lse():
+    q = _rand((1, 4, 1, 16), 41)
+    k = _rand((1, 4, 1, 16), 42)
+    v = _rand((1, 4, 1, 16), 43)
+    out, lse = oracle.attention_rows(inputs.bits(q), inputs.bits(k), inputs.bits(v), Hq=1,
+                                     Hkv=1, q_pos0=0, k_pos0=10, base=1e4, alpha=1.0, g=1,
+                                     scale=0.25, rows=[(0, 0, 3)])
+    assert (out == 0).all() and lse[0] == -math.inf
+
+
+# ---------------------------------------------------------------------------
+# the count: brute force, closed form, logarithmic growth
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("D", [4, 8, 16, 64, 128])
+@pytest.mark.parametrize("alpha", [0.05, 0.5, 1.0, 2.0, 7.3, float("inf")])
+def test_count_rows_equals_bruteforce(D, alpha):
+    for g in (1, 8):
+        if g == 8 and (D // 2) % 8:
+            continue
+        for (Nq, Nk, q0, k0) in [(1, 1, 0, 0), (37, 37, 0, 0), (50, 130, 80, 0),
+                                 (64, 20, 10, 30), (5, 300, 299, 0), (40, 40, 0, 50)]:
+            bf = oracle.count_bruteforce(D, 100.0 if D <= 8 else 1e4, alpha, g, Nq, Nk, q0, k0)
+            rw = oracle.count_rows(D, 100.0 if D <= 8 else 1e4, alpha, g, Nq, Nk, q0, k0)
+            assert bf == rw, (D, alpha, g, Nq, Nk, q0, k0)
+
+
+def test_pruned_fraction_grows_logarithmically():
+    """Continuum form of the count for a causal N x N square (our derivation of
+    the ATFlash Abstract's 'closed form logarithmic in N'):
+    fraction ~= (ln(N / (2 pi alpha)) - 3/2) / ln(base) while 2 pi alpha << N <= reach of the
+    last pair.  Doubling N adds ~ ln 2 / ln(base)."""
+    D, base, alpha = 128, 5e5, 1.0
+    prev = None
+    for N in (8192, 16384, 32768, 65536, 131072):
+        pr, tot = oracle.count_rows(D, base, alpha, 1, N, N)
+        frac = pr / tot
+        approx = (math.log(N / (2 * math.pi * alpha)) - 1.5) / math.log(base)
+        assert abs(frac - approx) < 0.02, (N, frac, approx)
+        if prev is not None:
+            assert abs((frac - prev) - math.log(2) / math.log(base)) < 0.01
+        prev = frac
+
+
+def test_count_monotone_in_alpha_and_suffix_structure():
+    D, base, N = 64, 1e4, 200
+    last = None
+    for alpha in (0.1, 0.5, 1.0, 2.0, 4.0):
+        pr, _ = oracle.count_rows(D, base, alpha, 1, N, N)
+        if last is not None:
+            assert pr <= last
+        last = pr
+        T, _ = oracle.thresholds(D, base, alpha, 1)
+        assert (np.diff(T) >= 0).all()          # kept set at any d is a suffix of pairs
+
+
+# ---------------------------------------------------------------------------
+# reachability (ATFlash Abstract: every key stays reachable through the
+# low-frequency pairs)
+# ---------------------------------------------------------------------------
+
+def test_planted_key_is_reachable():
+    w = inputs.Workload("plant", "prefill", 1, 4, 2, 128, 2048, 2048, 5e5, 1.0, 1, plant_key=True)
+    q, k, v, planted = inputs.prefill_inputs(w, seed=0)
+    for (b, hq, t, kvh, j) in planted:
+        out, lse = oracle.attention_rows(inputs.bits(q), inputs.bits(k), inputs.bits(v),
+                                         Hq=w.Hq, Hkv=w.Hkv, base=w.base, alpha=w.alpha,
+                                         g=w.g, scale=w.scale, rows=[(b, hq, t)])
+        s = oracle.scores(inputs.bits(q)[b, t, hq], inputs.bits(k)[b, :, kvh], q_pos=t,
+                          base=w.base, alpha=w.alpha, g=w.g)
+        weight = math.exp(w.scale * s[j] - lse[0])
+        assert weight > 0.99, weight
+        np.testing.assert_allclose(out[0], v[b, j, kvh].double().numpy(), atol=0.05)
+
+
+# ---------------------------------------------------------------------------
+# decode = the same definition with one query per sequence at kv_len - 1
+# ---------------------------------------------------------------------------
+
+def test_decode_rows_match_causal_sdpa_when_window_off():
+    B, Hq, Hkv, D, L = 3, 4, 2, 16, 40
+    q = _rand((B, Hq, D), 51)
+    kc = _rand((B, L, Hkv, D), 52)
+    vc = _rand((B, L, Hkv, D), 53)
+    kv_len = [40, 1, 17]
+    out, lse = oracle.decode_rows(inputs.bits(q), inputs.bits(kc), inputs.bits(vc), kv_len,
+                                  Hq=Hq, Hkv=Hkv, base=1e4, alpha=float("inf"), g=1, scale=0.25)
+    n = 0
+    for b in range(B):
+        for h in range(Hq):
+            kk = kc[b, :kv_len[b], h // (Hq // Hkv)].double()
+            vv = vc[b, :kv_len[b], h // (Hq // Hkv)].double()
+            z = 0.25 * (kk @ q[b, h].double())
+            want = torch.softmax(z, 0) @ vv
+            np.testing.assert_allclose(out[n], want.numpy(), atol=1e-10)
+            assert abs(lse[n] - float(torch.logsumexp(z, 0))) < 1e-10
+            n += 1
