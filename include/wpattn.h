@@ -1,0 +1,163 @@
+/*
+ * wpattn — per-RoPE-wavelength windowed causal attention on NVIDIA B200 (sm_100a).
+ *
+ * The method ("ATFlash: Per-RoPE-Wavelength Attention Windows", Abstract;
+ * "WavePrune: One period is often enough for RoPE", Original abstract):
+ * the RoPE attention score is a sum of one term per 2-D rotation pair p
+ * (dims p and p + D/2), and the window drops pair p's term once the
+ * query-key distance d = q_pos - k_pos exceeds T_p = floor(alpha * lambda_p),
+ * lambda_p = 2*pi * base^(2p/D).  Dropped terms add 0 to the score; the
+ * causal softmax over keys is unchanged:
+ *
+ *     s(i,j) = sum_p [d <= T_p] * (q[i,p] k[j,p] + q[i,p+D/2] k[j,p+D/2])
+ *     out_i  = softmax_j(scale * s(i,j)) . v_j      over keys with k_pos <= q_pos
+ *
+ * With group_pairs = 8 the pairs {8m..8m+7} (16 head dims, the Tensor-Core
+ * block size of WavePrune's kernels) share the threshold of the group's
+ * longest wavelength, T_{8m+7}.  alpha = +INFINITY disables the window.
+ *
+ * Conventions for every entry point:
+ *  - Return value: WPATTN_OK or an error code (wpattn_strerror names it).
+ *    Argument errors are reported synchronously and nothing is launched.
+ *  - Device pointers are plain CUDA device addresses of the current device;
+ *    the caller owns every buffer.  Kernels run asynchronously on
+ *    `cuda_stream` (a cudaStream_t; NULL = the legacy default stream); the
+ *    call does not synchronise.  A kernel fault shows at the caller's next
+ *    synchronisation.  A kernel that gives up waiting (a bounded spin ran out)
+ *    records WPATTN_ETIMEOUT, which wpattn_device_status returns.
+ *  - bf16 tensors are contiguous, row-major, in the layouts stated below, and
+ *    16-byte aligned.
+ *  - The library allocates no device memory in the calls below except a
+ *    4-byte status word per device, created on first use.
+ */
+#ifndef WPATTN_H
+#define WPATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define WPATTN_API __attribute__((visibility("default")))
+#else
+#define WPATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+enum {
+    WPATTN_OK = 0,
+    WPATTN_EINVAL = 1,        /* bad argument (null pointer, bad shape, alpha <= 0 or NaN, ...) */
+    WPATTN_EUNSUPPORTED = 2,  /* valid but not supported here (head_dim, device arch, size limit) */
+    WPATTN_ECUDA = 3,         /* a CUDA runtime call or a kernel launch failed */
+    WPATTN_ETIMEOUT = 4,      /* a kernel's bounded wait ran out (see wpattn_device_status) */
+    WPATTN_EWORKSPACE = 5     /* workspace null or smaller than wpattn_decode_workspace_size */
+};
+
+/*
+ * The window: head dim D (64 or 128 on the GPU paths; any even D for the
+ * host planner), RoPE base (> 1), factor alpha (> 0; +INFINITY = window off)
+ * and pair granularity g (1 or 8; 8 needs D/2 divisible by 8).
+ * T_p is evaluated on the host in IEEE double as
+ *     floor(alpha * (6.283185307179586 * pow(base, (double)(2p) / D)))
+ * and every device comparison is an integer one.
+ */
+typedef struct wpattn_window {
+    int32_t head_dim;
+    int32_t group_pairs;
+    double rope_base;
+    double alpha;
+} wpattn_window;
+
+/*
+ * Per-pair thresholds T_eff[p], p = 0 .. D/2 - 1 (host only; ATFlash
+ * Abstract: "wavelength-proportional distance").  With g = 8 each pair holds
+ * its group's threshold.  A disabled window reports INT64_MAX.
+ * T_eff: caller-owned host array of D/2 entries.
+ */
+WPATTN_API int wpattn_thresholds(const wpattn_window *w, int64_t *T_eff);
+
+/*
+ * Pruned pair-terms of one (batch, head) of a prefill (host only, O(D)
+ * closed form; ATFlash Abstract: "closed form logarithmic in the sequence
+ * length").  Queries t = 0..Nq-1 sit at q_pos0 + t, keys j = 0..Nk-1 at
+ * k_pos0 + j; every causal (query, key) pair contributes D/2 pair-terms and
+ * a term is pruned when its distance exceeds its pair's threshold.
+ * Outputs (host pointers, any may be NULL): pruned and total term counts and
+ * their ratio (0 when total is 0).
+ */
+WPATTN_API int wpattn_pruned_fraction(const wpattn_window *w, int64_t Nq, int64_t Nk,
+                           int64_t q_pos0, int64_t k_pos0,
+                           uint64_t *pruned_terms, uint64_t *total_terms,
+                           double *fraction);
+
+/*
+ * Prefill (ATFlash Abstract: the window as a slice of the query-key
+ * contraction axis inside a FlashAttention-style kernel; WavePrune: 16-dim
+ * head-dim blocks for the Tensor Cores).
+ *   q   : bf16 device [B, Nq, Hq, D]      query t at position q_pos0 + t
+ *   k, v: bf16 device [B, Nk, Hkv, D]     key j at position k_pos0 + j
+ *   out : bf16 device [B, Nq, Hq, D]      written
+ *   lse : fp32 device [B, Hq, Nq] natural-log sum-exp of scale*s, or NULL
+ * Query head h reads kv head h / (Hq / Hkv).  softmax_scale <= 0 means
+ * 1/sqrt(D).  A query with no causal key gets out = 0 and lse = -inf.
+ * Requires D in {64, 128}, Hq % Hkv == 0, an sm_100 device, and
+ * 0 <= Nq, Nk < 2^31.  Nq == 0 or B == 0 is a no-op.
+ */
+WPATTN_API int wpattn_prefill(const wpattn_window *w,
+                   const void *q, const void *k, const void *v,
+                   void *out, float *lse,
+                   int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
+                   int64_t q_pos0, int64_t k_pos0, float softmax_scale,
+                   void *cuda_stream);
+
+/*
+ * Bytes of device workspace wpattn_decode needs for up to B sequences of up
+ * to max_kv_len keys (0 on bad arguments).  The split of each sequence into
+ * key ranges depends only on (B, Hkv, max_kv_len) and the device's SM count.
+ */
+WPATTN_API size_t wpattn_decode_workspace_size(const wpattn_window *w, int32_t B, int32_t Hq,
+                                    int32_t Hkv, int64_t max_kv_len);
+
+/*
+ * Decode: one new query per sequence (ATFlash Abstract: the window ported
+ * into a FlashInfer-style decode; K is read only over the active head-dim
+ * slice of each key block).
+ *   q          : bf16 device [B, Hq, D]; sequence b's query sits at position kv_len[b]-1
+ *   k_cache,
+ *   v_cache    : bf16 device [B, Lmax, Hkv, D]; key j at position j, j < kv_len[b] valid
+ *   kv_len_host: host int32 [B], 1 <= kv_len[b] <= Lmax (read during the call)
+ *   out        : bf16 device [B, Hq, D];  lse: fp32 device [B, Hq] or NULL
+ *   workspace  : device, >= wpattn_decode_workspace_size(w, B, Hq, Hkv, Lmax)
+ *                bytes, 256-byte aligned; its contents are scratch (fp32 partial
+ *                results of each key range) and are overwritten.
+ * Requires D in {64, 128}, Hq % Hkv == 0, Hq / Hkv <= 16, B <= 4096.
+ */
+WPATTN_API int wpattn_decode(const wpattn_window *w,
+                  const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *kv_len_host, int64_t Lmax,
+                  int32_t B, int32_t Hq, int32_t Hkv, float softmax_scale,
+                  void *out, float *lse,
+                  void *workspace, size_t workspace_bytes,
+                  void *cuda_stream);
+
+/*
+ * Synchronises `cuda_stream`, then reads and clears the current device's
+ * kernel status word.  Returns WPATTN_OK, WPATTN_ETIMEOUT (a kernel gave up a
+ * bounded wait; its outputs are undefined) or WPATTN_ECUDA.
+ */
+WPATTN_API int wpattn_device_status(void *cuda_stream);
+
+/* Static English text for a status code. */
+WPATTN_API const char *wpattn_strerror(int code);
+
+/* Library version as "major.minor.patch". */
+WPATTN_API const char *wpattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WPATTN_H */

@@ -1,1 +1,191 @@
-"""Per-RoPE-wavelength windowed causal attention for NVIDIA B200 (sm_100a)."""
+"""Per-RoPE-wavelength windowed causal attention for NVIDIA B200 (sm_100a).
+
+Thin Python binding of the C ABI in ``include/wpattn.h`` (``libwpattn.so``,
+built in-tree by ``rope_wavelength_sparsity_b200.build``).  The binding only
+marshals arguments: tensors are passed as raw device pointers and every
+step of the computation runs in the library's CUDA kernels.  There is no
+fallback path: if the shared library is missing or a call fails, an
+exception is raised.
+
+Entry points (same names as the C ABI, without the ``wpattn_`` prefix):
+``prefill``, ``decode``, ``decode_workspace_size``, ``pruned_fraction``,
+``thresholds``, ``device_status``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libwpattn.so")
+
+OK, EINVAL, EUNSUPPORTED, ECUDA, ETIMEOUT, EWORKSPACE = range(6)
+
+
+class WpattnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {_strerror(code)} (code {code})")
+
+
+class _Window(ctypes.Structure):
+    _fields_ = [("head_dim", ctypes.c_int32), ("group_pairs", ctypes.c_int32),
+                ("rope_base", ctypes.c_double), ("alpha", ctypes.c_double)]
+
+
+@dataclass(frozen=True)
+class Window:
+    """RoPE window: head dim D, base, factor alpha (inf = off), pair granularity g (1 or 8)."""
+    head_dim: int
+    rope_base: float
+    alpha: float
+    group_pairs: int = 1
+
+    def _c(self) -> _Window:
+        return _Window(self.head_dim, self.group_pairs, float(self.rope_base), float(self.alpha))
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ``libwpattn.so``; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m rope_wavelength_sparsity_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+        wp = ctypes.POINTER(_Window)
+        L.wpattn_thresholds.argtypes = [wp, ctypes.POINTER(ctypes.c_int64)]
+        L.wpattn_pruned_fraction.argtypes = [wp, i64, i64, i64, i64,
+                                             ctypes.POINTER(ctypes.c_uint64),
+                                             ctypes.POINTER(ctypes.c_uint64),
+                                             ctypes.POINTER(ctypes.c_double)]
+        L.wpattn_prefill.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64, i64,
+                                     f32, vp]
+        L.wpattn_decode_workspace_size.restype = ctypes.c_size_t
+        L.wpattn_decode_workspace_size.argtypes = [wp, i32, i32, i32, i64]
+        L.wpattn_decode.argtypes = [wp, vp, vp, vp, ctypes.POINTER(ctypes.c_int32), i64, i32, i32,
+                                    i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
+        L.wpattn_device_status.argtypes = [vp]
+        L.wpattn_strerror.restype = ctypes.c_char_p
+        L.wpattn_strerror.argtypes = [ctypes.c_int]
+        L.wpattn_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _strerror(code: int) -> str:
+    try:
+        return lib().wpattn_strerror(code).decode()
+    except Exception:  # pragma: no cover - only when the library itself is absent
+        return "unknown"
+
+
+def _check(code: int, what: str):
+    if code != OK:
+        raise WpattnError(code, what)
+
+
+def version() -> str:
+    return lib().wpattn_version().decode()
+
+
+def thresholds(w: Window):
+    """Per-pair thresholds T_eff[p] (list of D/2 ints; 2**63-1 = no limit)."""
+    arr = (ctypes.c_int64 * (w.head_dim // 2))()
+    _check(lib().wpattn_thresholds(ctypes.byref(w._c()), arr), "wpattn_thresholds")
+    return list(arr)
+
+
+def pruned_fraction(w: Window, Nq: int, Nk: int, q_pos0: int = 0, k_pos0: int = 0):
+    """(pruned_terms, total_terms, fraction) per (batch, head) from the closed form."""
+    pr, tot, fr = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_double()
+    _check(lib().wpattn_pruned_fraction(ctypes.byref(w._c()), Nq, Nk, q_pos0, k_pos0,
+                                        ctypes.byref(pr), ctypes.byref(tot), ctypes.byref(fr)),
+           "wpattn_pruned_fraction")
+    return pr.value, tot.value, fr.value
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev_tensor(t, name):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16 or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous bf16 tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def prefill(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0, scale: float | None = None,
+            out=None, lse=None, want_lse: bool = True, stream=None):
+    """Windowed causal prefill.  q [B,Nq,Hq,D], k/v [B,Nk,Hkv,D] bf16 CUDA tensors.
+
+    Returns (out [B,Nq,Hq,D] bf16, lse [B,Hq,Nq] fp32 or None).
+    """
+    import torch
+    B, Nq, Hq, D = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = lib().wpattn_prefill(ctypes.byref(w._c()), _dev_tensor(q, "q"), _dev_tensor(k, "k"),
+                              _dev_tensor(v, "v"), _dev_tensor(out, "out"),
+                              ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+                              B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0,
+                              float(scale) if scale else 0.0, _stream_ptr(stream))
+    _check(rc, "wpattn_prefill")
+    return out, lse
+
+
+def decode_workspace_size(w: Window, B: int, Hq: int, Hkv: int, max_kv_len: int) -> int:
+    return int(lib().wpattn_decode_workspace_size(ctypes.byref(w._c()), B, Hq, Hkv, max_kv_len))
+
+
+def decode(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | None = None, out=None,
+           lse=None, want_lse: bool = True, workspace=None, stream=None):
+    """Windowed decode.  q [B,Hq,D]; caches [B,L,Hkv,D] bf16 CUDA; kv_len: host ints [B].
+
+    Returns (out [B,Hq,D] bf16, lse [B,Hq] fp32 or None).
+    """
+    import torch
+    B, Hq, D = q.shape
+    L, Hkv = k_cache.shape[1], k_cache.shape[2]
+    kvl = (ctypes.c_int32 * B)(*[int(x) for x in kv_len])
+    if workspace is None:
+        n = decode_workspace_size(w, B, Hq, Hkv, L)
+        if n == 0:
+            raise WpattnError(EINVAL, "wpattn_decode_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    rc = lib().wpattn_decode(ctypes.byref(w._c()), _dev_tensor(q, "q"),
+                             _dev_tensor(k_cache, "k_cache"), _dev_tensor(v_cache, "v_cache"),
+                             kvl, L, B, Hq, Hkv, float(scale) if scale else 0.0,
+                             _dev_tensor(out, "out"),
+                             ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+                             ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                             _stream_ptr(stream))
+    _check(rc, "wpattn_decode")
+    return out, lse
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the kernels' status word."""
+    return int(lib().wpattn_device_status(_stream_ptr(stream)))
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

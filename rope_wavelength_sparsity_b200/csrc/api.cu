@@ -1,0 +1,307 @@
+// C ABI of the windowed-attention library (declarations and contracts in
+// include/wpattn.h).  Host side: argument checks, the planner, TMA tensor
+// maps and kernel launches.  Every step of the computation runs in the
+// kernels of decode_kernels.cuh and prefill_kernel.cuh.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "wpattn.h"
+#include "planner.h"
+#include "device_util.cuh"
+#include "decode_kernels.cuh"
+#include "prefill_kernel.cuh"
+
+namespace wpattn {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library links no libcuda and loads on hosts without a GPU driver.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+struct DeviceInfo {
+  bool init = false;
+  bool supported = false;
+  int num_sms = 0;
+  bool prefill_attr[2] = {false, false};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WPATTN_ECUDA;
+  if (dev < 0 || dev >= kMaxDevices) return WPATTN_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return WPATTN_ECUDA;
+    d.supported = (major == 10 && minor == 0);
+    d.num_sms = sms;
+    d.init = true;
+  }
+  *out = &d;
+  return d.supported ? WPATTN_OK : WPATTN_EUNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int encode_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                   uint64_t d3, uint32_t box0, uint32_t box1, bool swizzle128) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return WPATTN_ECUDA;
+  const cuuint64_t dims[4] = {d0, d1, d2, d3};
+  const cuuint64_t strides[3] = {d0 * d2 * 2, d0 * 2, d0 * d1 * d2 * 2};  // row, head, batch
+  const cuuint32_t box[4] = {box0, box1, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? WPATTN_OK : WPATTN_ECUDA;
+}
+
+template <int D>
+int launch_prefill(const void* q, const void* k, const void* v, const PrefillParams& prm,
+                   DeviceInfo* dev, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  int rc;
+  // tensors are [B, N, H, D]: dims (fastest first) D, N, H, B
+  if ((rc = encode_bf16_4d(&tq, q, D, prm.Nq, prm.Hq, prm.B, 8, kBM, false)) != WPATTN_OK) return rc;
+  // with no key the kernel issues no K/V load; the maps only need to be valid
+  const uint64_t nk = prm.Nk > 0 ? prm.Nk : prm.Nq;
+  const uint64_t hk = prm.Nk > 0 ? prm.Hkv : prm.Hq;
+  if ((rc = encode_bf16_4d(&tk, k, D, nk, hk, prm.B, 8, kBN, false)) != WPATTN_OK) return rc;
+  if ((rc = encode_bf16_4d(&tv, v, D, nk, hk, prm.B, 64, kBN, true)) != WPATTN_OK) return rc;
+  constexpr int smem = PrefillSmem<D>::ALLOC;
+  const int slot = (D == 64) ? 0 : 1;
+  if (!dev->prefill_attr[slot]) {
+    if (cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return WPATTN_ECUDA;
+    dev->prefill_attr[slot] = true;
+  }
+  dim3 grid(prm.num_qtiles, prm.Hq, prm.B);
+  prefill_kernel<D><<<grid, kPrefillThreads, smem, st>>>(tq, tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
+}
+
+template <int D, int GC>
+int launch_decode_split(const DecodeParams& prm, cudaStream_t st) {
+  dim3 grid(prm.S, prm.Hkv * prm.hchunks, prm.B);
+  decode_split_kernel<D, GC><<<grid, kDecodeThreads, 0, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
+}
+
+template <int D>
+int launch_decode(const DecodeParams& prm, int gc, cudaStream_t st) {
+  int rc;
+  switch (gc) {
+    case 1: rc = launch_decode_split<D, 1>(prm, st); break;
+    case 2: rc = launch_decode_split<D, 2>(prm, st); break;
+    case 3: rc = launch_decode_split<D, 3>(prm, st); break;
+    case 4: rc = launch_decode_split<D, 4>(prm, st); break;
+    case 5: rc = launch_decode_split<D, 5>(prm, st); break;
+    case 6: rc = launch_decode_split<D, 6>(prm, st); break;
+    case 7: rc = launch_decode_split<D, 7>(prm, st); break;
+    case 8: rc = launch_decode_split<D, 8>(prm, st); break;
+    default: return WPATTN_EUNSUPPORTED;
+  }
+  if (rc != WPATTN_OK) return rc;
+  const size_t smem = static_cast<size_t>(prm.S) * 2 * sizeof(float);
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(decode_combine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return WPATTN_ECUDA;
+  }
+  decode_combine_kernel<D><<<prm.B * prm.Hq, D, smem, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
+}
+
+}  // namespace
+}  // namespace wpattn
+
+using namespace wpattn;
+
+extern "C" {
+
+const char* wpattn_version(void) { return "0.1.0"; }
+
+const char* wpattn_strerror(int code) {
+  switch (code) {
+    case WPATTN_OK: return "ok";
+    case WPATTN_EINVAL: return "invalid argument";
+    case WPATTN_EUNSUPPORTED: return "unsupported configuration or device";
+    case WPATTN_ECUDA: return "CUDA runtime or launch error";
+    case WPATTN_ETIMEOUT: return "a kernel gave up a bounded wait";
+    case WPATTN_EWORKSPACE: return "workspace missing or too small";
+    default: return "unknown status code";
+  }
+}
+
+int wpattn_thresholds(const wpattn_window* w, int64_t* T_eff) {
+  if (!w || !T_eff) return WPATTN_EINVAL;
+  WindowPlan plan;
+  const int rc = make_window_plan(w, &plan);
+  if (rc == WPATTN_EUNSUPPORTED) {
+    // wide head dims: host-only evaluation
+    for (int p = 0; p < w->head_dim / 2; ++p) T_eff[p] = effective_threshold(w, p);
+    return WPATTN_OK;
+  }
+  if (rc != WPATTN_OK) return rc;
+  for (int p = 0; p < plan.P; ++p) T_eff[p] = plan.T[p];
+  return WPATTN_OK;
+}
+
+int wpattn_pruned_fraction(const wpattn_window* w, int64_t Nq, int64_t Nk, int64_t q_pos0,
+                           int64_t k_pos0, uint64_t* pruned_terms, uint64_t* total_terms,
+                           double* fraction) {
+  if (!w || Nq < 0 || Nk < 0) return WPATTN_EINVAL;
+  WindowPlan plan;
+  const int rc = make_window_plan(w, &plan);
+  if (rc != WPATTN_OK && rc != WPATTN_EUNSUPPORTED) return rc;
+  const int P = w->head_dim / 2;
+  // causal (query, key) pairs = kept terms of a pair whose threshold never binds
+  const unsigned __int128 causal = kept_terms_one_pair(kNoLimit, Nq, Nk, q_pos0, k_pos0);
+  unsigned __int128 kept = 0;
+  for (int p = 0; p < P; ++p) kept += kept_terms_one_pair(effective_threshold(w, p), Nq, Nk, q_pos0, k_pos0);
+  const unsigned __int128 total = causal * static_cast<unsigned __int128>(P);
+  const unsigned __int128 pruned = total - kept;
+  if ((total >> 64) != 0) return WPATTN_EUNSUPPORTED;  // beyond 64-bit counts
+  if (pruned_terms) *pruned_terms = static_cast<uint64_t>(pruned);
+  if (total_terms) *total_terms = static_cast<uint64_t>(total);
+  if (fraction) *fraction = total ? static_cast<double>(pruned) / static_cast<double>(total) : 0.0;
+  return WPATTN_OK;
+}
+
+int wpattn_prefill(const wpattn_window* w, const void* q, const void* k, const void* v, void* out,
+                   float* lse, int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
+                   int64_t q_pos0, int64_t k_pos0, float softmax_scale, void* cuda_stream) {
+  WindowPlan plan;
+  int rc = make_window_plan(w, &plan);
+  if (rc != WPATTN_OK) return rc;
+  if (B < 0 || Nq < 0 || Nk < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0) return WPATTN_EINVAL;
+  if (!(softmax_scale == softmax_scale)) return WPATTN_EINVAL;  // NaN
+  if (plan.D != 64 && plan.D != 128) return WPATTN_EUNSUPPORTED;
+  if (B == 0 || Nq == 0) return WPATTN_OK;
+  if (!q || !out || (Nk > 0 && (!k || !v))) return WPATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(out) || (Nk > 0 && (!aligned16(k) || !aligned16(v))))
+    return WPATTN_EINVAL;
+  // positions must keep every distance well inside int64
+  if (q_pos0 < 0 || k_pos0 < 0 || q_pos0 > (int64_t(1) << 60) || k_pos0 > (int64_t(1) << 60))
+    return WPATTN_EINVAL;
+  if (static_cast<int64_t>(B) * Hq > 65535LL * 65535LL || Hq > 65535 || B > 65535)
+    return WPATTN_EUNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
+
+  PrefillParams prm;
+  std::memset(&prm, 0, sizeof prm);
+  prm.out = static_cast<uint16_t*>(out);
+  prm.lse = lse;
+  prm.B = B; prm.Nq = Nq; prm.Nk = Nk; prm.Hq = Hq; prm.Hkv = Hkv; prm.G = Hq / Hkv;
+  prm.num_qtiles = (Nq + kBM - 1) / kBM;
+  prm.q_pos0 = q_pos0;
+  prm.k_pos0 = k_pos0;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(plan.D));
+  prm.scale_log2 = scale * 1.44269504088896340736f;
+  for (int p = 0; p < 64; ++p) prm.T[p] = plan.T[p];
+  const void* kk = Nk > 0 ? k : q;
+  const void* vv = Nk > 0 ? v : q;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (plan.D == 64) return launch_prefill<64>(q, kk, vv, prm, dev, st);
+  return launch_prefill<128>(q, kk, vv, prm, dev, st);
+}
+
+size_t wpattn_decode_workspace_size(const wpattn_window* w, int32_t B, int32_t Hq, int32_t Hkv,
+                                    int64_t max_kv_len) {
+  WindowPlan plan;
+  if (make_window_plan(w, &plan) != WPATTN_OK) return 0;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0 || max_kv_len <= 0) return 0;
+  return decode_workspace_bytes(B, Hq, plan.D, decode_max_splits(B, Hkv, max_kv_len));
+}
+
+int wpattn_decode(const wpattn_window* w, const void* q, const void* k_cache, const void* v_cache,
+                  const int32_t* kv_len_host, int64_t Lmax, int32_t B, int32_t Hq, int32_t Hkv,
+                  float softmax_scale, void* out, float* lse, void* workspace,
+                  size_t workspace_bytes, void* cuda_stream) {
+  WindowPlan plan;
+  int rc = make_window_plan(w, &plan);
+  if (rc != WPATTN_OK) return rc;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0 || Lmax <= 0) return WPATTN_EINVAL;
+  if (!(softmax_scale == softmax_scale)) return WPATTN_EINVAL;
+  if (!q || !k_cache || !v_cache || !kv_len_host || !out) return WPATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return WPATTN_EINVAL;
+  if (plan.D != 64 && plan.D != 128) return WPATTN_EUNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G > 16 || B > kDecodeMaxB || Lmax >= (int64_t(1) << 31)) return WPATTN_EUNSUPPORTED;
+  for (int b = 0; b < B; ++b)
+    if (kv_len_host[b] < 1 || kv_len_host[b] > Lmax) return WPATTN_EINVAL;
+  DeviceInfo* dev = nullptr;
+  if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
+  const int S = decode_splits(B, Hkv, Lmax, dev->num_sms);
+  const size_t need = decode_workspace_bytes(B, Hq, plan.D, S);
+  if (!workspace || workspace_bytes < need) return WPATTN_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return WPATTN_EINVAL;
+
+  DecodeParams prm;
+  std::memset(&prm, 0, sizeof prm);
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.k = static_cast<const uint16_t*>(k_cache);
+  prm.v = static_cast<const uint16_t*>(v_cache);
+  prm.part = static_cast<float*>(workspace);
+  prm.out = static_cast<uint16_t*>(out);
+  prm.lse = lse;
+  prm.Lmax = Lmax;
+  prm.B = B; prm.Hq = Hq; prm.Hkv = Hkv; prm.G = G; prm.S = S;
+  prm.hchunks = (G + 7) / 8;
+  const int gc = (G + prm.hchunks - 1) / prm.hchunks;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(plan.D));
+  prm.scale_log2 = scale * 1.44269504088896340736f;
+  for (int p = 0; p < 64; ++p) prm.T[p] = plan.T[p] > INT32_MAX ? INT32_MAX : static_cast<int>(plan.T[p]);
+  for (int b = 0; b < B; ++b) prm.kv_len[b] = kv_len_host[b];
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (plan.D == 64) return launch_decode<64>(prm, gc, st);
+  return launch_decode<128>(prm, gc, st);
+}
+
+int wpattn_device_status(void* cuda_stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return WPATTN_ECUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof v) != cudaSuccess) return WPATTN_ECUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof zero) != cudaSuccess) return WPATTN_ECUDA;
+  }
+  return v == 0 ? WPATTN_OK : v;
+}
+
+}  // extern "C"

@@ -1,0 +1,70 @@
+"""Shared helpers for the GPU parity tests: run the CUDA path through the
+C ABI, run the oracle on the same bf16 bytes, compare element by element."""
+import math
+
+import numpy as np
+import torch
+
+import oracle
+import rope_wavelength_sparsity_b200 as wp
+from rope_wavelength_sparsity_b200 import inputs
+
+# tolerances of the parity bar (out in bf16 units of the output, LSE in nats)
+ATOL_OUT = 1e-2
+ATOL_LSE = 2e-3
+
+
+def check_rows(o_gpu, l_gpu, o_ref, l_ref, what):
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    l_gpu = np.asarray(l_gpu, dtype=np.float64)
+    empty = np.isneginf(l_ref)
+    assert np.array_equal(np.isneginf(l_gpu), empty), f"{what}: empty-row mismatch"
+    if empty.any():
+        assert (o_gpu[empty] == 0).all(), f"{what}: empty rows must be 0"
+    ok = ~empty
+    d_out = float(np.abs(o_gpu[ok] - o_ref[ok]).max()) if ok.any() else 0.0
+    d_lse = float(np.abs(l_gpu[ok] - l_ref[ok]).max()) if ok.any() else 0.0
+    assert d_out <= ATOL_OUT and d_lse <= ATOL_LSE, f"{what}: max|dout|={d_out:.3e} max|dlse|={d_lse:.3e}"
+    return d_out, d_lse
+
+
+def prefill_parity(q, k, v, *, Hq, Hkv, D, base, alpha, g, q_pos0=0, k_pos0=0, rows=None,
+                   scale=None, what=""):
+    """q, k, v: bf16 tensors (any device).  Returns (max dout, max dlse)."""
+    dev = torch.device("cuda:0")
+    B, Nq = q.shape[0], q.shape[1]
+    scale = scale or 1.0 / math.sqrt(D)
+    win = wp.Window(D, base, alpha, g)
+    out, lse = wp.prefill(q.to(dev), k.to(dev), v.to(dev), win, q_pos0=q_pos0, k_pos0=k_pos0,
+                          scale=scale)
+    assert wp.device_status() == wp.OK
+    if rows is None:
+        rows = [(b, h, t) for b in range(B) for h in range(Hq) for t in range(Nq)]
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
+    o_ref, l_ref = oracle.attention_rows(inputs.bits(q), inputs.bits(k), inputs.bits(v), Hq=Hq,
+                                         Hkv=Hkv, q_pos0=q_pos0, k_pos0=k_pos0, base=base,
+                                         alpha=alpha, g=g, scale=scale, rows=rows)
+    bi, hi, ti = (torch.as_tensor(rows[:, i]) for i in range(3))
+    o_gpu = out.float().cpu()[bi, ti, hi].numpy()
+    l_gpu = lse.cpu()[bi, hi, ti].numpy()
+    return check_rows(o_gpu, l_gpu, o_ref, l_ref, what)
+
+
+def decode_parity(q, kc, vc, kv_len, *, Hq, Hkv, D, base, alpha, g, rows=None, scale=None,
+                  what=""):
+    dev = torch.device("cuda:0")
+    B = q.shape[0]
+    scale = scale or 1.0 / math.sqrt(D)
+    win = wp.Window(D, base, alpha, g)
+    kv_len = [int(x) for x in kv_len]
+    out, lse = wp.decode(q.to(dev), kc.to(dev), vc.to(dev), kv_len, win, scale=scale)
+    assert wp.device_status() == wp.OK
+    if rows is None:
+        rows = [(b, h) for b in range(B) for h in range(Hq)]
+    o_ref, l_ref = oracle.decode_rows(inputs.bits(q), inputs.bits(kc), inputs.bits(vc), kv_len,
+                                      Hq=Hq, Hkv=Hkv, base=base, alpha=alpha, g=g, scale=scale,
+                                      rows=rows)
+    oc, lc = out.float().cpu(), lse.cpu()
+    o_gpu = np.stack([oc[b, h].numpy() for (b, h) in rows])
+    l_gpu = np.array([float(lc[b, h]) for (b, h) in rows])
+    return check_rows(o_gpu, l_gpu, o_ref, l_ref, what)
