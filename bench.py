@@ -1,0 +1,500 @@
+"""Benchmark of per-RoPE-wavelength windowed attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one pass of the hot path over one batch of synthetic input:
+the host planner (thresholds, tile plan) and the windowed prefill kernel of
+the chosen workload, called through the C ABI.  The default workload is the
+Qwen2.5-0.5B-shaped single-layer prefill (B=1, Hq=14, Hkv=2, D=64, N=32768,
+base 1e6, alpha 1, g = 8 pairs).  The same run also times the Llama-3.2-3B-
+shaped decode step (B=16, Hq=24, Hkv=8, D=128, L=131072) for the decode
+KV GB/s half of the metric, and the same kernels with the window off.
+
+Metric: effective TFLOP/s = (4 * kept QK pair-terms + 2 * D * causal
+(query, key) pairs) per (batch, query head), over the device time of the
+step; decode: algorithmic GB/s = K bytes of the kept pairs + all V bytes
+(+ q and out) over the decode call's device time.
+
+Timing: CUDA events on the launching stream around every step, an L2 flush
+(a 512 MiB write) between steps outside the events, W warm-up steps, barrier
++ synchronize around the timed region, max over ranks.  Multi-GPU: every rank
+runs its own independent problem (weak scaling, no data-path collective).
+
+``--impl reference`` times the oracle (the plain CPU definition) on a bounded
+sample of rows of the same workload, in the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "effective TFLOP/s (kept QK terms + PV) and decode KV GB/s, % of B200 roofline"
+DEFAULT_WORKLOAD = "qwen2.5-0.5b-32k"
+DECODE_WORKLOAD = "llama3.2-3b-decode-128k"
+FLUSH_BYTES = 512 << 20
+
+# DRAM bytes (read + write) per launch of the dominant kernel from one ncu
+# capture, keyed by the sha256 of the kernel sources at capture time; a
+# changed kernel reports null until it is captured again.
+NCU_TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rope_wavelength_sparsity_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            pk = json.load(fh)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk.get("bf16_tflops_sustained"), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ----------------------------------------------------------- work accounting
+def prefill_flops(w, win, wp):
+    """(effective FLOPs, window-off FLOPs) of one prefill of workload w."""
+    pruned, total, _ = wp.pruned_fraction(win, w.Nq, w.Nk, w.q_pos0, w.k_pos0)
+    P = w.D // 2
+    causal = total // P
+    kept = total - pruned
+    per_head = 4 * kept + 2 * w.D * causal
+    off = 4 * w.D * causal
+    return w.B * w.Hq * per_head, w.B * w.Hq * off
+
+
+def decode_bytes(w, win, wp, kv_len):
+    """(algorithmic bytes, window-off bytes) of one decode step."""
+    P = w.D // 2
+    kbytes = vbytes = kfull = 0
+    for L in kv_len:
+        pruned, total, _ = wp.pruned_fraction(win, 1, L, L - 1, 0)
+        kept = total - pruned
+        kbytes += kept * 2 * 2 * w.Hkv
+        kfull += total * 2 * 2 * w.Hkv
+        vbytes += L * w.D * 2 * w.Hkv
+    io = w.B * w.Hq * w.D * 2 * 2 + w.B * w.Hq * 4
+    return kbytes + vbytes + io, kfull + vbytes + io
+
+
+def row_flops(w, win, wp, t):
+    pruned, total, _ = wp.pruned_fraction(win, 1, w.Nk, w.q_pos0 + t, w.k_pos0)
+    P = w.D // 2
+    return 4 * (total - pruned) + 2 * w.D * (total // P)
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU arm
+def _dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def time_steps(step, n_warm, n_steps, flush, world, clocks=None, per_step_events=True):
+    """Device time (ms) of n_steps calls of step(); L2 flushed before each."""
+    import torch
+    for _ in range(n_warm):
+        flush()
+        step()
+    _barrier(world)
+    if clocks:
+        clocks.start()
+        time.sleep(0.25)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(n_steps)]
+    for i in range(n_steps):
+        flush()
+        starts[i].record()
+        step()
+        ends[i].record()
+    _barrier(world)
+    clk = clocks.stop() if clocks else None
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total = sum(per)
+    return _max_over_ranks(total, world), per, clk
+
+
+def gpu_arm(args):
+    import torch
+    import rope_wavelength_sparsity_b200 as wp
+    from rope_wavelength_sparsity_b200 import inputs
+
+    world, rank, local = _dist_setup(args)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    peaks = load_peaks()
+    w = inputs.WORKLOADS[args.workload]
+    win = wp.Window(w.D, w.base, w.alpha, w.g)
+    win_off = wp.Window(w.D, w.base, float("inf"), w.g)
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    result = {}
+    if w.kind == "prefill":
+        q, k, v, _ = inputs.prefill_inputs(w, seed=rank, device=dev)
+        out = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+        eff, off_flops = prefill_flops(w, win, wp)
+
+        def step():
+            wp.prefill(q, k, v, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale, out=out,
+                       lse=lse)
+
+        def step_off():
+            wp.prefill(q, k, v, win_off, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale, out=out,
+                       lse=lse)
+
+        clocks = ClockSampler(dev.index) if rank == 0 else None
+        total_ms, per, clk = time_steps(step, args.warmup, args.steps, flush, world, clocks)
+        if wp.device_status() != wp.OK:
+            raise RuntimeError("kernel status: timeout")
+        off_ms, _, _ = time_steps(step_off, args.warmup, max(3, args.steps // 4), flush, world)
+        off_ms_step = off_ms / max(3, args.steps // 4)
+        ms_step = total_ms / args.steps
+        value = world * eff / (ms_step * 1e-3) / 1e12
+        kernel_ms = statistics.mean(per)
+        achieved = eff / (kernel_ms * 1e-3) / 1e12
+        traffic = NCU_TRAFFIC.get((args.workload, kernel_source_hash()))
+        result.update({
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms_step, 4),
+            "dtype": "bf16",
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2),
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(achieved / peaks["bf16_tflops"], 4),
+                         "traffic": traffic,
+                         "peak_source": f"{peaks['source']} bf16 dense (burst)"},
+            "window_off": {"ms_per_step": round(off_ms_step, 4),
+                           "speedup": round(off_ms_step / ms_step, 3),
+                           "ideal_speedup": round(off_flops / eff, 3),
+                           "effective_tflops_at_window_off_time": round(eff / (off_ms_step * 1e-3) / 1e12, 2)},
+            "work": {"effective_tflop_per_step": round(world * eff / 1e12, 4),
+                     "window_off_tflop_per_step": round(world * off_flops / 1e12, 4),
+                     "pruned_fraction": wp.pruned_fraction(win, w.Nq, w.Nk, w.q_pos0, w.k_pos0)[2]},
+            "gpu_launches": args.steps,
+            "clocks": clk,
+        })
+        # end to end through the public API with pinned host buffers
+        qh = q.cpu().pin_memory()
+        kh = k.cpu().pin_memory()
+        vh = v.cpu().pin_memory()
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def step_e2e():
+            qd = q.copy_(qh, non_blocking=True)
+            kd = k.copy_(kh, non_blocking=True)
+            vd = v.copy_(vh, non_blocking=True)
+            o, _ = wp.prefill(qd, kd, vd, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale,
+                              out=out, lse=lse)
+            oh.copy_(o, non_blocking=True)
+
+        n_e2e = max(5, args.steps // 4)
+        e2e_ms, _, _ = time_steps(step_e2e, 2, n_e2e, flush, world)
+        h2d = (q.numel() + k.numel() + v.numel()) * 2
+        result["e2e"] = {"value": round(world * eff / (e2e_ms / n_e2e * 1e-3) / 1e12, 2),
+                         "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                         "d2h_bytes_per_step": out.numel() * 2}
+        result["config"] = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                            "Nq": w.Nq, "Nk": w.Nk, "q_pos0": w.q_pos0, "rope_base": w.base,
+                            "alpha": w.alpha, "group_pairs": w.g, "global_batch": w.B * world,
+                            "seq_len": w.Nk, "parallelism": f"independent problem per GPU x{world}",
+                            "l2": "flushed between steps (512 MiB write)"}
+        del q, k, v, out, lse, qh, kh, vh, oh
+        torch.cuda.empty_cache()
+    if w.kind == "decode" or (args.workload == DEFAULT_WORKLOAD and not args.only_primary):
+        wd = w if w.kind == "decode" else inputs.WORKLOADS[DECODE_WORKLOAD]
+        dres = bench_decode(wd, args, world, rank, dev, flush, peaks,
+                            primary=(w.kind == "decode"))
+        if w.kind == "decode":
+            result.update(dres)
+        else:
+            result["decode"] = dres
+    result.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                   "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                   "data": "synthetic (seeded N(0,1) bf16; pair magnitudes / planted key per workload)"})
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, time_budget_s=args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return rank, result
+
+
+def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
+    import torch
+    import rope_wavelength_sparsity_b200 as wp
+    from rope_wavelength_sparsity_b200 import inputs
+    win = wp.Window(w.D, w.base, w.alpha, w.g)
+    win_off = wp.Window(w.D, w.base, float("inf"), w.g)
+    q, kc, vc, kv_len = inputs.decode_inputs(w, seed=rank, device=dev)
+    kv_len = [int(x) for x in kv_len]
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(wp.decode_workspace_size(win, w.B, w.Hq, w.Hkv, w.Nk), dtype=torch.uint8,
+                     device=dev)
+    alg, off_bytes = decode_bytes(w, win, wp, kv_len)
+
+    def step():
+        wp.decode(q, kc, vc, kv_len, win, scale=w.scale, out=out, lse=lse, workspace=ws)
+
+    def step_off():
+        wp.decode(q, kc, vc, kv_len, win_off, scale=w.scale, out=out, lse=lse, workspace=ws)
+
+    steps = args.steps
+    clocks = ClockSampler(dev.index) if (rank == 0 and primary) else None
+    total_ms, per, clk = time_steps(step, args.warmup, steps, flush, world, clocks)
+    if wp.device_status() != wp.OK:
+        raise RuntimeError("decode kernel status: timeout")
+    off_ms, _, _ = time_steps(step_off, args.warmup, max(3, steps // 4), flush, world)
+    ms = total_ms / steps
+    off_step = off_ms / max(3, steps // 4)
+    achieved = alg / (statistics.mean(per) * 1e-3) / 1e9
+    res = {
+        "metric": METRIC, "value": round(world * alg / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "ms_per_step": round(ms, 4), "dtype": "bf16",
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": NCU_TRAFFIC.get((w.name, kernel_source_hash())),
+                     "peak_source": f"{peaks['source']} HBM copy",
+                     "timed": "split + combine kernels (one decode call)"},
+        "window_off": {"ms_per_step": round(off_step, 4), "speedup": round(off_step / ms, 3),
+                       "ideal_speedup": round(off_bytes / alg, 3)},
+        "work": {"algorithmic_bytes_per_step": alg * world, "window_off_bytes_per_step": off_bytes * world},
+        "gpu_launches": 2 * steps,
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.Nk,
+                   "rope_base": w.base, "alpha": w.alpha, "group_pairs": w.g,
+                   "global_batch": w.B * world, "seq_len": w.Nk,
+                   "parallelism": f"independent problem per GPU x{world}",
+                   "l2": "flushed between steps (512 MiB write)"},
+    }
+    if primary:
+        res["clocks"] = clk
+        qh = q.cpu().pin_memory()
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def step_e2e():
+            qd = q.copy_(qh, non_blocking=True)
+            o, _ = wp.decode(qd, kc, vc, kv_len, win, scale=w.scale, out=out, lse=lse, workspace=ws)
+            oh.copy_(o, non_blocking=True)
+
+        n_e2e = max(5, steps // 4)
+        e2e_ms, _, _ = time_steps(step_e2e, 2, n_e2e, flush, world)
+        res["e2e"] = {"value": round(world * alg / (e2e_ms / n_e2e * 1e-3) / 1e9, 1), "unit": "GB/s",
+                      "h2d_bytes_per_step": q.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
+                      "note": "the KV cache is resident on the device, as in serving"}
+    del q, kc, vc, out, lse, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+# --------------------------------------------------------- oracle (CPU) arm
+def oracle_sample(w, n_rows, seed=0):
+    """Query rows spread over heads and positions, and the inputs to run them."""
+    import numpy as np
+    from rope_wavelength_sparsity_b200 import inputs
+    rng = np.random.default_rng(seed)
+    rows = []
+    if w.kind == "prefill":
+        for i in range(n_rows):
+            h = i % w.Hq
+            t = int(rng.integers(0, w.Nq))
+            rows.append((0, h, t))
+    else:
+        for i in range(n_rows):
+            rows.append((i % w.B, (i * 7) % w.Hq))
+    return rows
+
+
+def cpu_baseline(w, time_budget_s=15.0):
+    """Time the oracle on a bounded sample of the workload (one host thread)."""
+    import torch
+    import oracle
+    import rope_wavelength_sparsity_b200 as wp
+    from rope_wavelength_sparsity_b200 import inputs
+    win = wp.Window(w.D, w.base, w.alpha, w.g)
+    if w.kind == "prefill":
+        q, k, v, _ = inputs.prefill_inputs(w, seed=0, device="cuda" if torch.cuda.is_available() else "cpu")
+        qb, kb, vb = inputs.bits(q), inputs.bits(k), inputs.bits(v)
+        rows = oracle_sample(w, 4096)
+        done, flops, t0 = 0, 0, time.perf_counter()
+        while done < len(rows) and time.perf_counter() - t0 < time_budget_s:
+            b, h, t = rows[done]
+            oracle.attention_rows(qb, kb, vb, Hq=w.Hq, Hkv=w.Hkv, q_pos0=w.q_pos0, k_pos0=w.k_pos0,
+                                  base=w.base, alpha=w.alpha, g=w.g, scale=w.scale, rows=[(b, h, t)])
+            flops += row_flops(w, win, wp, t)
+            done += 1
+        dt = time.perf_counter() - t0
+        return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+                "kind": "oracle",
+                "sample": f"{done} query rows (random heads/positions) of {w.name}, {dt:.1f} s, "
+                          "effective FLOPs of those rows / wall time"}
+    q, kc, vc, kv_len = inputs.decode_inputs(w, seed=0, device="cuda" if torch.cuda.is_available() else "cpu")
+    qb, kb, vb = inputs.bits(q), inputs.bits(kc), inputs.bits(vc)
+    kv_len = [int(x) for x in kv_len]
+    rows = oracle_sample(w, 1024)
+    done, nbytes, t0 = 0, 0, time.perf_counter()
+    P = w.D // 2
+    while done < len(rows) and time.perf_counter() - t0 < time_budget_s:
+        b, h = rows[done]
+        oracle.decode_rows(qb, kb, vb, kv_len, Hq=w.Hq, Hkv=w.Hkv, base=w.base, alpha=w.alpha,
+                           g=w.g, scale=w.scale, rows=[(b, h)])
+        pruned, total, _ = wp.pruned_fraction(win, 1, kv_len[b], kv_len[b] - 1, 0)
+        # one (sequence, kv head) worth of bytes is shared by the G heads of the group
+        nbytes += ((total - pruned) * 4 + kv_len[b] * w.D * 2) / (w.Hq // w.Hkv)
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} (sequence, head) rows of {w.name}, {dt:.1f} s, algorithmic bytes "
+                      "of those rows (per-head share of the group's K/V) / wall time"}
+
+
+def reference_arm(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return rank, None
+    from rope_wavelength_sparsity_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    per_step = max(0.2, 90.0 / max(1, args.steps + args.warmup))
+    vals = []
+    cb = None
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(w, time_budget_s=per_step)
+        if i >= args.warmup:
+            vals.append(cb["value"])
+    value = statistics.mean(vals) if vals else cb["value"]
+    unit = cb["unit"]
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name},
+           "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
+                            "sample": f"each step: {cb['sample']}"},
+           "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return rank, out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only-primary", action="store_true",
+                    help="skip the secondary decode measurement of the default workload")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank, res = reference_arm(args)
+    else:
+        rank, res = gpu_arm(args)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -107,7 +107,7 @@ int launch_prefill(const void* q, const void* k, const void* v, const PrefillPar
       return WPATTN_ECUDA;
     dev->prefill_attr[slot] = true;
   }
-  dim3 grid(prm.num_qtiles, prm.Hq, prm.B);
+  dim3 grid(prm.num_ctas_q, prm.Hq, prm.B);
   prefill_kernel<D><<<grid, kPrefillThreads, smem, st>>>(tq, tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
@@ -226,11 +226,12 @@ int wpattn_prefill(const wpattn_window* w, const void* q, const void* k, const v
   prm.out = static_cast<uint16_t*>(out);
   prm.lse = lse;
   prm.B = B; prm.Nq = Nq; prm.Nk = Nk; prm.Hq = Hq; prm.Hkv = Hkv; prm.G = Hq / Hkv;
-  prm.num_qtiles = (Nq + kBM - 1) / kBM;
+  prm.num_ctas_q = (Nq + kQT * kBM - 1) / (kQT * kBM);
   prm.q_pos0 = q_pos0;
   prm.k_pos0 = k_pos0;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(plan.D));
   prm.scale_log2 = scale * 1.44269504088896340736f;
+  prm.g8 = plan.g == 8 ? 1 : 0;
   for (int p = 0; p < 64; ++p) prm.T[p] = plan.T[p];
   const void* kk = Nk > 0 ? k : q;
   const void* vv = Nk > 0 ? v : q;

@@ -84,8 +84,11 @@ decode_split_kernel(const __grid_constant__ DecodeParams p) {
   const int c = lane % TPK;               // head-dim chunk [8c, 8c+8)
   const int slot = warp * KPW + lane / TPK;
   const int pb = (c % HALF) * 8;          // first pair of this chunk
-  const int T_first = p.T[pb];
-  const int T_last = p.T[pb + 7];
+  int Tc[8];  // thresholds of this chunk's 8 pairs
+#pragma unroll
+  for (int e = 0; e < 8; ++e) Tc[e] = p.T[pb + e];
+  const int T_first = Tc[0];
+  const int T_last = Tc[7];
 
   float qf[GC][8];
 #pragma unroll
@@ -128,14 +131,16 @@ decode_split_kernel(const __grid_constant__ DecodeParams p) {
       vraw[u] = valid[u] ? ldg_stream(vbase + (size_t)j * row_stride) : make_uint4(0, 0, 0, 0);
     }
     float s[U][GC];
+    float vf[U][8];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
+      unpack8(vraw[u], vf[u]);
       float kf[8];
       unpack8(kraw[u], kf);
       if (dist[u] > T_first) {  // chunk only partly kept at this distance
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          if (dist[u] > p.T[pb + e]) kf[e] = 0.f;
+          if (dist[u] > Tc[e]) kf[e] = 0.f;
       }
 #pragma unroll
       for (int hh = 0; hh < GC; ++hh) {
@@ -160,11 +165,9 @@ decode_split_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const float pu = ex2_approx(s[u][hh] - mx);
-        float vf[8];
-        unpack8(vraw[u], vf);
         l[hh] += pu;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[hh][e] = fmaf(pu, vf[e], o[hh][e]);
+        for (int e = 0; e < 8; ++e) o[hh][e] = fmaf(pu, vf[u][e], o[hh][e]);
       }
       m[hh] = mx;
     }

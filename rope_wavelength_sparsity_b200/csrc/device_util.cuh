@@ -49,14 +49,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                ::"r"(bar), "r"(bytes) : "memory");
 }
 
+// One bounded try: the thread may sleep in the hardware until the phase
+// completes or the hint (nanoseconds) expires, instead of spinning.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }
@@ -65,14 +67,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
-  while (true) {
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+  while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       record_status(4 /* WPATTN_ETIMEOUT */);
       return false;
     }
   }
+  return true;
 }
 
 // ---------------------------------------------------------------- TMA loads
@@ -131,9 +132,9 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
       : "memory");
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
-  uint32_t* u = reinterpret_cast<uint32_t*>(r);
+// 32 consecutive 32-bit columns of this thread's TMEM lane (r[0..31]).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* r) {
+  uint32_t u[32];
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
       "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
@@ -144,10 +145,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
         "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]), "=r"(u[25]),
         "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
       : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&r)[32]) {
-  const uint32_t* u = reinterpret_cast<const uint32_t*>(r);
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* u) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
       "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
@@ -158,6 +160,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&r)[32]) 
       "r"(u[22]), "r"(u[23]), "r"(u[24]), "r"(u[25]), "r"(u[26]), "r"(u[27]), "r"(u[28]),
       "r"(u[29]), "r"(u[30]), "r"(u[31])
       : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* r) {
+  uint32_t u[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(r[i]);
+  tmem_st32u(taddr, u);
 }
 
 __device__ __forceinline__ void tmem_ld_wait() {
@@ -195,6 +204,16 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int a_mn, i
          | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Register reallocation between warpgroups (all 4 warps of a warpgroup run it).
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------ small math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -206,6 +225,62 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Packed fp32 pairs (Blackwell f32x2 FMA-pipe instructions): d = a*b + c, d = a + b.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// 2^x for a pair, on the FMA and integer pipes instead of the MUFU unit.
+// Range reduction x = n + f with n = round(x), f in [-1/2, 1/2]: adding
+// 1.5 * 2^23 leaves n in the low mantissa bits of y, so n is exact, and
+// ((bits(y) + 127) << 23) is the float 2^n (0.0 when n = -127).  2^f is a
+// degree-3 polynomial fitted for minimum maximum relative error on
+// [-1/2, 1/2] (Lawson's iteratively reweighted least squares, our own fit);
+// with fp32 Horner evaluation its relative error stays below 8e-5.  Inputs
+// are clamped to -127, so -inf (a masked score) gives exactly 0.
+__device__ __forceinline__ void exp2_poly2(float& r0, float& r1, float x0, float x1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261117f, c3 = 0.05517166f;
+  x0 = fmaxf(x0, -127.f);
+  x1 = fmaxf(x1, -127.f);
+  float y0, y1, n0, n1, f0, f1;
+  add2(y0, y1, x0, x1, kShift, kShift);
+  add2(n0, n1, y0, y1, -kShift, -kShift);
+  add2(f0, f1, x0, x1, -n0, -n1);
+  float p0, p1;
+  fma2(p0, p1, c3, c3, f0, f1, c2, c2);
+  fma2(p0, p1, p0, p1, f0, f1, c1, c1);
+  fma2(p0, p1, p0, p1, f0, f1, c0, c0);
+  const float s0 = __uint_as_float((__float_as_uint(y0) + 127u) << 23);
+  const float s1 = __uint_as_float((__float_as_uint(y1) + 127u) << 23);
+  mul2(r0, r1, p0, p1, s0, s1);
 }
 
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }

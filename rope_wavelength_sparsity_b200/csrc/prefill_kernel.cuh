@@ -6,16 +6,19 @@
 // are grouped in blocks of 16 so the pruned contraction still runs on the
 // Tensor Cores.
 //
-// One CTA owns 128 query rows of one (batch, query head) and walks the key
-// tiles from the diagonal outwards.  Warp roles:
-//   warps 0-3  softmax: row r of the tile is TMEM lane r; they read S from
-//              TMEM, subtract the pairs that are pruned at some but not all
-//              of the tile's distances, mask, run the online softmax with a
-//              lazily rescaled O, write P (bf16) to shared memory and finish
-//              with O / l.
-//   warp 4     TMA producer: Q once, then K and V tiles into a ring.
-//   warp 5     MMA issuer (one lane): S = Q K^T over the active k-steps, then
-//              O += P V; owns the TMEM allocation.
+// One CTA owns two 128-row query tiles (256 consecutive rows) of one
+// (batch, query head); both walk the same key tiles from the diagonal
+// outwards, so every K and V tile is loaded once for 256 rows.  Warp roles:
+//   warps 0-3, 4-7  softmax of query tile 0 / 1: row r of a tile is TMEM lane
+//              r.  They read S from TMEM, subtract the pairs that are pruned
+//              at some but not all distances of the tile, mask, run the
+//              online softmax with a lazily rescaled O, write P (bf16) back
+//              into TMEM over S, and finish with O / l.  The two groups
+//              alternate with the tensor core (ping-pong).
+//   warp 8     TMA producer: both Q tiles once, then K and V tiles into a ring.
+//   warp 9     MMA issuer (one lane): S_t = Q_t K^T over the active k-steps,
+//              O_t += P_t V with P_t read from TMEM; owns the TMEM allocation.
+//   warps 10-11 idle (they complete warpgroup 2 for the register hand-over).
 //
 // Shared-memory layouts.  Q and K use the no-swizzle canonical K-major layout
 // with one 16-byte column panel per 8 head dims: panel c holds dims
@@ -25,45 +28,55 @@
 // halves of pairs 8m..8m+7) with panel D/16 + m (their second halves): every
 // k-step carries 8 whole RoPE pairs, and skipping steps below k0 drops exactly
 // the pairs 0 .. 8*k0 - 1.  V uses the 128-byte-swizzled MN-major layout
-// (64-dim panels of 128 keys), P the same no-swizzle K-major layout as Q.
+// (64-dim panels of 128 keys).
 //
-// TMEM columns: S double buffer at [0,128) and [128,256), O at [256, 256+D).
+// TMEM columns: S_0 / P_0 at [0,128), S_1 / P_1 at [128,256), O_0 at
+// [256, 256+D), O_1 at [256+D, 256+2D).  P_t (bf16 pairs) overwrites the
+// first 64 columns of S_t; the next QK of tile t is issued after PV_t, and
+// tcgen05 MMAs of one thread run in issue order.
 #pragma once
 
 #include "device_util.cuh"
 
 namespace wpattn {
 
-constexpr int kBM = 128;              // query rows per CTA
+constexpr int kBM = 128;              // query rows per tile (TMEM lanes)
 constexpr int kBN = 128;              // keys per tile
-constexpr int kPrefillThreads = 192;  // 4 softmax warps + producer + MMA
+constexpr int kQT = 2;                // query tiles per CTA
+constexpr int kPrefillThreads = 384;  // 8 softmax warps + producer + MMA + 2 idle
+// Registers: launched at 168 per thread (384 x 168 = 64512); the softmax
+// warpgroups grow to 224 and warpgroup 2 (producer, MMA, idle) shrinks to 56:
+// 256 x 224 + 128 x 56 = 64512.
+constexpr uint32_t kRegsSoftmax = 224;
+constexpr uint32_t kRegsOther = 56;
 
 struct PrefillParams {
   uint16_t* out;      // [B, Nq, Hq, D] bf16
   float* lse;         // [B, Hq, Nq] or null
   int B, Nq, Nk, Hq, Hkv, G;
-  int num_qtiles;
+  int num_ctas_q;     // CTAs along the query axis (256 rows each)
   int64_t q_pos0, k_pos0;
   float scale_log2;   // softmax scale * log2(e)
+  int g8;             // 1: pairs share thresholds in groups of 8
   int64_t T[64];      // per-pair thresholds (nondecreasing)
 };
 
 template <int D>
 struct PrefillSmem {
-  static constexpr int NS = (D == 64) ? 3 : 2;       // K/V ring depth
+  static constexpr int NS = (D == 64) ? 4 : 2;       // K/V ring depth
+  static constexpr int NPOLY = 0;                    // of every 8 column pairs, exp2 on the FMA pipe
   static constexpr int TILE = kBM * D * 2;           // one Q, K or V tile in bytes
-  static constexpr int PBUF = kBM * kBN * 2;         // one P tile
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + TILE;
+  static constexpr int OFF_K = OFF_Q + kQT * TILE;
   static constexpr int OFF_V = OFF_K + NS * TILE;
-  static constexpr int OFF_P = OFF_V + NS * TILE;
-  static constexpr int OFF_BAR = OFF_P + 2 * PBUF;
+  static constexpr int OFF_QM = OFF_V + NS * TILE;        // masked first k-step of Q, per tile
+  static constexpr int OFF_BAR = OFF_QM + kQT * 2 * kBM * 16;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
-  //           s_full[2], s_free[2], p_full[2], pv_done[2]
+  //           s_full[2], p_full[2], o_final[2], qm_init[2]
   static constexpr int NBAR = 1 + 4 * NS + 8;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_TMEM + 16;
-  static constexpr int ALLOC = BYTES + 1024;          // slack for 1024-byte alignment
+  static constexpr int ALLOC = BYTES;
 };
 
 __device__ __forceinline__ int dev_pmin(const int64_t* T, int P, int64_t d) {
@@ -75,6 +88,15 @@ __device__ __forceinline__ int dev_pmin(const int64_t* T, int P, int64_t d) {
   return lo;
 }
 
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 template <int D>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -84,68 +106,76 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   constexpr int P = D / 2;
   constexpr int KS = D / 16;          // k-steps of the QK contraction (8 pairs each)
   constexpr int PANEL = kBM * 16;     // bytes of one 8-dim column panel
-  constexpr uint32_t TMEM_S = 0, TMEM_O = 256;
+  constexpr uint32_t TMEM_O = 256;
+  constexpr uint32_t FULL = 0xffffffffu;
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + L::OFF_Q;
   const uint32_t sK = sbase + L::OFF_K;
   const uint32_t sV = sbase + L::OFF_V;
-  const uint32_t sP = sbase + L::OFF_P;
   const uint32_t bar = sbase + L::OFF_BAR;
   const uint32_t q_full = bar;
   auto k_full = [&](int s) { return bar + 8 * (1 + s); };
   auto k_empty = [&](int s) { return bar + 8 * (1 + NS + s); };
   auto v_full = [&](int s) { return bar + 8 * (1 + 2 * NS + s); };
   auto v_empty = [&](int s) { return bar + 8 * (1 + 3 * NS + s); };
-  auto s_full = [&](int b) { return bar + 8 * (1 + 4 * NS + b); };
-  auto s_free = [&](int b) { return bar + 8 * (3 + 4 * NS + b); };
-  auto p_full = [&](int b) { return bar + 8 * (5 + 4 * NS + b); };
-  auto pv_done = [&](int b) { return bar + 8 * (7 + 4 * NS + b); };
+  auto s_full = [&](int t) { return bar + 8 * (1 + 4 * NS + t); };
+  auto p_full = [&](int t) { return bar + 8 * (3 + 4 * NS + t); };
+  auto o_final = [&](int t) { return bar + 8 * (5 + 4 * NS + t); };
+  auto qm_init = [&](int t) { return bar + 8 * (7 + 4 * NS + t); };
+  const uint32_t sQM = sbase + L::OFF_QM;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
 
+  // the 128-byte-swizzled V tiles need a 1024-byte aligned shared window
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) record_status(2 /* WPATTN_EUNSUPPORTED */);
+    return;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = p.num_qtiles - 1 - blockIdx.x;  // longest rows first
+  const int cq = p.num_ctas_q - 1 - blockIdx.x;  // longest rows first
   const int h = blockIdx.y, b = blockIdx.z;
   const int kvh = h / p.G;
-
-  // key tiles this query tile sees: keys at positions <= its last row
-  const int64_t i_min = p.q_pos0 + (int64_t)kBM * qt;
-  const int64_t i_max = p.q_pos0 + (int64_t)min(kBM * qt + kBM - 1, p.Nq - 1);
   const int nkt = (p.Nk + kBN - 1) / kBN;
-  int n_tiles = 0;
-  int kt_last = -1;
-  if (i_max >= p.k_pos0 && p.Nk > 0) {
+
+  // key tiles of query tile t: positions <= its last row, iterated from kt_top down
+  auto last_key_tile = [&](int t) -> int {
+    const int row0 = (kQT * cq + t) * kBM;
+    if (row0 >= p.Nq || p.Nk <= 0) return -1;
+    const int64_t i_max = p.q_pos0 + min(row0 + kBM - 1, p.Nq - 1);
+    if (i_max < p.k_pos0) return -1;
     const int64_t last = (i_max - p.k_pos0) / kBN;
-    kt_last = (int)(last < (int64_t)(nkt - 1) ? last : (int64_t)(nkt - 1));
-    n_tiles = kt_last + 1;
-  }
-  // first active k-step of tile j: pairs active at the tile's smallest distance
-  auto tile_k0 = [&](int j) -> int {
-    const int64_t kp0 = p.k_pos0 + (int64_t)kBN * (kt_last - j);
-    int64_t dlo = i_min - (kp0 + kBN - 1);
+    return (int)(last < (int64_t)(nkt - 1) ? last : (int64_t)(nkt - 1));
+  };
+  const int kt_last0 = last_key_tile(0), kt_last1 = last_key_tile(1);
+  const int kt_top = max(kt_last0, kt_last1);
+  const int n_iter = kt_top + 1;  // shared K/V iterations j: key tile kt_top - j
+  // first pair of query tile t that is kept somewhere in key tile kt: pairs
+  // below it are pruned at the tile's smallest distance, hence everywhere
+  auto tile_plo = [&](int t, int kt) -> int {
+    const int64_t i_min = p.q_pos0 + (int64_t)(kQT * cq + t) * kBM;
+    int64_t dlo = i_min - (p.k_pos0 + (int64_t)kBN * kt + kBN - 1);
     if (dlo < 0) dlo = 0;
-    return dev_pmin(p.T, P, dlo) / 8;
+    return dev_pmin(p.T, P, dlo);
   };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(k_full(s), 1);
-      mbar_init(k_empty(s), 5);  // MMA commit + 4 softmax warps (they read K for corrections)
+      mbar_init(k_empty(s), 1 + 8);  // MMA commit + 8 softmax warps (they read K for corrections)
       mbar_init(v_full(s), 1);
       mbar_init(v_empty(s), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full(i), 1);
-      mbar_init(s_free(i), 4);
-      mbar_init(p_full(i), 4);
-      mbar_init(pv_done(i), 1);
+    for (int t = 0; t < kQT; ++t) {
+      mbar_init(s_full(t), 1);
+      mbar_init(p_full(t), 4);
+      mbar_init(o_final(t), 1);
+      mbar_init(qm_init(t), 4);
     }
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -154,17 +184,23 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp >= 8) {
+  regs_decrease<kRegsOther>();
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0 && n_iter > 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      mbar_arrive_expect_tx(q_full, L::TILE);
-      for (int c = 0; c < D / 8; ++c)
-        tma_load_4d(sQ + c * PANEL, &tmQ, q_full, 8 * c, kBM * qt, h, b);
-      for (int j = 0; j < n_tiles; ++j) {
-        const int kt = kt_last - j;
+      // a query tile wholly past Nq is not loaded (its rows are never used)
+      int nq_tiles = 0;
+      for (int t = 0; t < kQT; ++t) nq_tiles += ((kQT * cq + t) * kBM < p.Nq) ? 1 : 0;
+      mbar_arrive_expect_tx(q_full, nq_tiles * L::TILE);
+      for (int t = 0; t < nq_tiles; ++t)
+        for (int c = 0; c < D / 8; ++c)
+          tma_load_4d(sQ + t * L::TILE + c * PANEL, &tmQ, q_full, 8 * c, (kQT * cq + t) * kBM, h, b);
+      for (int j = 0; j < n_iter; ++j) {
+        const int kt = kt_top - j;
         const int s = j % NS;
         const uint32_t ph = (j / NS) & 1;
         if (j >= NS && !mbar_wait(k_empty(s), ph ^ 1)) break;
@@ -177,202 +213,353 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tma_load_4d(sV + s * L::TILE + c * (kBN * 128), &tmV, v_full(s), 64 * c, kBN * kt, kvh, b);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0 && n_iter > 0) {
       constexpr uint32_t idesc_qk = make_idesc_bf16(kBM, kBN, 0, 0);
       constexpr uint32_t idesc_pv = make_idesc_bf16(kBM, D, 0, 1);
       constexpr uint32_t LBO_QK = (D / 16) * PANEL;  // first half -> second half of a pair
       bool ok = mbar_wait(q_full, 0);
-      int last_pv = -1;
-      auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(p_full(i & 1), (i >> 1) & 1)) return false;
-        if (!mbar_wait(v_full(i % NS), (i / NS) & 1)) return false;
-        tc_fence_after();
-        const uint32_t pbuf = sP + (i & 1) * L::PBUF;
-        const uint32_t vbuf = sV + (i % NS) * L::TILE;
-#pragma unroll
-        for (int ks = 0; ks < kBN / 16; ++ks) {
-          const uint64_t ad = make_sdesc(pbuf + ks * 2 * PANEL, PANEL, 128, 0);
-          const uint64_t bd = make_sdesc(vbuf + ks * 2048, kBN * 128, 1024, 2);
-          umma_ss(tmem + TMEM_O, ad, bd, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
+      int cnt0 = 0, cnt1 = 0;  // tiles processed so far by query tile 0 / 1
+      bool qm_seen0 = false, qm_seen1 = false;
+      auto issue_qk = [&](int t, int j) -> bool {
+        bool& seen = t ? qm_seen1 : qm_seen0;
+        if (!seen) {  // the softmax warps prepared the masked k-step of tile t's first tile
+          if (!mbar_wait(qm_init(t), 0)) return false;
+          seen = true;
         }
-        umma_commit(pv_done(i & 1));
-        umma_commit(v_empty(i % NS));
-        last_pv = i;
+        const int kt = kt_top - j;
+        const int plo = tile_plo(t, kt);
+        const int k0 = plo >> 3;
+        const uint32_t kbuf = sK + (j % NS) * L::TILE;
+        const uint32_t qbuf = sQ + t * L::TILE;
+        for (int ks = k0; ks < KS; ++ks) {
+          // pairs 8*k0 .. plo-1 are pruned everywhere in the tile: the first
+          // step reads a copy of Q with those pairs zeroed
+          const uint64_t ad = (ks == k0 && (plo & 7))
+                                  ? make_sdesc(sQM + t * 2 * PANEL, PANEL, 128, 0)
+                                  : make_sdesc(qbuf + ks * PANEL, LBO_QK, 128, 0);
+          const uint64_t bd = make_sdesc(kbuf + ks * PANEL, LBO_QK, 128, 0);
+          umma_ss(tmem + t * kBN, ad, bd, idesc_qk, ks > k0 ? 1u : 0u);
+        }
+        umma_commit(s_full(t));
         return true;
       };
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % NS;
-        if (!mbar_wait(k_full(s), (j / NS) & 1)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(s_free(j & 1), ((j - 2) >> 1) & 1)) { ok = false; break; }
+      if (ok && mbar_wait(k_full(0), 0)) {
         tc_fence_after();
-        const int k0 = tile_k0(j);
-        const uint32_t kbuf = sK + s * L::TILE;
-        for (int ks = k0; ks < KS; ++ks) {
-          const uint64_t ad = make_sdesc(sQ + ks * PANEL, LBO_QK, 128, 0);
-          const uint64_t bd = make_sdesc(kbuf + ks * PANEL, LBO_QK, 128, 0);
-          umma_ss(tmem + TMEM_S + (j & 1) * kBN, ad, bd, idesc_qk, ks > k0 ? 1u : 0u);
-        }
-        umma_commit(s_full(j & 1));
-        umma_commit(k_empty(s));
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
-      }
-      if (ok) issue_pv(n_tiles - 1);
-      // do not release TMEM while an MMA may still write it
-      if (last_pv >= 0) mbar_wait(pv_done(last_pv & 1), (last_pv >> 1) & 1);
-    }
-  } else {
-    // ------------------------------------------------------------- softmax
-    const int r = threadIdx.x;               // row within the tile = TMEM lane
-    const int t = kBM * qt + r;
-    const int64_t i_pos = i_min + r;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const uint8_t* smem_q = smem + L::OFF_Q;
-    float m_ref = -INFINITY;   // max used as the exponent reference of O and l (log2 units)
-    float l_run = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int kt = kt_last - j;
-      const int s = j % NS;
-      const int bsel = j & 1;
-      const int64_t kp0 = p.k_pos0 + (int64_t)kBN * kt;
-      const int64_t d_row = i_pos - kp0;     // distance to the tile's first key
-      const int k0 = tile_k0(j);
-
-      if (!mbar_wait(s_full(bsel), (j >> 1) & 1)) { ok = false; break; }
-      tc_fence_after();
-      float sc[kBN];
-#pragma unroll
-      for (int cc = 0; cc < kBN / 32; ++cc)
-        tmem_ld32(lane_base + TMEM_S + bsel * kBN + 32 * cc,
-                  *reinterpret_cast<float(*)[32]>(&sc[32 * cc]));
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free(bsel));
-
-      if (k0 >= KS) {
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) sc[c] = 0.f;   // every pair pruned: score 0
+        if (kt_last0 >= kt_top && !issue_qk(0, 0)) ok = false;
+        if (ok && kt_last1 >= kt_top && !issue_qk(1, 0)) ok = false;
+        umma_commit(k_empty(0));
       } else {
-        // pairs 8*k0 .. p_min(d)-1 went through the MMA but are pruned at d
-        const int pm_row = d_row > 0 ? dev_pmin(p.T, P, d_row) : 0;
-        const int pc_lo = 8 * k0;
-        const int pc_hi = __reduce_max_sync(0xffffffffu, pm_row);
-        if (pc_hi > pc_lo) {
-          if (!mbar_wait(k_full(s), (j / NS) & 1)) { ok = false; break; }
-          const uint8_t* kb = smem + L::OFF_K + s * L::TILE;
-          for (int pp = pc_lo; pp < pc_hi; ++pp) {
-            int64_t lim64 = d_row - p.T[pp];        // columns c < lim have d > T_pp
-            const int lim = (int)(lim64 < 0 ? 0 : (lim64 > kBN ? kBN : lim64));
-            if (!__any_sync(0xffffffffu, lim > 0)) continue;
-            const int off_lo = (pp >> 3) * PANEL + (pp & 7) * 2;
-            const int off_hi = (P / 8 + (pp >> 3)) * PANEL + (pp & 7) * 2;
-            const float qa = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + off_lo + r * 16)) << 16);
-            const float qb = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + off_hi + r * 16)) << 16);
+        ok = false;
+      }
+      for (int j = 0; ok && j < n_iter; ++j) {
+        const int kt = kt_top - j;
+        const bool next = j + 1 < n_iter;
+        if (next && !mbar_wait(k_full((j + 1) % NS), ((j + 1) / NS) & 1)) { ok = false; break; }
+        if (!mbar_wait(v_full(j % NS), (j / NS) & 1)) { ok = false; break; }
+        const uint32_t vbuf = sV + (j % NS) * L::TILE;
 #pragma unroll
-            for (int c = 0; c < kBN; ++c) {
-              if (c < lim) {
-                const float ka = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(kb + off_lo + c * 16)) << 16);
-                const float kb2 = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(kb + off_hi + c * 16)) << 16);
-                sc[c] -= fmaf(qa, ka, qb * kb2);
+        for (int t = 0; t < kQT; ++t) {
+          const int ktl = t ? kt_last1 : kt_last0;
+          int& cnt = t ? cnt1 : cnt0;
+          if (ok && kt <= ktl) {
+            if (!mbar_wait(p_full(t), cnt & 1)) { ok = false; }
+            if (ok) {
+              tc_fence_after();
+#pragma unroll
+              for (int ks = 0; ks < kBN / 16; ++ks) {
+                const uint64_t bd = make_sdesc(vbuf + ks * 2048, kBN * 128, 1024, 2);
+                umma_ts(tmem + TMEM_O + t * D, tmem + t * kBN + ks * 8, bd, idesc_pv,
+                        (cnt > 0 || ks > 0) ? 1u : 0u);
               }
+              ++cnt;
             }
           }
+          if (ok && next && kt - 1 <= ktl && !issue_qk(t, j + 1)) ok = false;
         }
+        if (!ok) break;
+        umma_commit(v_empty(j % NS));
+        if (next) umma_commit(k_empty((j + 1) % NS));
+      }
+      // O_t final: every MMA issued so far has completed once this arrives
+      for (int t = 0; t < kQT; ++t) umma_commit(o_final(t));
+      if (!ok) mbar_wait(o_final(0), 0);
+    }
+  }
+  } else {
+    regs_increase<kRegsSoftmax>();
+    // ------------------------------------------------------------- softmax
+    const int t = warp >> 2;                   // query tile of this warpgroup
+    const int wq = warp & 3;                   // TMEM lane quarter
+    const int r = wq * 32 + lane;              // row within the tile = TMEM lane
+    const int row = (kQT * cq + t) * kBM + r;  // query index
+    const int64_t i_pos = p.q_pos0 + row;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t tS = lane_base + t * kBN;
+    const uint32_t tO = lane_base + TMEM_O + t * D;
+    const uint8_t* smem_q = smem + L::OFF_Q + t * L::TILE;
+    uint8_t* smem_qm = smem + L::OFF_QM + t * 2 * PANEL;
+    const int64_t i_tile0 = p.q_pos0 + (int64_t)(kQT * cq + t) * kBM;  // first row position
+    const int my_kt_last = t ? kt_last1 : kt_last0;
+    float m_ref = -INFINITY;   // exponent reference of O and l (log2 units)
+    float l_run = 0.f;
+    int cnt = 0;
+    bool ok = true;
+
+    // Copy of Q's first active k-step for a key tile whose first kept pair is
+    // plo, with the pairs that are pruned over the whole tile zeroed (the MMA
+    // reads it instead of Q).
+    auto write_masked_q = [&](int plo) {
+      const int rz = plo & 7;
+      if (rz == 0 || (plo >> 3) >= KS) return;
+      uint4 lo = *reinterpret_cast<const uint4*>(smem_q + (plo >> 3) * PANEL + r * 16);
+      uint4 hi = *reinterpret_cast<const uint4*>(smem_q + (P / 8 + (plo >> 3)) * PANEL + r * 16);
+      const uint32_t m0 = (rz > 0 ? 0u : 0xFFFFu) | (rz > 1 ? 0u : 0xFFFF0000u);
+      const uint32_t m1 = (rz > 2 ? 0u : 0xFFFFu) | (rz > 3 ? 0u : 0xFFFF0000u);
+      const uint32_t m2 = (rz > 4 ? 0u : 0xFFFFu) | (rz > 5 ? 0u : 0xFFFF0000u);
+      const uint32_t m3 = (rz > 6 ? 0u : 0xFFFFu) | 0xFFFF0000u;
+      lo.x &= m0; lo.y &= m1; lo.z &= m2; lo.w &= m3;
+      hi.x &= m0; hi.y &= m1; hi.z &= m2; hi.w &= m3;
+      *reinterpret_cast<uint4*>(smem_qm + r * 16) = lo;
+      *reinterpret_cast<uint4*>(smem_qm + PANEL + r * 16) = hi;
+      fence_proxy_async_smem();
+    };
+
+    // Q is read from shared memory for the masked copy and the corrections
+    ok = __all_sync(FULL, mbar_wait(q_full, 0));
+    int plo_next = my_kt_last >= 0 ? tile_plo(t, my_kt_last) : P;
+    if (ok && my_kt_last >= 0) write_masked_q(plo_next);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(qm_init(t));
+
+    for (int j = 0; ok && j < n_iter; ++j) {
+      const int kt = kt_top - j;
+      const int s = j % NS;
+      if (kt > my_kt_last) {
+        // no key of this tile is causal for us: only release K.  Wait for the
+        // stage's fill first, so that this arrival counts towards iteration j
+        // and not towards an earlier phase of the same stage.
+        if (!__all_sync(FULL, mbar_wait(k_full(s), (j / NS) & 1))) { ok = false; break; }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(k_empty(s));
+        continue;
+      }
+      const int64_t kp0 = p.k_pos0 + (int64_t)kBN * kt;
+      const int64_t d_row = i_pos - kp0;     // distance to the tile's first key
+      const int plo = plo_next;
+      const bool all_pruned = plo >= P;
+      if (kt > 0) plo_next = tile_plo(t, kt - 1);
+
+      if (!__all_sync(FULL, mbar_wait(s_full(t), cnt & 1))) { ok = false; break; }
+      tc_fence_after();
+
+      // Pairs plo .. p_min(d)-1 are kept at some distances of the tile and
+      // pruned at this element's: subtract their terms (per element).  Pair
+      // plo is pruned somewhere in this row iff the row's largest distance
+      // exceeds its threshold.
+      if (!all_pruned && __any_sync(FULL, d_row > p.T[plo])) {
+        const int pm_row = d_row > 0 ? dev_pmin(p.T, P, d_row) : 0;
+        const int pc_hi = __reduce_max_sync(FULL, pm_row);
+        if (!__all_sync(FULL, mbar_wait(k_full(s), (j / NS) & 1))) { ok = false; break; }
+        const uint8_t* kb = smem + L::OFF_K + s * L::TILE;
+        if (p.g8) {
+          // whole groups of 8 pairs share a threshold: one 16-dim dot product per element
+#pragma unroll 1
+          for (int gp = plo; gp < pc_hi; gp += 8) {
+            const int64_t lim0 = d_row - p.T[gp];         // columns c < lim0: d > T_group
+            if (!__any_sync(FULL, lim0 > 0)) continue;
+            const int off_lo = (gp >> 3) * PANEL;
+            const int off_hi = (P / 8 + (gp >> 3)) * PANEL;
+            float qv[16];
+            {
+              const uint4 a = *reinterpret_cast<const uint4*>(smem_q + off_lo + r * 16);
+              const uint4 c = *reinterpret_cast<const uint4*>(smem_q + off_hi + r * 16);
+              qv[0] = bf16lo_to_f32(a.x); qv[1] = bf16hi_to_f32(a.x);
+              qv[2] = bf16lo_to_f32(a.y); qv[3] = bf16hi_to_f32(a.y);
+              qv[4] = bf16lo_to_f32(a.z); qv[5] = bf16hi_to_f32(a.z);
+              qv[6] = bf16lo_to_f32(a.w); qv[7] = bf16hi_to_f32(a.w);
+              qv[8] = bf16lo_to_f32(c.x); qv[9] = bf16hi_to_f32(c.x);
+              qv[10] = bf16lo_to_f32(c.y); qv[11] = bf16hi_to_f32(c.y);
+              qv[12] = bf16lo_to_f32(c.z); qv[13] = bf16hi_to_f32(c.z);
+              qv[14] = bf16lo_to_f32(c.w); qv[15] = bf16hi_to_f32(c.w);
+            }
+#pragma unroll 1
+            for (int cc = 0; cc < kBN / 32; ++cc) {
+              const int64_t l64 = lim0 - 32 * cc;
+              const int lim = (int)(l64 < 0 ? 0 : (l64 > 32 ? 32 : l64));
+              if (!__any_sync(FULL, lim > 0)) continue;
+              float v[32];
+              tmem_ld32(tS + 32 * cc, v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                const uint4 a = *reinterpret_cast<const uint4*>(kb + off_lo + (32 * cc + c) * 16);
+                const uint4 b2 = *reinterpret_cast<const uint4*>(kb + off_hi + (32 * cc + c) * 16);
+                float d0 = 0.f, d1 = 0.f;
+                fma2(d0, d1, qv[0], qv[1], bf16lo_to_f32(a.x), bf16hi_to_f32(a.x), d0, d1);
+                fma2(d0, d1, qv[2], qv[3], bf16lo_to_f32(a.y), bf16hi_to_f32(a.y), d0, d1);
+                fma2(d0, d1, qv[4], qv[5], bf16lo_to_f32(a.z), bf16hi_to_f32(a.z), d0, d1);
+                fma2(d0, d1, qv[6], qv[7], bf16lo_to_f32(a.w), bf16hi_to_f32(a.w), d0, d1);
+                fma2(d0, d1, qv[8], qv[9], bf16lo_to_f32(b2.x), bf16hi_to_f32(b2.x), d0, d1);
+                fma2(d0, d1, qv[10], qv[11], bf16lo_to_f32(b2.y), bf16hi_to_f32(b2.y), d0, d1);
+                fma2(d0, d1, qv[12], qv[13], bf16lo_to_f32(b2.z), bf16hi_to_f32(b2.z), d0, d1);
+                fma2(d0, d1, qv[14], qv[15], bf16lo_to_f32(b2.w), bf16hi_to_f32(b2.w), d0, d1);
+                if (c < lim) v[c] -= d0 + d1;
+              }
+              tmem_st32(tS + 32 * cc, v);
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int cc = 0; cc < kBN / 32; ++cc) {
+            // thresholds grow with the pair index: pair plo reaches furthest into the tile
+            const int64_t first = d_row - p.T[plo] - 32 * cc;
+            if (!__any_sync(FULL, first > 0)) break;
+            float v[32];
+            tmem_ld32(tS + 32 * cc, v);
+            tmem_ld_wait();
+#pragma unroll 1
+            for (int pp = plo; pp < pc_hi; ++pp) {
+              const int64_t lim64 = d_row - p.T[pp] - 32 * cc;  // columns c < lim: d > T_pp
+              const int lim = (int)(lim64 < 0 ? 0 : (lim64 > 32 ? 32 : lim64));
+              if (!__any_sync(FULL, lim > 0)) break;
+              const int off_lo = (pp >> 3) * PANEL + (pp & 7) * 2;
+              const int off_hi = (P / 8 + (pp >> 3)) * PANEL + (pp & 7) * 2;
+              const float qa = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + off_lo + r * 16)) << 16);
+              const float qb = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + off_hi + r * 16)) << 16);
+              const uint8_t* klo = kb + off_lo + cc * 32 * 16;
+              const uint8_t* khi = kb + off_hi + cc * 32 * 16;
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                if (c < lim) {
+                  const float ka = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(klo + c * 16)) << 16);
+                  const float kb2 = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(khi + c * 16)) << 16);
+                  v[c] -= fmaf(qa, ka, qb * kb2);
+                }
+              }
+            }
+            tmem_st32(tS + 32 * cc, v);
+          }
+        }
+        tmem_st_wait();
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(k_empty(s));
 
-      // causal mask (d < 0) and the ragged key tail
-      const int64_t dlo_tile = i_min - (kp0 + kBN - 1);
-      const bool tail = (int64_t)kBN * kt + kBN > p.Nk;
-      if (dlo_tile < 0 || tail) {
-        int64_t cmax = d_row;                                 // last column with d >= 0
-        const int64_t cnk = (int64_t)p.Nk - 1 - (int64_t)kBN * kt;  // last real key
-        if (cnk < cmax) cmax = cnk;
+      float sc[kBN];
 #pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (c > cmax) sc[c] = -INFINITY;
+      for (int cc = 0; cc < kBN / 32; ++cc) tmem_ld32(tS + 32 * cc, &sc[32 * cc]);
+      tmem_ld_wait();
+      if (all_pruned) {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) sc[c] = 0.f;   // every pair pruned: score 0
       }
 
-      float mt = -INFINITY;
+      // causal mask (d < 0) and the ragged key tail: columns c > cm
+      const bool need_mask = (i_tile0 - (kp0 + kBN - 1) < 0) || ((int64_t)kBN * kt + kBN > p.Nk);
+      int cm = kBN - 1;
+      if (need_mask) {
+        int64_t cmax = d_row;                                      // last column with d >= 0
+        const int64_t cnk = (int64_t)p.Nk - 1 - (int64_t)kBN * kt; // last real key
+        if (cnk < cmax) cmax = cnk;
+        cm = (int)(cmax < -1 ? -1 : (cmax > kBN ? kBN : cmax));
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) mt = fmaxf(mt, sc[c]);
+        for (int c = 0; c < kBN; ++c)
+          if (c > cm) sc[c] = -INFINITY;
+      }
+
+      // row max: 16 independent 3-input max chains, then a tree
+      float a16[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        a16[k] = max3(max3(sc[8 * k], sc[8 * k + 1], sc[8 * k + 2]),
+                      max3(sc[8 * k + 3], sc[8 * k + 4], sc[8 * k + 5]),
+                      fmaxf(sc[8 * k + 6], sc[8 * k + 7]));
+      float b6[6];
+#pragma unroll
+      for (int k = 0; k < 5; ++k) b6[k] = max3(a16[3 * k], a16[3 * k + 1], a16[3 * k + 2]);
+      b6[5] = a16[15];
+      float mt = max3(max3(b6[0], b6[1], b6[2]), max3(b6[3], b6[4], b6[5]), -INFINITY);
       mt *= p.scale_log2;
 
-      // lazy rescale: move the reference only when the max grew by > 8 (x256)
+      // lazy rescale: move the reference only when the max grew by > 8 (x256).
+      // s_full of this tile implies the previous PV of this tile has completed.
       float f = 1.f;
       bool resc = false;
-      if (j == 0) {
+      if (cnt == 0) {
         m_ref = mt;
       } else if (mt > m_ref + 8.f) {
         f = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mt);
         m_ref = mt;
         resc = true;
       }
-      if (__any_sync(0xffffffffu, resc)) {
-        if (!mbar_wait(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
+      if (__any_sync(FULL, resc)) {
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           float o[32];
-          tmem_ld32(lane_base + TMEM_O + 32 * cc, o);
+          tmem_ld32(tO + 32 * cc, o);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= f;
-          tmem_st32(lane_base + TMEM_O + 32 * cc, o);
+          tmem_st32(tO + 32 * cc, o);
         }
-        tmem_st_wait();
       }
       l_run *= f;
 
-      // P buffer bsel was last read by PV(j-2)
-      if (j >= 2 && !mbar_wait(pv_done(bsel), ((j - 2) >> 1) & 1)) { ok = false; break; }
-      const float msafe = (m_ref == -INFINITY) ? 0.f : m_ref;
-      uint8_t* pb = smem + L::OFF_P + bsel * L::PBUF + r * 16;
-      float rowsum = 0.f;
+      // p = 2^(s * scale * log2 e - m): exponents two at a time, part of them
+      // on the FMA pipe; masked columns get exactly 0.
+      const float nm = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      const float sl = p.scale_log2;
+      float acc[8];
 #pragma unroll
-      for (int kc = 0; kc < kBN / 8; ++kc) {
-        float pv[8];
+      for (int k = 0; k < 8; ++k) acc[k] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pv[e] = ex2_approx(fmaf(sc[8 * kc + e], p.scale_log2, -msafe));
-          rowsum += pv[e];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int c = 64 * half + 2 * i;
+          float x0, x1, e0, e1;
+          fma2(x0, x1, sc[c], sc[c + 1], sl, sl, nm, nm);
+          if ((i & 7) >= 8 - L::NPOLY) {
+            exp2_poly2(e0, e1, x0, x1);
+          } else {
+            e0 = ex2_approx(x0);
+            e1 = ex2_approx(x1);
+          }
+          add2(acc[2 * (i & 3)], acc[2 * (i & 3) + 1], acc[2 * (i & 3)], acc[2 * (i & 3) + 1], e0, e1);
+          pk[i] = pack_bf16x2(e0, e1);
         }
-        uint4 w;
-        w.x = pack_bf16x2(pv[0], pv[1]);
-        w.y = pack_bf16x2(pv[2], pv[3]);
-        w.z = pack_bf16x2(pv[4], pv[5]);
-        w.w = pack_bf16x2(pv[6], pv[7]);
-        *reinterpret_cast<uint4*>(pb + kc * PANEL) = w;
+        tmem_st32u(tS + 32 * half, pk);
       }
-      l_run += rowsum;
-      fence_proxy_async_smem();
+      l_run += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      // the next tile's masked Q step, before P is released to the MMA warp
+      if (kt > 0) write_masked_q(plo_next);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full(bsel));
+      if (lane == 0) mbar_arrive(p_full(t));
+      ++cnt;
     }
 
     // epilogue: O / l
-    const bool row_ok = t < p.Nq;
-    uint16_t* orow = p.out + (((size_t)b * p.Nq + t) * p.Hq + h) * D;
-    if (ok && n_tiles > 0) {
-      const int last = n_tiles - 1;
-      ok = mbar_wait(pv_done(last & 1), (last >> 1) & 1);
+    const bool row_ok = row < p.Nq;
+    uint16_t* orow = p.out + (((size_t)b * p.Nq + (row_ok ? row : 0)) * p.Hq + h) * D;
+    if (cnt > 0) {
+      ok = __all_sync(FULL, mbar_wait(o_final(t), 0)) && ok;
       tc_fence_after();
     }
     const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
       float o[32];
-      if (n_tiles > 0) {
-        tmem_ld32(lane_base + TMEM_O + 32 * cc, o);
+      if (cnt > 0) {
+        tmem_ld32(tO + 32 * cc, o);
         tmem_ld_wait();
       }
 #pragma unroll
-      for (int e = 0; e < 32; ++e) o[e] = (n_tiles > 0) ? o[e] * inv : 0.f;
+      for (int e = 0; e < 32; ++e) o[e] = (cnt > 0) ? o[e] * inv : 0.f;
       if (row_ok) {
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4) {
@@ -386,14 +573,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
     }
     if (row_ok && p.lse)
-      p.lse[((size_t)b * p.Hq + h) * p.Nq + t] =
+      p.lse[((size_t)b * p.Hq + h) * p.Nq + row] =
           (l_run > 0.f) ? (m_ref + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, 512);
+  if (warp == 9) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace wpattn

@@ -60,6 +60,11 @@ WORKLOADS = {
                                       1048576, 1e7, 1.0, 8, q_pos0=1048576 - 16384),
     "qwen2.5-7b-1m-decode": Workload("qwen2.5-7b-1m-decode", "decode", 1, 28, 4, 128, 1,
                                      1048576, 1e7, 1.0, 8),
+    # reduced shapes of the same kernels, for profiler captures (inputs still larger than L2)
+    "llama3.2-3b-32k-a1": Workload("llama3.2-3b-32k-a1", "prefill", 1, 24, 8, 128, 32768, 32768,
+                                   5e5, 1.0, 1),
+    "llama3.2-3b-decode-32k": Workload("llama3.2-3b-decode-32k", "decode", 4, 24, 8, 128, 1,
+                                       32768, 5e5, 1.0, 1),
 }
 
 

@@ -22,9 +22,13 @@ def check_rows(o_gpu, l_gpu, o_ref, l_ref, what):
     if empty.any():
         assert (o_gpu[empty] == 0).all(), f"{what}: empty rows must be 0"
     ok = ~empty
-    d_out = float(np.abs(o_gpu[ok] - o_ref[ok]).max()) if ok.any() else 0.0
-    d_lse = float(np.abs(l_gpu[ok] - l_ref[ok]).max()) if ok.any() else 0.0
-    assert d_out <= ATOL_OUT and d_lse <= ATOL_LSE, f"{what}: max|dout|={d_out:.3e} max|dlse|={d_lse:.3e}"
+    err_o = np.where(ok[:, None], np.abs(o_gpu - o_ref), 0.0).max(axis=1)
+    err_l = np.where(ok, np.abs(l_gpu - l_ref), 0.0)
+    d_out, d_lse = float(err_o.max()), float(err_l.max())
+    bad = np.nonzero((err_o > ATOL_OUT) | (err_l > ATOL_LSE))[0]
+    assert d_out <= ATOL_OUT and d_lse <= ATOL_LSE, (
+        f"{what}: max|dout|={d_out:.3e} max|dlse|={d_lse:.3e}; {len(bad)} of {len(ok)} rows "
+        f"out of tolerance, first: {bad[:12].tolist()}")
     return d_out, d_lse
 
 
