@@ -27,8 +27,8 @@
  *    records WPATTN_ETIMEOUT, which wpattn_device_status returns.
  *  - bf16 tensors are contiguous, row-major, in the layouts stated below, and
  *    16-byte aligned.
- *  - The library allocates no device memory in the calls below except a
- *    4-byte status word per device, created on first use.
+ *  - No entry point allocates device memory.  The library's device image holds
+ *    a 4-byte status word and the scratch array of wpattn_decode_noalloc.
  */
 #ifndef WPATTN_H
 #define WPATTN_H
@@ -142,6 +142,35 @@ WPATTN_API int wpattn_decode(const wpattn_window *w,
                   void *out, float *lse,
                   void *workspace, size_t workspace_bytes,
                   void *cuda_stream);
+
+/*
+ * Decode without any allocation: the same computation as wpattn_decode, with
+ * its scratch (the per-split partial results) taken from a fixed array built
+ * into the library instead of a caller-supplied workspace.  The paper has no
+ * counterpart; it is for callers that cannot allocate device memory at the
+ * point of the call: a serving runtime whose allocator already reserved the
+ * GPU's memory, a plugin that only receives tensors from its host, or code on
+ * a latency path where cudaMalloc (which can synchronise the device) is not
+ * allowed.  Arguments as for wpattn_decode, minus the workspace.
+ *  - The scratch array holds wpattn_decode_noalloc_max_bytes() bytes (4 MiB)
+ *    on every GPU that loads the library, until the process exits.  A problem
+ *    whose partial results need more (B * Hq * splits * (D + 2) * 4 bytes)
+ *    is rejected with WPATTN_EWORKSPACE and nothing runs.
+ *  - The first call on a device looks up the array's device address for that
+ *    device (cudaGetSymbolAddress); make that first call before capturing a
+ *    stream into a CUDA graph.
+ *  - Every call on a device shares the one array: calls whose kernels can
+ *    overlap on the GPU (different streams, no ordering) race on it.  Nothing
+ *    in it needs clearing: each call writes every partial it later reads.
+ */
+WPATTN_API int wpattn_decode_noalloc(const wpattn_window *w,
+                  const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *kv_len_host, int64_t Lmax,
+                  int32_t B, int32_t Hq, int32_t Hkv, float softmax_scale,
+                  void *out, float *lse, void *cuda_stream);
+
+/* Size in bytes of the built-in scratch array wpattn_decode_noalloc uses. */
+WPATTN_API size_t wpattn_decode_noalloc_max_bytes(void);
 
 /*
  * Synchronises `cuda_stream`, then reads and clears the current device's

@@ -182,6 +182,41 @@ def decode(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | None = None
     return out, lse
 
 
+def decode_noalloc(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | None = None,
+                   out=None, lse=None, want_lse: bool = True, stream=None):
+    """Decode with the library's built-in scratch instead of a workspace.
+
+    For callers that cannot allocate device memory at the call site; the
+    problem's partial results must fit the built-in array
+    (``decode_noalloc_max_bytes()``), calls on one device share it.
+    """
+    import torch
+    B, Hq, D = q.shape
+    L, Hkv = k_cache.shape[1], k_cache.shape[2]
+    kvl = (ctypes.c_int32 * B)(*[int(x) for x in kv_len])
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    fn = lib().wpattn_decode_noalloc
+    fn.argtypes = [ctypes.POINTER(_Window), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                   ctypes.POINTER(ctypes.c_int32), ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                   ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                   ctypes.c_void_p]
+    rc = fn(ctypes.byref(w._c()), _dev_tensor(q, "q"), _dev_tensor(k_cache, "k_cache"),
+            _dev_tensor(v_cache, "v_cache"), kvl, L, B, Hq, Hkv, float(scale) if scale else 0.0,
+            _dev_tensor(out, "out"), ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+            _stream_ptr(stream))
+    _check(rc, "wpattn_decode_noalloc")
+    return out, lse
+
+
+def decode_noalloc_max_bytes() -> int:
+    fn = lib().wpattn_decode_noalloc_max_bytes
+    fn.restype = ctypes.c_size_t
+    return int(fn())
+
+
 def device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the kernels' status word."""
     return int(lib().wpattn_device_status(_stream_ptr(stream)))

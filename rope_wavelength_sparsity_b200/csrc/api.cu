@@ -46,6 +46,7 @@ struct DeviceInfo {
   bool supported = false;
   int num_sms = 0;
   bool prefill_attr[2] = {false, false};
+  void* static_scratch = nullptr;  // device address of g_decode_static_scratch
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -146,6 +147,12 @@ int launch_decode(const DecodeParams& prm, int gc, cudaStream_t st) {
 
 }  // namespace
 }  // namespace wpattn
+
+// Scratch for wpattn_decode_noalloc: a fixed-size array in the library's own
+// device image, so that entry point never allocates.  Every GPU that loads
+// the library holds these bytes until the process exits.
+constexpr size_t kDecodeStaticScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_decode_static_scratch[kDecodeStaticScratchBytes];
 
 using namespace wpattn;
 
@@ -291,6 +298,36 @@ int wpattn_decode(const wpattn_window* w, const void* q, const void* k_cache, co
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   if (plan.D == 64) return launch_decode<64>(prm, gc, st);
   return launch_decode<128>(prm, gc, st);
+}
+
+size_t wpattn_decode_noalloc_max_bytes(void) { return kDecodeStaticScratchBytes; }
+
+int wpattn_decode_noalloc(const wpattn_window* w, const void* q, const void* k_cache,
+                          const void* v_cache, const int32_t* kv_len_host, int64_t Lmax, int32_t B,
+                          int32_t Hq, int32_t Hkv, float softmax_scale, void* out, float* lse,
+                          void* cuda_stream) {
+  WindowPlan plan;
+  int rc = make_window_plan(w, &plan);
+  if (rc != WPATTN_OK) return rc;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0 || Lmax <= 0) return WPATTN_EINVAL;
+  DeviceInfo* dev = nullptr;
+  if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
+  // scratch this problem needs under the current device's split plan
+  const int S = decode_splits(B, Hkv, Lmax, dev->num_sms);
+  if (decode_workspace_bytes(B, Hq, plan.D, S) > kDecodeStaticScratchBytes) return WPATTN_EWORKSPACE;
+  {
+    // once per device, with that device current: the array's device address
+    // (host code cannot use the symbol itself as a device pointer)
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!dev->static_scratch) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_decode_static_scratch) != cudaSuccess || !ptr)
+        return WPATTN_ECUDA;
+      dev->static_scratch = ptr;
+    }
+  }
+  return wpattn_decode(w, q, k_cache, v_cache, kv_len_host, Lmax, B, Hq, Hkv, softmax_scale, out,
+                       lse, dev->static_scratch, kDecodeStaticScratchBytes, cuda_stream);
 }
 
 int wpattn_device_status(void* cuda_stream) {
