@@ -44,15 +44,22 @@ DECODE_WORKLOAD = "llama3.2-3b-decode-128k"
 FLUSH_BYTES = 512 << 20
 
 # DRAM bytes (read + write) per launch of the dominant kernel from one ncu
-# capture, keyed by the sha256 of the kernel sources at capture time; a
-# changed kernel reports null until it is captured again.
-NCU_TRAFFIC = {}
+# capture (profiles/ holds the summaries), keyed by workload and by a hash of
+# that kernel's sources at capture time: a changed kernel reports null until
+# it is captured again.
+NCU_TRAFFIC = {
+    # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.25 MB read + 24.16 MB written
+    ("qwen2.5-0.5b-32k", "962f4baf275be7cd"): 100412416,
+}
+
+KERNEL_SOURCES = {"prefill": ("prefill_kernel.cuh", "device_util.cuh"),
+                  "decode": ("decode_kernels.cuh", "device_util.cuh")}
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rope_wavelength_sparsity_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -171,13 +178,20 @@ def _dist_setup(args):
 
 
 def _max_over_ranks(x: float, world: int) -> float:
+    """Largest value over all ranks (the timing reduction; no data-path collective)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, world: int, max_ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's step time."""
+    return world * units_per_rank / (max_ms_per_step * 1e-3)
 
 
 def _barrier(world):
@@ -250,10 +264,10 @@ def gpu_arm(args):
         off_ms, _, _ = time_steps(step_off, args.warmup, max(3, args.steps // 4), flush, world)
         off_ms_step = off_ms / max(3, args.steps // 4)
         ms_step = total_ms / args.steps
-        value = world * eff / (ms_step * 1e-3) / 1e12
+        value = weak_scaling_value(eff, world, ms_step) / 1e12
         kernel_ms = statistics.mean(per)
         achieved = eff / (kernel_ms * 1e-3) / 1e12
-        traffic = NCU_TRAFFIC.get((args.workload, kernel_source_hash()))
+        traffic = NCU_TRAFFIC.get((args.workload, kernel_source_hash("prefill")))
         result.update({
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s",
             "ms_per_step": round(ms_step, 4),
@@ -350,11 +364,11 @@ def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
     off_step = off_ms / max(3, steps // 4)
     achieved = alg / (statistics.mean(per) * 1e-3) / 1e9
     res = {
-        "metric": METRIC, "value": round(world * alg / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "metric": METRIC, "value": round(weak_scaling_value(alg, world, ms) / 1e9, 1), "unit": "GB/s",
         "ms_per_step": round(ms, 4), "dtype": "bf16",
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "traffic": NCU_TRAFFIC.get((w.name, kernel_source_hash())),
+                     "traffic": NCU_TRAFFIC.get((w.name, kernel_source_hash("decode"))),
                      "peak_source": f"{peaks['source']} HBM copy",
                      "timed": "split + combine kernels (one decode call)"},
         "window_off": {"ms_per_step": round(off_step, 4), "speedup": round(off_step / ms, 3),
