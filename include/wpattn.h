@@ -103,8 +103,9 @@ WPATTN_API int wpattn_pruned_fraction(const wpattn_window *w, int64_t Nq, int64_
  *   lse : fp32 device [B, Hq, Nq] natural-log sum-exp of scale*s, or NULL
  * Query head h reads kv head h / (Hq / Hkv).  softmax_scale <= 0 means
  * 1/sqrt(D).  A query with no causal key gets out = 0 and lse = -inf.
- * Requires D in {64, 128}, Hq % Hkv == 0, an sm_100 device, and
- * 0 <= Nq, Nk < 2^31.  Nq == 0 or B == 0 is a no-op.
+ * Requires D in {64, 128}, Hq % Hkv == 0, an sm_100 device,
+ * 0 <= Nq, Nk <= 2^30 and |q_pos0 - k_pos0| <= 2^30 (else WPATTN_EUNSUPPORTED).
+ * Nq == 0 or B == 0 is a no-op.
  */
 WPATTN_API int wpattn_prefill(const wpattn_window *w,
                    const void *q, const void *k, const void *v,

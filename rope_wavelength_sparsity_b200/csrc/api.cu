@@ -234,12 +234,16 @@ int wpattn_prefill(const wpattn_window* w, const void* q, const void* k, const v
   prm.lse = lse;
   prm.B = B; prm.Nq = Nq; prm.Nk = Nk; prm.Hq = Hq; prm.Hkv = Hkv; prm.G = Hq / Hkv;
   prm.num_ctas_q = (Nq + kQT * kBM - 1) / (kQT * kBM);
-  prm.q_pos0 = q_pos0;
-  prm.k_pos0 = k_pos0;
+  // the kernel works in positions relative to k_pos0, in 32-bit integers
+  const int64_t qk_off = q_pos0 - k_pos0;
+  if (qk_off < -(int64_t(1) << 30) || qk_off > (int64_t(1) << 30) || Nq > (1 << 30) ||
+      Nk > (1 << 30))
+    return WPATTN_EUNSUPPORTED;
+  prm.qk_off = static_cast<int>(qk_off);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(plan.D));
   prm.scale_log2 = scale * 1.44269504088896340736f;
   prm.g8 = plan.g == 8 ? 1 : 0;
-  for (int p = 0; p < 64; ++p) prm.T[p] = plan.T[p];
+  for (int p = 0; p < 64; ++p) prm.T[p] = plan.T[p] > INT32_MAX ? INT32_MAX : static_cast<int>(plan.T[p]);
   const void* kk = Nk > 0 ? k : q;
   const void* vv = Nk > 0 ? v : q;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);

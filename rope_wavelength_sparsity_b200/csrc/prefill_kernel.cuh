@@ -55,10 +55,10 @@ struct PrefillParams {
   float* lse;         // [B, Hq, Nq] or null
   int B, Nq, Nk, Hq, Hkv, G;
   int num_ctas_q;     // CTAs along the query axis (256 rows each)
-  int64_t q_pos0, k_pos0;
+  int qk_off;         // q_pos0 - k_pos0: query t is at relative position qk_off + t, key j at j
   float scale_log2;   // softmax scale * log2(e)
   int g8;             // 1: pairs share thresholds in groups of 8
-  int64_t T[64];      // per-pair thresholds (nondecreasing)
+  int T[64];          // per-pair thresholds (nondecreasing), clamped to INT32_MAX
 };
 
 template <int D>
@@ -79,7 +79,7 @@ struct PrefillSmem {
   static constexpr int ALLOC = BYTES;
 };
 
-__device__ __forceinline__ int dev_pmin(const int64_t* T, int P, int64_t d) {
+__device__ __forceinline__ int dev_pmin(const int* T, int P, int d) {
   int lo = 0, hi = P;
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
@@ -124,6 +124,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   auto p_full = [&](int t) { return bar + 8 * (3 + 4 * NS + t); };
   auto o_final = [&](int t) { return bar + 8 * (5 + 4 * NS + t); };
   auto qm_init = [&](int t) { return bar + 8 * (7 + 4 * NS + t); };
+
   const uint32_t sQM = sbase + L::OFF_QM;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
 
@@ -142,21 +143,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   auto last_key_tile = [&](int t) -> int {
     const int row0 = (kQT * cq + t) * kBM;
     if (row0 >= p.Nq || p.Nk <= 0) return -1;
-    const int64_t i_max = p.q_pos0 + min(row0 + kBM - 1, p.Nq - 1);
-    if (i_max < p.k_pos0) return -1;
-    const int64_t last = (i_max - p.k_pos0) / kBN;
-    return (int)(last < (int64_t)(nkt - 1) ? last : (int64_t)(nkt - 1));
+    const int i_max = p.qk_off + min(row0 + kBM - 1, p.Nq - 1);
+    if (i_max < 0) return -1;
+    return min(i_max / kBN, nkt - 1);
   };
   const int kt_last0 = last_key_tile(0), kt_last1 = last_key_tile(1);
   const int kt_top = max(kt_last0, kt_last1);
   const int n_iter = kt_top + 1;  // shared K/V iterations j: key tile kt_top - j
-  // first pair of query tile t that is kept somewhere in key tile kt: pairs
-  // below it are pruned at the tile's smallest distance, hence everywhere
-  auto tile_plo = [&](int t, int kt) -> int {
-    const int64_t i_min = p.q_pos0 + (int64_t)(kQT * cq + t) * kBM;
-    int64_t dlo = i_min - (p.k_pos0 + (int64_t)kBN * kt + kBN - 1);
-    if (dlo < 0) dlo = 0;
-    return dev_pmin(p.T, P, dlo);
+  // Smallest distance of query tile t in key tile kt (negative on the diagonal).
+  // Going down the key tiles it grows by 128, so the first kept pair of the
+  // tile (p_min of that distance) only moves forward: advance it in place.
+  auto advance_plo = [&](int t, int kt, int& plo) {
+    const int dlo = p.qk_off + (kQT * cq + t) * kBM - (kBN * kt + kBN - 1);
+    while (plo < P && p.T[plo] < dlo) ++plo;
   };
 
   if (threadIdx.x == 0) {
@@ -172,6 +171,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(p_full(t), 4);
       mbar_init(o_final(t), 1);
       mbar_init(qm_init(t), 4);
+
     }
     fence_barrier_init();
   }
@@ -222,6 +222,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = mbar_wait(q_full, 0);
       int cnt0 = 0, cnt1 = 0;  // tiles processed so far by query tile 0 / 1
       bool qm_seen0 = false, qm_seen1 = false;
+      int plo0 = 0, plo1 = 0;
+      // descriptors: start addresses advance by adding (byte offset >> 4)
+      const uint64_t qdesc0 = make_sdesc(sQ, LBO_QK, 128, 0);
+      const uint64_t qmdesc0 = make_sdesc(sQM, PANEL, 128, 0);
+      const uint64_t kdesc0 = make_sdesc(sK, LBO_QK, 128, 0);
+      const uint64_t vdesc0 = make_sdesc(sV, kBN * 128, 1024, 2);
       auto issue_qk = [&](int t, int j) -> bool {
         bool& seen = t ? qm_seen1 : qm_seen0;
         if (!seen) {  // the softmax warps prepared the masked k-step of tile t's first tile
@@ -229,18 +235,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           seen = true;
         }
         const int kt = kt_top - j;
-        const int plo = tile_plo(t, kt);
+        int& plo = t ? plo1 : plo0;
+        advance_plo(t, kt, plo);
         const int k0 = plo >> 3;
-        const uint32_t kbuf = sK + (j % NS) * L::TILE;
-        const uint32_t qbuf = sQ + t * L::TILE;
+        const uint64_t kbase = kdesc0 + (uint64_t)(((j % NS) * L::TILE) >> 4);
+        const uint64_t qbase = qdesc0 + (uint64_t)((t * L::TILE) >> 4);
+        const uint32_t d_tmem = tmem + t * kBN;
         for (int ks = k0; ks < KS; ++ks) {
           // pairs 8*k0 .. plo-1 are pruned everywhere in the tile: the first
           // step reads a copy of Q with those pairs zeroed
           const uint64_t ad = (ks == k0 && (plo & 7))
-                                  ? make_sdesc(sQM + t * 2 * PANEL, PANEL, 128, 0)
-                                  : make_sdesc(qbuf + ks * PANEL, LBO_QK, 128, 0);
-          const uint64_t bd = make_sdesc(kbuf + ks * PANEL, LBO_QK, 128, 0);
-          umma_ss(tmem + t * kBN, ad, bd, idesc_qk, ks > k0 ? 1u : 0u);
+                                  ? qmdesc0 + (uint64_t)((t * 2 * PANEL) >> 4)
+                                  : qbase + (uint64_t)((ks * PANEL) >> 4);
+          umma_ss(d_tmem, ad, kbase + (uint64_t)((ks * PANEL) >> 4), idesc_qk, ks > k0 ? 1u : 0u);
         }
         umma_commit(s_full(t));
         return true;
@@ -258,7 +265,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const bool next = j + 1 < n_iter;
         if (next && !mbar_wait(k_full((j + 1) % NS), ((j + 1) / NS) & 1)) { ok = false; break; }
         if (!mbar_wait(v_full(j % NS), (j / NS) & 1)) { ok = false; break; }
-        const uint32_t vbuf = sV + (j % NS) * L::TILE;
+        const uint64_t vbase = vdesc0 + (uint64_t)(((j % NS) * L::TILE) >> 4);
 #pragma unroll
         for (int t = 0; t < kQT; ++t) {
           const int ktl = t ? kt_last1 : kt_last0;
@@ -268,11 +275,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (ok) {
               tc_fence_after();
 #pragma unroll
-              for (int ks = 0; ks < kBN / 16; ++ks) {
-                const uint64_t bd = make_sdesc(vbuf + ks * 2048, kBN * 128, 1024, 2);
-                umma_ts(tmem + TMEM_O + t * D, tmem + t * kBN + ks * 8, bd, idesc_pv,
-                        (cnt > 0 || ks > 0) ? 1u : 0u);
-              }
+              for (int ks = 0; ks < kBN / 16; ++ks)
+                umma_ts(tmem + TMEM_O + t * D, tmem + t * kBN + ks * 8,
+                        vbase + (uint64_t)((ks * 2048) >> 4), idesc_pv, (cnt > 0 || ks > 0) ? 1u : 0u);
               ++cnt;
             }
           }
@@ -294,13 +299,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int wq = warp & 3;                   // TMEM lane quarter
     const int r = wq * 32 + lane;              // row within the tile = TMEM lane
     const int row = (kQT * cq + t) * kBM + r;  // query index
-    const int64_t i_pos = p.q_pos0 + row;
+    const int i_pos = p.qk_off + row;          // relative position of this row
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t tS = lane_base + t * kBN;
     const uint32_t tO = lane_base + TMEM_O + t * D;
     const uint8_t* smem_q = smem + L::OFF_Q + t * L::TILE;
     uint8_t* smem_qm = smem + L::OFF_QM + t * 2 * PANEL;
-    const int64_t i_tile0 = p.q_pos0 + (int64_t)(kQT * cq + t) * kBM;  // first row position
+    const int i_tile0 = p.qk_off + (kQT * cq + t) * kBM;  // relative position of the first row
     const int my_kt_last = t ? kt_last1 : kt_last0;
     float m_ref = -INFINITY;   // exponent reference of O and l (log2 units)
     float l_run = 0.f;
@@ -328,7 +333,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     // Q is read from shared memory for the masked copy and the corrections
     ok = __all_sync(FULL, mbar_wait(q_full, 0));
-    int plo_next = my_kt_last >= 0 ? tile_plo(t, my_kt_last) : P;
+    int plo_next = 0;
+    if (my_kt_last >= 0) advance_plo(t, my_kt_last, plo_next); else plo_next = P;
     if (ok && my_kt_last >= 0) write_masked_q(plo_next);
     __syncwarp();
     if (lane == 0) mbar_arrive(qm_init(t));
@@ -345,11 +351,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (lane == 0) mbar_arrive(k_empty(s));
         continue;
       }
-      const int64_t kp0 = p.k_pos0 + (int64_t)kBN * kt;
-      const int64_t d_row = i_pos - kp0;     // distance to the tile's first key
+      const int kp0 = kBN * kt;
+      const int d_row = i_pos - kp0;         // distance to the tile's first key
       const int plo = plo_next;
       const bool all_pruned = plo >= P;
-      if (kt > 0) plo_next = tile_plo(t, kt - 1);
+      if (kt > 0) advance_plo(t, kt - 1, plo_next);
 
       if (!__all_sync(FULL, mbar_wait(s_full(t), cnt & 1))) { ok = false; break; }
       tc_fence_after();
@@ -367,7 +373,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           // whole groups of 8 pairs share a threshold: one 16-dim dot product per element
 #pragma unroll 1
           for (int gp = plo; gp < pc_hi; gp += 8) {
-            const int64_t lim0 = d_row - p.T[gp];         // columns c < lim0: d > T_group
+            const int lim0 = d_row - p.T[gp];             // columns c < lim0: d > T_group
             if (!__any_sync(FULL, lim0 > 0)) continue;
             const int off_lo = (gp >> 3) * PANEL;
             const int off_hi = (P / 8 + (gp >> 3)) * PANEL;
@@ -386,8 +392,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             }
 #pragma unroll 1
             for (int cc = 0; cc < kBN / 32; ++cc) {
-              const int64_t l64 = lim0 - 32 * cc;
-              const int lim = (int)(l64 < 0 ? 0 : (l64 > 32 ? 32 : l64));
+              const int lim = min(max(lim0 - 32 * cc, 0), 32);
               if (!__any_sync(FULL, lim > 0)) continue;
               float v[32];
               tmem_ld32(tS + 32 * cc, v);
@@ -414,15 +419,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll 1
           for (int cc = 0; cc < kBN / 32; ++cc) {
             // thresholds grow with the pair index: pair plo reaches furthest into the tile
-            const int64_t first = d_row - p.T[plo] - 32 * cc;
+            const int first = d_row - p.T[plo] - 32 * cc;
             if (!__any_sync(FULL, first > 0)) break;
             float v[32];
             tmem_ld32(tS + 32 * cc, v);
             tmem_ld_wait();
 #pragma unroll 1
             for (int pp = plo; pp < pc_hi; ++pp) {
-              const int64_t lim64 = d_row - p.T[pp] - 32 * cc;  // columns c < lim: d > T_pp
-              const int lim = (int)(lim64 < 0 ? 0 : (lim64 > 32 ? 32 : lim64));
+              const int lim = min(max(d_row - p.T[pp] - 32 * cc, 0), 32);  // columns c < lim: d > T_pp
               if (!__any_sync(FULL, lim > 0)) break;
               const int off_lo = (pp >> 3) * PANEL + (pp & 7) * 2;
               const int off_hi = (P / 8 + (pp >> 3)) * PANEL + (pp & 7) * 2;
@@ -457,69 +461,42 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
 
       // causal mask (d < 0) and the ragged key tail: columns c > cm
-      const bool need_mask = (i_tile0 - (kp0 + kBN - 1) < 0) || ((int64_t)kBN * kt + kBN > p.Nk);
+      const bool need_mask = (i_tile0 - (kp0 + kBN - 1) < 0) || (kp0 + kBN > p.Nk);
       int cm = kBN - 1;
       if (need_mask) {
-        int64_t cmax = d_row;                                      // last column with d >= 0
-        const int64_t cnk = (int64_t)p.Nk - 1 - (int64_t)kBN * kt; // last real key
-        if (cnk < cmax) cmax = cnk;
-        cm = (int)(cmax < -1 ? -1 : (cmax > kBN ? kBN : cmax));
+        // last column with d >= 0, and the last real key
+        cm = min(max(min(d_row, p.Nk - 1 - kp0), -1), kBN);
 #pragma unroll
         for (int c = 0; c < kBN; ++c)
           if (c > cm) sc[c] = -INFINITY;
       }
 
-      // row max: 16 independent 3-input max chains, then a tree
-      float a16[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k)
-        a16[k] = max3(max3(sc[8 * k], sc[8 * k + 1], sc[8 * k + 2]),
-                      max3(sc[8 * k + 3], sc[8 * k + 4], sc[8 * k + 5]),
-                      fmaxf(sc[8 * k + 6], sc[8 * k + 7]));
-      float b6[6];
-#pragma unroll
-      for (int k = 0; k < 5; ++k) b6[k] = max3(a16[3 * k], a16[3 * k + 1], a16[3 * k + 2]);
-      b6[5] = a16[15];
-      float mt = max3(max3(b6[0], b6[1], b6[2]), max3(b6[3], b6[4], b6[5]), -INFINITY);
-      mt *= p.scale_log2;
-
-      // lazy rescale: move the reference only when the max grew by > 8 (x256).
-      // s_full of this tile implies the previous PV of this tile has completed.
-      float f = 1.f;
-      bool resc = false;
-      if (cnt == 0) {
-        m_ref = mt;
-      } else if (mt > m_ref + 8.f) {
-        f = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mt);
-        m_ref = mt;
-        resc = true;
-      }
-      if (__any_sync(FULL, resc)) {
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          float o[32];
-          tmem_ld32(tO + 32 * cc, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= f;
-          tmem_st32(tO + 32 * cc, o);
-        }
-      }
-      l_run *= f;
-
-      // p = 2^(s * scale * log2 e - m): exponents two at a time, part of them
-      // on the FMA pipe; masked columns get exactly 0.
-      const float nm = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      // Row max first, then the exponentials against the (lazily moved) reference.
       const float sl = p.scale_log2;
-      float acc[8];
+      auto tile_max = [&]() -> float {
+        float a16[16];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+        for (int k = 0; k < 16; ++k)
+          a16[k] = max3(max3(sc[8 * k], sc[8 * k + 1], sc[8 * k + 2]),
+                        max3(sc[8 * k + 3], sc[8 * k + 4], sc[8 * k + 5]),
+                        fmaxf(sc[8 * k + 6], sc[8 * k + 7]));
+        float b6[6];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+        for (int k = 0; k < 5; ++k) b6[k] = max3(a16[3 * k], a16[3 * k + 1], a16[3 * k + 2]);
+        b6[5] = a16[15];
+        return max3(max3(b6[0], b6[1], b6[2]), max3(b6[3], b6[4], b6[5]), -INFINITY) * sl;
+      };
+      // p for every column against reference m, packed to bf16 pairs in pk;
+      // returns the row sum of p
+      uint32_t pk[kBN / 2];
+      auto exps = [&](float m) -> float {
+        const float nm = (m == -INFINITY) ? 0.f : -m;
+        float acc[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int c = 64 * half + 2 * i;
+        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+#pragma unroll
+        for (int i = 0; i < kBN / 2; ++i) {
+          const int c = 2 * i;
           float x0, x1, e0, e1;
           fma2(x0, x1, sc[c], sc[c + 1], sl, sl, nm, nm);
           if ((i & 7) >= 8 - L::NPOLY) {
@@ -531,9 +508,34 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           add2(acc[2 * (i & 3)], acc[2 * (i & 3) + 1], acc[2 * (i & 3)], acc[2 * (i & 3) + 1], e0, e1);
           pk[i] = pack_bf16x2(e0, e1);
         }
-        tmem_st32u(tS + 32 * half, pk);
+        return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      };
+
+      const float mt = tile_max();
+      // lazy rescale: move the reference only when the max grew by > 8 (x256).
+      // s_full of this tile implies the previous PV of this tile has completed.
+      float f = 1.f;
+      if (cnt == 0) {
+        m_ref = mt;
+      } else if (mt > m_ref + 8.f) {
+        f = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mt);
+        m_ref = mt;
       }
-      l_run += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      if (cnt > 0 && __any_sync(FULL, f != 1.f)) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          float o[32];
+          tmem_ld32(tO + 32 * cc, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= f;
+          tmem_st32(tO + 32 * cc, o);
+        }
+      }
+      const float rowsum = exps(m_ref);
+      l_run = l_run * f + rowsum;
+      tmem_st32u(tS, &pk[0]);       // P overwrites the first 64 columns of S
+      tmem_st32u(tS + 32, &pk[32]);
       // the next tile's masked Q step, before P is released to the MMA warp
       if (kt > 0) write_masked_q(plo_next);
       tmem_st_wait();
