@@ -114,24 +114,41 @@ int launch_prefill(const void* q, const void* k, const void* v, const PrefillPar
 }
 
 template <int D, int GC>
-int launch_decode_split(const DecodeParams& prm, cudaStream_t st) {
+int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& prm,
+                        cudaStream_t st) {
+  constexpr int smem = DecodeSmem<D>::ALLOC;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WPATTN_ECUDA;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(decode_split_kernel<D, GC>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return WPATTN_ECUDA;
+    attr_set[dev] = true;
+  }
   dim3 grid(prm.S, prm.Hkv * prm.hchunks, prm.B);
-  decode_split_kernel<D, GC><<<grid, kDecodeThreads, 0, st>>>(prm);
+  decode_split_kernel<D, GC><<<grid, (decode_compute_warps(GC) + 1) * 32, smem, st>>>(tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
 template <int D>
 int launch_decode(const DecodeParams& prm, int gc, cudaStream_t st) {
   int rc;
+  CUtensorMap tk, tv;
+  // caches are [B, Lmax, Hkv, D]: dims (fastest first) D, Lmax, Hkv, B; 64-dim x 32-key boxes
+  if ((rc = encode_bf16_4d(&tk, prm.k, D, prm.Lmax, prm.Hkv, prm.B, 64, DecodeSmem<D>::KB, true)) != WPATTN_OK)
+    return rc;
+  if ((rc = encode_bf16_4d(&tv, prm.v, D, prm.Lmax, prm.Hkv, prm.B, 64, DecodeSmem<D>::KB, true)) != WPATTN_OK)
+    return rc;
   switch (gc) {
-    case 1: rc = launch_decode_split<D, 1>(prm, st); break;
-    case 2: rc = launch_decode_split<D, 2>(prm, st); break;
-    case 3: rc = launch_decode_split<D, 3>(prm, st); break;
-    case 4: rc = launch_decode_split<D, 4>(prm, st); break;
-    case 5: rc = launch_decode_split<D, 5>(prm, st); break;
-    case 6: rc = launch_decode_split<D, 6>(prm, st); break;
-    case 7: rc = launch_decode_split<D, 7>(prm, st); break;
-    case 8: rc = launch_decode_split<D, 8>(prm, st); break;
+    case 1: rc = launch_decode_split<D, 1>(tk, tv, prm, st); break;
+    case 2: rc = launch_decode_split<D, 2>(tk, tv, prm, st); break;
+    case 3: rc = launch_decode_split<D, 3>(tk, tv, prm, st); break;
+    case 4: rc = launch_decode_split<D, 4>(tk, tv, prm, st); break;
+    case 5: rc = launch_decode_split<D, 5>(tk, tv, prm, st); break;
+    case 6: rc = launch_decode_split<D, 6>(tk, tv, prm, st); break;
+    case 7: rc = launch_decode_split<D, 7>(tk, tv, prm, st); break;
+    case 8: rc = launch_decode_split<D, 8>(tk, tv, prm, st); break;
     default: return WPATTN_EUNSUPPORTED;
   }
   if (rc != WPATTN_OK) return rc;
