@@ -10,11 +10,12 @@
 // (batch, query head); both walk the same key tiles from the diagonal
 // outwards, so every K and V tile is loaded once for 256 rows.  Warp roles:
 //   warps 0-3, 4-7  softmax of query tile 0 / 1: row r of a tile is TMEM lane
-//              r.  They read S from TMEM, subtract the pairs that are pruned
-//              at some but not all distances of the tile, mask, run the
-//              online softmax with a lazily rescaled O, write P (bf16) back
-//              into TMEM over S, and finish with O / l.  The two groups
-//              alternate with the tensor core (ping-pong).
+//              r.  They correct the pairs that are kept at some but not all
+//              distances of the tile (adding those left out of the
+//              contraction, subtracting those contracted but pruned), read S
+//              from TMEM, mask, run the online softmax with a lazily rescaled
+//              O, write P (bf16) back into TMEM over S, and finish with O / l.
+//              The two groups alternate with the tensor core (ping-pong).
 //   warp 8     TMA producer: both Q tiles once, then K and V tiles into a ring.
 //   warp 9     MMA issuer (one lane): S_t = Q_t K^T over the active k-steps,
 //              O_t += P_t V with P_t read from TMEM; owns the TMEM allocation.
@@ -49,6 +50,7 @@ constexpr int kPrefillThreads = 384;  // 8 softmax warps + producer + MMA + 2 id
 // 256 x 224 + 128 x 56 = 64512.
 constexpr uint32_t kRegsSoftmax = 224;
 constexpr uint32_t kRegsOther = 56;
+constexpr int kCT = 16;               // pairs per batch of the per-warp K transpose (g = 1)
 
 struct PrefillParams {
   uint16_t* out;      // [B, Nq, Hq, D] bf16
@@ -70,7 +72,9 @@ struct PrefillSmem {
   static constexpr int OFF_K = OFF_Q + kQT * TILE;
   static constexpr int OFF_V = OFF_K + NS * TILE;
   static constexpr int OFF_QM = OFF_V + NS * TILE;        // masked first k-step of Q, per tile
-  static constexpr int OFF_BAR = OFF_QM + kQT * 2 * kBM * 16;
+  static constexpr int OFF_CT = OFF_QM + kQT * 2 * kBM * 16;  // per-warp transposed K pairs
+  static constexpr int OFF_T = OFF_CT + 8 * kCT * 32 * 4;     // thresholds (64 x int32)
+  static constexpr int OFF_BAR = OFF_T + 64 * 4;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
   //           s_full[2], p_full[2], o_final[2], qm_init[2]
   static constexpr int NBAR = 1 + 4 * NS + 8;
@@ -78,15 +82,6 @@ struct PrefillSmem {
   static constexpr int BYTES = OFF_TMEM + 16;
   static constexpr int ALLOC = BYTES;
 };
-
-__device__ __forceinline__ int dev_pmin(const int* T, int P, int d) {
-  int lo = 0, hi = P;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (T[mid] < d) lo = mid + 1; else hi = mid;
-  }
-  return lo;
-}
 
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
                                         uint32_t idesc, uint32_t accumulate) {
@@ -126,6 +121,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   auto qm_init = [&](int t) { return bar + 8 * (7 + 4 * NS + t); };
 
   const uint32_t sQM = sbase + L::OFF_QM;
+  int* sT = reinterpret_cast<int*>(smem + L::OFF_T);  // per-pair thresholds, read by every role
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
 
   // the 128-byte-swizzled V tiles need a 1024-byte aligned shared window
@@ -155,9 +151,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // tile (p_min of that distance) only moves forward: advance it in place.
   auto advance_plo = [&](int t, int kt, int& plo) {
     const int dlo = p.qk_off + (kQT * cq + t) * kBM - (kBN * kt + kBN - 1);
-    while (plo < P && p.T[plo] < dlo) ++plo;
+    while (plo < P && sT[plo] < dlo) ++plo;
+  };
+  // Split pair of the tile: pairs plo .. ps-1 (kept somewhere in the tile) are
+  // left out of the contraction and added back where they are kept; pairs
+  // ps .. P-1 are contracted and subtracted where they are pruned.  Splitting
+  // at the pair first kept 32 past the tile's centre distance keeps both
+  // correction sets small (each element only pays for pairs whose threshold
+  // lies between its distance and the centre).  Groups of 8 pairs share a
+  // threshold, so for g = 8 the split falls on a group start.
+  // The centre distance grows along the walk, so the first pair kept past it
+  // (psr, carried by the caller) is advanced in place like plo.
+  auto split_pair = [&](int t, int kt, int plo, int& psr) -> int {
+    if (plo >= P) return plo;
+    const int dc = max(p.qk_off + (kQT * cq + t) * kBM - kBN * kt, 0);  // row 0 to key 0
+    const int target = dc > 0x7FFFFFDF ? 0x7FFFFFFF : dc + 32;
+    while (psr < P && sT[psr] < target) ++psr;
+    return min(max(psr, plo), P - (p.g8 ? 8 : 1));
   };
 
+  if (threadIdx.x < 64) sT[threadIdx.x] = p.T[threadIdx.x];
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < NS; ++s) {
@@ -222,29 +235,33 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = mbar_wait(q_full, 0);
       int cnt0 = 0, cnt1 = 0;  // tiles processed so far by query tile 0 / 1
       bool qm_seen0 = false, qm_seen1 = false;
-      int plo0 = 0, plo1 = 0;
+      int plo0 = 0, plo1 = 0, psr0 = 0, psr1 = 0;
       // descriptors: start addresses advance by adding (byte offset >> 4)
       const uint64_t qdesc0 = make_sdesc(sQ, LBO_QK, 128, 0);
       const uint64_t qmdesc0 = make_sdesc(sQM, PANEL, 128, 0);
       const uint64_t kdesc0 = make_sdesc(sK, LBO_QK, 128, 0);
       const uint64_t vdesc0 = make_sdesc(sV, kBN * 128, 1024, 2);
-      auto issue_qk = [&](int t, int j) -> bool {
+      // split pair of QK_t(j): planned ahead of the wait for P_t(j - 1)
+      auto plan_qk = [&](int t, int j) -> int {
+        const int kt = kt_top - j;
+        int& plo = t ? plo1 : plo0;
+        advance_plo(t, kt, plo);
+        return split_pair(t, kt, plo, t ? psr1 : psr0);
+      };
+      auto issue_qk = [&](int t, int j, int ps) -> bool {
         bool& seen = t ? qm_seen1 : qm_seen0;
         if (!seen) {  // the softmax warps prepared the masked k-step of tile t's first tile
           if (!mbar_wait(qm_init(t), 0)) return false;
           seen = true;
         }
-        const int kt = kt_top - j;
-        int& plo = t ? plo1 : plo0;
-        advance_plo(t, kt, plo);
-        const int k0 = plo >> 3;
+        const int k0 = ps >> 3;
         const uint64_t kbase = kdesc0 + (uint64_t)(((j % NS) * L::TILE) >> 4);
         const uint64_t qbase = qdesc0 + (uint64_t)((t * L::TILE) >> 4);
         const uint32_t d_tmem = tmem + t * kBN;
         for (int ks = k0; ks < KS; ++ks) {
-          // pairs 8*k0 .. plo-1 are pruned everywhere in the tile: the first
-          // step reads a copy of Q with those pairs zeroed
-          const uint64_t ad = (ks == k0 && (plo & 7))
+          // pairs 8*k0 .. ps-1 are not contracted: the first step reads a
+          // copy of Q with those pairs zeroed
+          const uint64_t ad = (ks == k0 && (ps & 7))
                                   ? qmdesc0 + (uint64_t)((t * 2 * PANEL) >> 4)
                                   : qbase + (uint64_t)((ks * PANEL) >> 4);
           umma_ss(d_tmem, ad, kbase + (uint64_t)((ks * PANEL) >> 4), idesc_qk, ks > k0 ? 1u : 0u);
@@ -254,8 +271,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       };
       if (ok && mbar_wait(k_full(0), 0)) {
         tc_fence_after();
-        if (kt_last0 >= kt_top && !issue_qk(0, 0)) ok = false;
-        if (ok && kt_last1 >= kt_top && !issue_qk(1, 0)) ok = false;
+        if (kt_last0 >= kt_top && !issue_qk(0, 0, plan_qk(0, 0))) ok = false;
+        if (ok && kt_last1 >= kt_top && !issue_qk(1, 0, plan_qk(1, 0))) ok = false;
         umma_commit(k_empty(0));
       } else {
         ok = false;
@@ -270,6 +287,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int t = 0; t < kQT; ++t) {
           const int ktl = t ? kt_last1 : kt_last0;
           int& cnt = t ? cnt1 : cnt0;
+          const bool do_qk = ok && next && kt - 1 <= ktl;
+          const int ps_n = do_qk ? plan_qk(t, j + 1) : 0;
           if (ok && kt <= ktl) {
             if (!mbar_wait(p_full(t), cnt & 1)) { ok = false; }
             if (ok) {
@@ -281,7 +300,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               ++cnt;
             }
           }
-          if (ok && next && kt - 1 <= ktl && !issue_qk(t, j + 1)) ok = false;
+          if (ok && do_qk && !issue_qk(t, j + 1, ps_n)) ok = false;
         }
         if (!ok) break;
         umma_commit(v_empty(j % NS));
@@ -312,14 +331,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     int cnt = 0;
     bool ok = true;
 
-    // Copy of Q's first active k-step for a key tile whose first kept pair is
-    // plo, with the pairs that are pruned over the whole tile zeroed (the MMA
-    // reads it instead of Q).
-    auto write_masked_q = [&](int plo) {
-      const int rz = plo & 7;
-      if (rz == 0 || (plo >> 3) >= KS) return;
-      uint4 lo = *reinterpret_cast<const uint4*>(smem_q + (plo >> 3) * PANEL + r * 16);
-      uint4 hi = *reinterpret_cast<const uint4*>(smem_q + (P / 8 + (plo >> 3)) * PANEL + r * 16);
+    // Copy of Q's first contracted k-step for a key tile whose split pair is
+    // ps, with the pairs below ps zeroed (the MMA reads it instead of Q).
+    auto write_masked_q = [&](int ps) {
+      const int rz = ps & 7;
+      if (rz == 0 || (ps >> 3) >= KS) return;
+      uint4 lo = *reinterpret_cast<const uint4*>(smem_q + (ps >> 3) * PANEL + r * 16);
+      uint4 hi = *reinterpret_cast<const uint4*>(smem_q + (P / 8 + (ps >> 3)) * PANEL + r * 16);
       const uint32_t m0 = (rz > 0 ? 0u : 0xFFFFu) | (rz > 1 ? 0u : 0xFFFF0000u);
       const uint32_t m1 = (rz > 2 ? 0u : 0xFFFFu) | (rz > 3 ? 0u : 0xFFFF0000u);
       const uint32_t m2 = (rz > 4 ? 0u : 0xFFFFu) | (rz > 5 ? 0u : 0xFFFF0000u);
@@ -335,7 +353,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     ok = __all_sync(FULL, mbar_wait(q_full, 0));
     int plo_next = 0;
     if (my_kt_last >= 0) advance_plo(t, my_kt_last, plo_next); else plo_next = P;
-    if (ok && my_kt_last >= 0) write_masked_q(plo_next);
+    int psr = 0;
+    int ps_next = my_kt_last >= 0 ? split_pair(t, my_kt_last, plo_next, psr) : P;
+    if (ok && my_kt_last >= 0) write_masked_q(ps_next);
     __syncwarp();
     if (lane == 0) mbar_arrive(qm_init(t));
 
@@ -353,50 +373,81 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       const int kp0 = kBN * kt;
       const int d_row = i_pos - kp0;         // distance to the tile's first key
-      const int plo = plo_next;
+      const int plo = plo_next, ps = ps_next;
       const bool all_pruned = plo >= P;
-      if (kt > 0) advance_plo(t, kt - 1, plo_next);
+      if (kt > 0) {
+        advance_plo(t, kt - 1, plo_next);
+        ps_next = split_pair(t, kt - 1, plo_next, psr);
+      }
 
-      if (!__all_sync(FULL, mbar_wait(s_full(t), cnt & 1))) { ok = false; break; }
-      tc_fence_after();
-
-      // Pairs plo .. p_min(d)-1 are kept at some distances of the tile and
-      // pruned at this element's: subtract their terms (per element).  Pair
-      // plo is pruned somewhere in this row iff the row's largest distance
-      // exceeds its threshold.
-      if (!all_pruned && __any_sync(FULL, d_row > p.T[plo])) {
-        const int pm_row = d_row > 0 ? dev_pmin(p.T, P, d_row) : 0;
-        const int pc_hi = __reduce_max_sync(FULL, pm_row);
-        if (!__all_sync(FULL, mbar_wait(k_full(s), (j / NS) & 1))) { ok = false; break; }
+      // Per-element corrections, d = d_row - c for column c of the tile:
+      //   pairs plo .. ps-1 were left out of the contraction: add their terms
+      //   where they are kept (0 <= d <= T);
+      //   pairs ps .. P-1 were contracted: subtract their terms where they
+      //   are pruned (d > T).  Thresholds grow with the pair index.
+      // They depend on Q and K only, so they are summed into sc while the
+      // tensor core is still computing S; S is added once it is ready.
+      const bool need_sub = !all_pruned && __any_sync(FULL, d_row > sT[ps]);
+      const bool need_add = !all_pruned && ps > plo &&
+                            __any_sync(FULL, d_row >= 0 && d_row - (kBN - 1) <= sT[ps - 1]);
+      const bool corr = need_sub || need_add;
+      // K stage s is released below; waiting for its fill first makes the
+      // arrival count towards iteration j (the stage's previous phase is over)
+      if (!__all_sync(FULL, mbar_wait(k_full(s), (j / NS) & 1))) { ok = false; break; }
+      float sc[kBN];
+      if (corr) {
         const uint8_t* kb = smem + L::OFF_K + s * L::TILE;
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) sc[c] = 0.f;
+        // the chunk loops are not unrolled (this path runs on few tiles and
+        // must stay small in the instruction cache): a chunk's terms are
+        // summed into dl and added to sc by a switch on the chunk index
+#define WPATTN_ADD_CHUNK(K)                                                  \
+  case K:                                                                    \
+    _Pragma("unroll") for (int c = 0; c < 32; ++c) sc[32 * K + c] += dl[c]; \
+    break;
         if (p.g8) {
           // whole groups of 8 pairs share a threshold: one 16-dim dot product per element
 #pragma unroll 1
-          for (int gp = plo; gp < pc_hi; gp += 8) {
-            const int lim0 = d_row - p.T[gp];             // columns c < lim0: d > T_group
-            if (!__any_sync(FULL, lim0 > 0)) continue;
-            const int off_lo = (gp >> 3) * PANEL;
-            const int off_hi = (P / 8 + (gp >> 3)) * PANEL;
-            float qv[16];
-            {
-              const uint4 a = *reinterpret_cast<const uint4*>(smem_q + off_lo + r * 16);
-              const uint4 c = *reinterpret_cast<const uint4*>(smem_q + off_hi + r * 16);
-              qv[0] = bf16lo_to_f32(a.x); qv[1] = bf16hi_to_f32(a.x);
-              qv[2] = bf16lo_to_f32(a.y); qv[3] = bf16hi_to_f32(a.y);
-              qv[4] = bf16lo_to_f32(a.z); qv[5] = bf16hi_to_f32(a.z);
-              qv[6] = bf16lo_to_f32(a.w); qv[7] = bf16hi_to_f32(a.w);
-              qv[8] = bf16lo_to_f32(c.x); qv[9] = bf16hi_to_f32(c.x);
-              qv[10] = bf16lo_to_f32(c.y); qv[11] = bf16hi_to_f32(c.y);
-              qv[12] = bf16lo_to_f32(c.z); qv[13] = bf16hi_to_f32(c.z);
-              qv[14] = bf16lo_to_f32(c.w); qv[15] = bf16hi_to_f32(c.w);
-            }
+          for (int cc = 0; cc < kBN / 32; ++cc) {
+            const int dc = d_row - 32 * cc;  // distance at the chunk's first column
+            float dl[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) dl[c] = 0.f;
+            bool any = false;
 #pragma unroll 1
-            for (int cc = 0; cc < kBN / 32; ++cc) {
-              const int lim = min(max(lim0 - 32 * cc, 0), 32);
-              if (!__any_sync(FULL, lim > 0)) continue;
-              float v[32];
-              tmem_ld32(tS + 32 * cc, v);
-              tmem_ld_wait();
+            for (int gp = plo; gp < P; gp += 8) {
+              const bool sub = gp >= ps;
+              const int T = sT[gp];
+              int lo, hi;  // chunk columns of this row that take the group's term
+              if (sub) {
+                lo = 0;
+                hi = dc > T ? min(dc - T, 32) - 1 : -1;
+              } else {
+                lo = T >= dc ? 0 : dc - T;
+                hi = min(dc, 31);
+              }
+              if (!__any_sync(FULL, lo <= hi)) {
+                if (sub) break;  // later groups are pruned at even fewer columns
+                continue;
+              }
+              any = true;
+              const float sgn = sub ? -1.f : 1.f;
+              const int off_lo = (gp >> 3) * PANEL;
+              const int off_hi = (P / 8 + (gp >> 3)) * PANEL;
+              float qv[16];
+              {
+                const uint4 a = *reinterpret_cast<const uint4*>(smem_q + off_lo + r * 16);
+                const uint4 c = *reinterpret_cast<const uint4*>(smem_q + off_hi + r * 16);
+                qv[0] = bf16lo_to_f32(a.x) * sgn; qv[1] = bf16hi_to_f32(a.x) * sgn;
+                qv[2] = bf16lo_to_f32(a.y) * sgn; qv[3] = bf16hi_to_f32(a.y) * sgn;
+                qv[4] = bf16lo_to_f32(a.z) * sgn; qv[5] = bf16hi_to_f32(a.z) * sgn;
+                qv[6] = bf16lo_to_f32(a.w) * sgn; qv[7] = bf16hi_to_f32(a.w) * sgn;
+                qv[8] = bf16lo_to_f32(c.x) * sgn; qv[9] = bf16hi_to_f32(c.x) * sgn;
+                qv[10] = bf16lo_to_f32(c.y) * sgn; qv[11] = bf16hi_to_f32(c.y) * sgn;
+                qv[12] = bf16lo_to_f32(c.z) * sgn; qv[13] = bf16hi_to_f32(c.z) * sgn;
+                qv[14] = bf16lo_to_f32(c.w) * sgn; qv[15] = bf16hi_to_f32(c.w) * sgn;
+              }
 #pragma unroll
               for (int c = 0; c < 32; ++c) {
                 const uint4 a = *reinterpret_cast<const uint4*>(kb + off_lo + (32 * cc + c) * 16);
@@ -410,51 +461,117 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 fma2(d0, d1, qv[10], qv[11], bf16lo_to_f32(b2.y), bf16hi_to_f32(b2.y), d0, d1);
                 fma2(d0, d1, qv[12], qv[13], bf16lo_to_f32(b2.z), bf16hi_to_f32(b2.z), d0, d1);
                 fma2(d0, d1, qv[14], qv[15], bf16lo_to_f32(b2.w), bf16hi_to_f32(b2.w), d0, d1);
-                if (c < lim) v[c] -= d0 + d1;
+                if (c >= lo && c <= hi) dl[c] += d0 + d1;
               }
-              tmem_st32(tS + 32 * cc, v);
+            }
+            if (any) {
+              switch (cc) {
+                WPATTN_ADD_CHUNK(0)
+                WPATTN_ADD_CHUNK(1)
+                WPATTN_ADD_CHUNK(2)
+                WPATTN_ADD_CHUNK(3)
+              }
             }
           }
         } else {
+          // One pair per term.  For each 32-column chunk the warp first
+          // transposes the K values of the pairs its 32 x 32 block needs into
+          // a private buffer (lane k writes key 32 cc + k), so that the
+          // column loop reads four keys per broadcast load.
+          uint32_t* ct = reinterpret_cast<uint32_t*>(smem + L::OFF_CT) + warp * (kCT * 32);
+          const int T_lo = ps > plo ? sT[ps - 1] : 0;
 #pragma unroll 1
           for (int cc = 0; cc < kBN / 32; ++cc) {
-            // thresholds grow with the pair index: pair plo reaches furthest into the tile
-            const int first = d_row - p.T[plo] - 32 * cc;
-            if (!__any_sync(FULL, first > 0)) break;
-            float v[32];
-            tmem_ld32(tS + 32 * cc, v);
-            tmem_ld_wait();
-#pragma unroll 1
-            for (int pp = plo; pp < pc_hi; ++pp) {
-              const int lim = min(max(d_row - p.T[pp] - 32 * cc, 0), 32);  // columns c < lim: d > T_pp
-              if (!__any_sync(FULL, lim > 0)) break;
-              const int off_lo = (pp >> 3) * PANEL + (pp & 7) * 2;
-              const int off_hi = (P / 8 + (pp >> 3)) * PANEL + (pp & 7) * 2;
-              const float qa = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + off_lo + r * 16)) << 16);
-              const float qb = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + off_hi + r * 16)) << 16);
-              const uint8_t* klo = kb + off_lo + cc * 32 * 16;
-              const uint8_t* khi = kb + off_hi + cc * 32 * 16;
+            const int dc = d_row - 32 * cc;                  // distance at the chunk's first column
+            const int dmax = __shfl_sync(FULL, dc, 31);      // largest distance of the block
+            const int dmin = max(__shfl_sync(FULL, dc, 0) - 31, 0);
+            if (dmax < 0) continue;                          // wholly acausal
+            // pairs ps .. pb-1 are pruned somewhere in the block, pa .. ps-1 kept somewhere
+            int pb = ps;
+            if (need_sub)
+              while (pb < P && sT[pb] < dmax) ++pb;
+            int pa = ps;
+            if (need_add && T_lo >= dmin)
+              while (pa > plo && sT[pa - 1] >= dmin) --pa;
+            if (pa >= pb) continue;
+            float dl[32];
 #pragma unroll
-              for (int c = 0; c < 32; ++c) {
-                if (c < lim) {
-                  const float ka = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(klo + c * 16)) << 16);
-                  const float kb2 = __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(khi + c * 16)) << 16);
-                  v[c] -= fmaf(qa, ka, qb * kb2);
+            for (int c = 0; c < 32; ++c) dl[c] = 0.f;
+#pragma unroll 1
+            for (int p0 = pa; p0 < pb; p0 += kCT) {
+              const int p1 = min(pb, p0 + kCT);
+              __syncwarp();  // the previous batch has been read
+              const uint8_t* krow = kb + (32 * cc + lane) * 16;
+#pragma unroll 1
+              for (int pp = p0; pp < p1; ++pp) {
+                const int o = (pp >> 3) * PANEL + (pp & 7) * 2;
+                const uint32_t klo = *reinterpret_cast<const uint16_t*>(krow + o);
+                const uint32_t khi = *reinterpret_cast<const uint16_t*>(krow + o + (P / 8) * PANEL);
+                ct[(pp - p0) * 32 + lane] = klo | (khi << 16);
+              }
+              __syncwarp();
+#pragma unroll 1
+              for (int pp = p0; pp < p1; ++pp) {
+                const int T = sT[pp];
+                int lo, hi;  // chunk columns of this row that take the pair's term
+                float sgn;
+                if (pp >= ps) {
+                  lo = 0;
+                  hi = dc > T ? min(dc - T, 32) - 1 : -1;
+                  sgn = -1.f;
+                } else {
+                  lo = T >= dc ? 0 : dc - T;
+                  hi = min(dc, 31);
+                  sgn = 1.f;
+                }
+                const int o = (pp >> 3) * PANEL + (pp & 7) * 2 + r * 16;
+                const float qa = sgn * __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + o)) << 16);
+                const float qb = sgn * __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + o + (P / 8) * PANEL)) << 16);
+                const uint4* w4 = reinterpret_cast<const uint4*>(ct + (pp - p0) * 32);
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4) {
+                  const uint4 w = w4[c4];
+                  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const int c = 4 * c4 + e;
+                    const float ka = __uint_as_float(ww[e] << 16);
+                    const float kh = __uint_as_float(ww[e] & 0xFFFF0000u);
+                    if (c >= lo && c <= hi) dl[c] = fmaf(qa, ka, fmaf(qb, kh, dl[c]));
+                  }
                 }
               }
             }
-            tmem_st32(tS + 32 * cc, v);
+            switch (cc) {
+              WPATTN_ADD_CHUNK(0)
+              WPATTN_ADD_CHUNK(1)
+              WPATTN_ADD_CHUNK(2)
+              WPATTN_ADD_CHUNK(3)
+            }
           }
         }
-        tmem_st_wait();
+#undef WPATTN_ADD_CHUNK
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(k_empty(s));
 
-      float sc[kBN];
+      if (!__all_sync(FULL, mbar_wait(s_full(t), cnt & 1))) { ok = false; break; }
+      tc_fence_after();
+      if (corr) {
 #pragma unroll
-      for (int cc = 0; cc < kBN / 32; ++cc) tmem_ld32(tS + 32 * cc, &sc[32 * cc]);
-      tmem_ld_wait();
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          float v[32];
+          tmem_ld32(tS + 32 * cc, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) sc[32 * cc + c] += v[c];
+        }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < kBN / 32; ++cc) tmem_ld32(tS + 32 * cc, &sc[32 * cc]);
+        tmem_ld_wait();
+      }
+
       if (all_pruned) {
 #pragma unroll
         for (int c = 0; c < kBN; ++c) sc[c] = 0.f;   // every pair pruned: score 0
@@ -537,7 +654,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_st32u(tS, &pk[0]);       // P overwrites the first 64 columns of S
       tmem_st32u(tS + 32, &pk[32]);
       // the next tile's masked Q step, before P is released to the MMA warp
-      if (kt > 0) write_masked_q(plo_next);
+      if (kt > 0) write_masked_q(ps_next);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
