@@ -45,7 +45,7 @@ struct DeviceInfo {
   bool init = false;
   bool supported = false;
   int num_sms = 0;
-  bool prefill_attr[2] = {false, false};
+  bool prefill_attr[4] = {false, false, false, false};  // (D 64, 128) x (g 1, 8)
   void* static_scratch = nullptr;  // device address of g_decode_static_scratch
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -88,7 +88,7 @@ int encode_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
   return r == CUDA_SUCCESS ? WPATTN_OK : WPATTN_ECUDA;
 }
 
-template <int D>
+template <int D, bool G8>
 int launch_prefill(const void* q, const void* k, const void* v, const PrefillParams& prm,
                    DeviceInfo* dev, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
@@ -101,15 +101,15 @@ int launch_prefill(const void* q, const void* k, const void* v, const PrefillPar
   if ((rc = encode_bf16_4d(&tk, k, D, nk, hk, prm.B, 8, kBN, false)) != WPATTN_OK) return rc;
   if ((rc = encode_bf16_4d(&tv, v, D, nk, hk, prm.B, 64, kBN, true)) != WPATTN_OK) return rc;
   constexpr int smem = PrefillSmem<D>::ALLOC;
-  const int slot = (D == 64) ? 0 : 1;
+  const int slot = (D == 64 ? 0 : 2) + (G8 ? 1 : 0);
   if (!dev->prefill_attr[slot]) {
-    if (cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(prefill_kernel<D, G8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
       return WPATTN_ECUDA;
     dev->prefill_attr[slot] = true;
   }
   dim3 grid(prm.num_ctas_q, prm.Hq, prm.B);
-  prefill_kernel<D><<<grid, kPrefillThreads, smem, st>>>(tq, tk, tv, prm);
+  prefill_kernel<D, G8><<<grid, kPrefillThreads, smem, st>>>(tq, tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
@@ -264,8 +264,11 @@ int wpattn_prefill(const wpattn_window* w, const void* q, const void* k, const v
   const void* kk = Nk > 0 ? k : q;
   const void* vv = Nk > 0 ? v : q;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  if (plan.D == 64) return launch_prefill<64>(q, kk, vv, prm, dev, st);
-  return launch_prefill<128>(q, kk, vv, prm, dev, st);
+  if (plan.D == 64)
+    return prm.g8 ? launch_prefill<64, true>(q, kk, vv, prm, dev, st)
+                  : launch_prefill<64, false>(q, kk, vv, prm, dev, st);
+  return prm.g8 ? launch_prefill<128, true>(q, kk, vv, prm, dev, st)
+                : launch_prefill<128, false>(q, kk, vv, prm, dev, st);
 }
 
 size_t wpattn_decode_workspace_size(const wpattn_window* w, int32_t B, int32_t Hq, int32_t Hkv,

@@ -92,7 +92,9 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       : "memory");
 }
 
-template <int D>
+// G8: pairs share thresholds in groups of 8 (a compile-time switch, so the
+// two correction paths do not share a register allocation)
+template <int D, bool G8>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ PrefillParams p) {
@@ -167,7 +169,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int dc = max(p.qk_off + (kQT * cq + t) * kBM - kBN * kt, 0);  // row 0 to key 0
     const int target = dc > 0x7FFFFFDF ? 0x7FFFFFFF : dc + 32;
     while (psr < P && sT[psr] < target) ++psr;
-    return min(max(psr, plo), P - (p.g8 ? 8 : 1));
+    return min(max(psr, plo), P - (G8 ? 8 : 1));
   };
 
   if (threadIdx.x < 64) sT[threadIdx.x] = p.T[threadIdx.x];
@@ -385,8 +387,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       //   where they are kept (0 <= d <= T);
       //   pairs ps .. P-1 were contracted: subtract their terms where they
       //   are pruned (d > T).  Thresholds grow with the pair index.
-      // They depend on Q and K only, so they are summed into sc while the
-      // tensor core is still computing S; S is added once it is ready.
+      // For g = 1 they depend on Q and K only, so they are summed into sc
+      // while the tensor core is still computing S, and S is added once it
+      // is ready; for g = 8 they are applied to S in TMEM before it is read.
       const bool need_sub = !all_pruned && __any_sync(FULL, d_row > sT[ps]);
       const bool need_add = !all_pruned && ps > plo &&
                             __any_sync(FULL, d_row >= 0 && d_row - (kBN - 1) <= sT[ps - 1]);
@@ -395,7 +398,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // arrival count towards iteration j (the stage's previous phase is over)
       if (!__all_sync(FULL, mbar_wait(k_full(s), (j / NS) & 1))) { ok = false; break; }
       float sc[kBN];
-      if (corr) {
+      if (corr && !G8) {
         const uint8_t* kb = smem + L::OFF_K + s * L::TILE;
 #pragma unroll
         for (int c = 0; c < kBN; ++c) sc[c] = 0.f;
@@ -406,158 +409,155 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   case K:                                                                    \
     _Pragma("unroll") for (int c = 0; c < 32; ++c) sc[32 * K + c] += dl[c]; \
     break;
-        if (p.g8) {
-          // whole groups of 8 pairs share a threshold: one 16-dim dot product per element
+        // One pair per term.  For each 32-column chunk the warp first
+        // transposes the K values of the pairs its 32 x 32 block needs into
+        // a private buffer (lane k writes key 32 cc + k), so that the
+        // column loop reads four keys per broadcast load.
+        uint32_t* ct = reinterpret_cast<uint32_t*>(smem + L::OFF_CT) + warp * (kCT * 32);
+        const int T_lo = ps > plo ? sT[ps - 1] : 0;
 #pragma unroll 1
-          for (int cc = 0; cc < kBN / 32; ++cc) {
-            const int dc = d_row - 32 * cc;  // distance at the chunk's first column
-            float dl[32];
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          const int dc = d_row - 32 * cc;                  // distance at the chunk's first column
+          const int dmax = __shfl_sync(FULL, dc, 31);      // largest distance of the block
+          const int dmin = max(__shfl_sync(FULL, dc, 0) - 31, 0);
+          if (dmax < 0) continue;                          // wholly acausal
+          // pairs ps .. pb-1 are pruned somewhere in the block, pa .. ps-1 kept somewhere
+          int pb = ps;
+          if (need_sub)
+            while (pb < P && sT[pb] < dmax) ++pb;
+          int pa = ps;
+          if (need_add && T_lo >= dmin)
+            while (pa > plo && sT[pa - 1] >= dmin) --pa;
+          if (pa >= pb) continue;
+          float dl[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) dl[c] = 0.f;
-            bool any = false;
+          for (int c = 0; c < 32; ++c) dl[c] = 0.f;
 #pragma unroll 1
-            for (int gp = plo; gp < P; gp += 8) {
-              const bool sub = gp >= ps;
-              const int T = sT[gp];
-              int lo, hi;  // chunk columns of this row that take the group's term
-              if (sub) {
+          for (int p0 = pa; p0 < pb; p0 += kCT) {
+            const int p1 = min(pb, p0 + kCT);
+            __syncwarp();  // the previous batch has been read
+            const uint8_t* krow = kb + (32 * cc + lane) * 16;
+#pragma unroll 1
+            for (int pp = p0; pp < p1; ++pp) {
+              const int o = (pp >> 3) * PANEL + (pp & 7) * 2;
+              const uint32_t klo = *reinterpret_cast<const uint16_t*>(krow + o);
+              const uint32_t khi = *reinterpret_cast<const uint16_t*>(krow + o + (P / 8) * PANEL);
+              ct[(pp - p0) * 32 + lane] = klo | (khi << 16);
+            }
+            __syncwarp();
+#pragma unroll 1
+            for (int pp = p0; pp < p1; ++pp) {
+              const int T = sT[pp];
+              int lo, hi;  // chunk columns of this row that take the pair's term
+              float sgn;
+              if (pp >= ps) {
                 lo = 0;
                 hi = dc > T ? min(dc - T, 32) - 1 : -1;
+                sgn = -1.f;
               } else {
                 lo = T >= dc ? 0 : dc - T;
                 hi = min(dc, 31);
+                sgn = 1.f;
               }
-              if (!__any_sync(FULL, lo <= hi)) {
-                if (sub) break;  // later groups are pruned at even fewer columns
-                continue;
-              }
-              any = true;
-              const float sgn = sub ? -1.f : 1.f;
-              const int off_lo = (gp >> 3) * PANEL;
-              const int off_hi = (P / 8 + (gp >> 3)) * PANEL;
-              float qv[16];
-              {
-                const uint4 a = *reinterpret_cast<const uint4*>(smem_q + off_lo + r * 16);
-                const uint4 c = *reinterpret_cast<const uint4*>(smem_q + off_hi + r * 16);
-                qv[0] = bf16lo_to_f32(a.x) * sgn; qv[1] = bf16hi_to_f32(a.x) * sgn;
-                qv[2] = bf16lo_to_f32(a.y) * sgn; qv[3] = bf16hi_to_f32(a.y) * sgn;
-                qv[4] = bf16lo_to_f32(a.z) * sgn; qv[5] = bf16hi_to_f32(a.z) * sgn;
-                qv[6] = bf16lo_to_f32(a.w) * sgn; qv[7] = bf16hi_to_f32(a.w) * sgn;
-                qv[8] = bf16lo_to_f32(c.x) * sgn; qv[9] = bf16hi_to_f32(c.x) * sgn;
-                qv[10] = bf16lo_to_f32(c.y) * sgn; qv[11] = bf16hi_to_f32(c.y) * sgn;
-                qv[12] = bf16lo_to_f32(c.z) * sgn; qv[13] = bf16hi_to_f32(c.z) * sgn;
-                qv[14] = bf16lo_to_f32(c.w) * sgn; qv[15] = bf16hi_to_f32(c.w) * sgn;
-              }
+              const int o = (pp >> 3) * PANEL + (pp & 7) * 2 + r * 16;
+              const float qa = sgn * __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + o)) << 16);
+              const float qb = sgn * __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + o + (P / 8) * PANEL)) << 16);
+              const uint4* w4 = reinterpret_cast<const uint4*>(ct + (pp - p0) * 32);
 #pragma unroll
-              for (int c = 0; c < 32; ++c) {
-                const uint4 a = *reinterpret_cast<const uint4*>(kb + off_lo + (32 * cc + c) * 16);
-                const uint4 b2 = *reinterpret_cast<const uint4*>(kb + off_hi + (32 * cc + c) * 16);
-                float d0 = 0.f, d1 = 0.f;
-                fma2(d0, d1, qv[0], qv[1], bf16lo_to_f32(a.x), bf16hi_to_f32(a.x), d0, d1);
-                fma2(d0, d1, qv[2], qv[3], bf16lo_to_f32(a.y), bf16hi_to_f32(a.y), d0, d1);
-                fma2(d0, d1, qv[4], qv[5], bf16lo_to_f32(a.z), bf16hi_to_f32(a.z), d0, d1);
-                fma2(d0, d1, qv[6], qv[7], bf16lo_to_f32(a.w), bf16hi_to_f32(a.w), d0, d1);
-                fma2(d0, d1, qv[8], qv[9], bf16lo_to_f32(b2.x), bf16hi_to_f32(b2.x), d0, d1);
-                fma2(d0, d1, qv[10], qv[11], bf16lo_to_f32(b2.y), bf16hi_to_f32(b2.y), d0, d1);
-                fma2(d0, d1, qv[12], qv[13], bf16lo_to_f32(b2.z), bf16hi_to_f32(b2.z), d0, d1);
-                fma2(d0, d1, qv[14], qv[15], bf16lo_to_f32(b2.w), bf16hi_to_f32(b2.w), d0, d1);
-                if (c >= lo && c <= hi) dl[c] += d0 + d1;
-              }
-            }
-            if (any) {
-              switch (cc) {
-                WPATTN_ADD_CHUNK(0)
-                WPATTN_ADD_CHUNK(1)
-                WPATTN_ADD_CHUNK(2)
-                WPATTN_ADD_CHUNK(3)
+              for (int c4 = 0; c4 < 8; ++c4) {
+                const uint4 w = w4[c4];
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int c = 4 * c4 + e;
+                  const float ka = __uint_as_float(ww[e] << 16);
+                  const float kh = __uint_as_float(ww[e] & 0xFFFF0000u);
+                  if (c >= lo && c <= hi) dl[c] = fmaf(qa, ka, fmaf(qb, kh, dl[c]));
+                }
               }
             }
           }
-        } else {
-          // One pair per term.  For each 32-column chunk the warp first
-          // transposes the K values of the pairs its 32 x 32 block needs into
-          // a private buffer (lane k writes key 32 cc + k), so that the
-          // column loop reads four keys per broadcast load.
-          uint32_t* ct = reinterpret_cast<uint32_t*>(smem + L::OFF_CT) + warp * (kCT * 32);
-          const int T_lo = ps > plo ? sT[ps - 1] : 0;
-#pragma unroll 1
-          for (int cc = 0; cc < kBN / 32; ++cc) {
-            const int dc = d_row - 32 * cc;                  // distance at the chunk's first column
-            const int dmax = __shfl_sync(FULL, dc, 31);      // largest distance of the block
-            const int dmin = max(__shfl_sync(FULL, dc, 0) - 31, 0);
-            if (dmax < 0) continue;                          // wholly acausal
-            // pairs ps .. pb-1 are pruned somewhere in the block, pa .. ps-1 kept somewhere
-            int pb = ps;
-            if (need_sub)
-              while (pb < P && sT[pb] < dmax) ++pb;
-            int pa = ps;
-            if (need_add && T_lo >= dmin)
-              while (pa > plo && sT[pa - 1] >= dmin) --pa;
-            if (pa >= pb) continue;
-            float dl[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) dl[c] = 0.f;
-#pragma unroll 1
-            for (int p0 = pa; p0 < pb; p0 += kCT) {
-              const int p1 = min(pb, p0 + kCT);
-              __syncwarp();  // the previous batch has been read
-              const uint8_t* krow = kb + (32 * cc + lane) * 16;
-#pragma unroll 1
-              for (int pp = p0; pp < p1; ++pp) {
-                const int o = (pp >> 3) * PANEL + (pp & 7) * 2;
-                const uint32_t klo = *reinterpret_cast<const uint16_t*>(krow + o);
-                const uint32_t khi = *reinterpret_cast<const uint16_t*>(krow + o + (P / 8) * PANEL);
-                ct[(pp - p0) * 32 + lane] = klo | (khi << 16);
-              }
-              __syncwarp();
-#pragma unroll 1
-              for (int pp = p0; pp < p1; ++pp) {
-                const int T = sT[pp];
-                int lo, hi;  // chunk columns of this row that take the pair's term
-                float sgn;
-                if (pp >= ps) {
-                  lo = 0;
-                  hi = dc > T ? min(dc - T, 32) - 1 : -1;
-                  sgn = -1.f;
-                } else {
-                  lo = T >= dc ? 0 : dc - T;
-                  hi = min(dc, 31);
-                  sgn = 1.f;
-                }
-                const int o = (pp >> 3) * PANEL + (pp & 7) * 2 + r * 16;
-                const float qa = sgn * __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + o)) << 16);
-                const float qb = sgn * __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + o + (P / 8) * PANEL)) << 16);
-                const uint4* w4 = reinterpret_cast<const uint4*>(ct + (pp - p0) * 32);
-#pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
-                  const uint4 w = w4[c4];
-                  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    const int c = 4 * c4 + e;
-                    const float ka = __uint_as_float(ww[e] << 16);
-                    const float kh = __uint_as_float(ww[e] & 0xFFFF0000u);
-                    if (c >= lo && c <= hi) dl[c] = fmaf(qa, ka, fmaf(qb, kh, dl[c]));
-                  }
-                }
-              }
-            }
-            switch (cc) {
-              WPATTN_ADD_CHUNK(0)
-              WPATTN_ADD_CHUNK(1)
-              WPATTN_ADD_CHUNK(2)
-              WPATTN_ADD_CHUNK(3)
-            }
+          switch (cc) {
+            WPATTN_ADD_CHUNK(0)
+            WPATTN_ADD_CHUNK(1)
+            WPATTN_ADD_CHUNK(2)
+            WPATTN_ADD_CHUNK(3)
           }
         }
 #undef WPATTN_ADD_CHUNK
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(k_empty(s));
+      if (!(corr && G8)) {  // K stage s is no longer read by this warp
+        __syncwarp();
+        if (lane == 0) mbar_arrive(k_empty(s));
+      }
 
       if (!__all_sync(FULL, mbar_wait(s_full(t), cnt & 1))) { ok = false; break; }
       tc_fence_after();
-      if (corr) {
+      if (corr && G8) {
+        const uint8_t* kb = smem + L::OFF_K + s * L::TILE;
+        // whole groups of 8 pairs share a threshold: one 16-dim dot product per element
+#pragma unroll 1
+        for (int gp = plo; gp < P; gp += 8) {
+          const bool sub = gp >= ps;
+          const int T = sT[gp];
+          int c_lo, c_hi;  // columns of this row that take the group's term
+          if (sub) {
+            c_lo = 0;
+            c_hi = d_row > T ? min(d_row - T - 1, kBN - 1) : -1;
+          } else {
+            c_lo = T >= d_row ? 0 : d_row - T;
+            c_hi = min(d_row, kBN - 1);
+          }
+          if (!__any_sync(FULL, c_lo <= c_hi)) {
+            if (sub) break;  // later groups are pruned at even fewer columns
+            continue;
+          }
+          const float sgn = sub ? -1.f : 1.f;
+          const int off_lo = (gp >> 3) * PANEL;
+          const int off_hi = (P / 8 + (gp >> 3)) * PANEL;
+          float qv[16];
+          {
+            const uint4 a = *reinterpret_cast<const uint4*>(smem_q + off_lo + r * 16);
+            const uint4 c = *reinterpret_cast<const uint4*>(smem_q + off_hi + r * 16);
+            qv[0] = bf16lo_to_f32(a.x); qv[1] = bf16hi_to_f32(a.x);
+            qv[2] = bf16lo_to_f32(a.y); qv[3] = bf16hi_to_f32(a.y);
+            qv[4] = bf16lo_to_f32(a.z); qv[5] = bf16hi_to_f32(a.z);
+            qv[6] = bf16lo_to_f32(a.w); qv[7] = bf16hi_to_f32(a.w);
+            qv[8] = bf16lo_to_f32(c.x); qv[9] = bf16hi_to_f32(c.x);
+            qv[10] = bf16lo_to_f32(c.y); qv[11] = bf16hi_to_f32(c.y);
+            qv[12] = bf16lo_to_f32(c.z); qv[13] = bf16hi_to_f32(c.z);
+            qv[14] = bf16lo_to_f32(c.w); qv[15] = bf16hi_to_f32(c.w);
+          }
+#pragma unroll 1
+          for (int cc = 0; cc < kBN / 32; ++cc) {
+            const int lo = c_lo - 32 * cc, hi = c_hi - 32 * cc;  // chunk-local range
+            if (!__any_sync(FULL, lo <= 31 && hi >= 0 && lo <= hi)) continue;
+            float v[32];
+            tmem_ld32(tS + 32 * cc, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const uint4 a = *reinterpret_cast<const uint4*>(kb + off_lo + (32 * cc + c) * 16);
+              const uint4 b2 = *reinterpret_cast<const uint4*>(kb + off_hi + (32 * cc + c) * 16);
+              float d0 = 0.f, d1 = 0.f;
+              fma2(d0, d1, qv[0], qv[1], bf16lo_to_f32(a.x), bf16hi_to_f32(a.x), d0, d1);
+              fma2(d0, d1, qv[2], qv[3], bf16lo_to_f32(a.y), bf16hi_to_f32(a.y), d0, d1);
+              fma2(d0, d1, qv[4], qv[5], bf16lo_to_f32(a.z), bf16hi_to_f32(a.z), d0, d1);
+              fma2(d0, d1, qv[6], qv[7], bf16lo_to_f32(a.w), bf16hi_to_f32(a.w), d0, d1);
+              fma2(d0, d1, qv[8], qv[9], bf16lo_to_f32(b2.x), bf16hi_to_f32(b2.x), d0, d1);
+              fma2(d0, d1, qv[10], qv[11], bf16lo_to_f32(b2.y), bf16hi_to_f32(b2.y), d0, d1);
+              fma2(d0, d1, qv[12], qv[13], bf16lo_to_f32(b2.z), bf16hi_to_f32(b2.z), d0, d1);
+              fma2(d0, d1, qv[14], qv[15], bf16lo_to_f32(b2.w), bf16hi_to_f32(b2.w), d0, d1);
+              if (c >= lo && c <= hi) v[c] = fmaf(sgn, d0 + d1, v[c]);
+            }
+            tmem_st32(tS + 32 * cc, v);
+          }
+        }
+        tmem_st_wait();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(k_empty(s));
+      }
+      if (corr && !G8) {
 #pragma unroll
         for (int cc = 0; cc < kBN / 32; ++cc) {
           float v[32];
