@@ -127,7 +127,7 @@ int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
     attr_set[dev] = true;
   }
   dim3 grid(prm.S, prm.Hkv * prm.hchunks, prm.B);
-  decode_split_kernel<D, GC><<<grid, (decode_compute_warps(GC) + 1) * 32, smem, st>>>(tk, tv, prm);
+  decode_split_kernel<D, GC><<<grid, (kDecodeComputeWarps + 1) * 32, smem, st>>>(tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 

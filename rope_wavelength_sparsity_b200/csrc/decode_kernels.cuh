@@ -5,15 +5,14 @@
 // decode kernel.  Each CTA covers one (sequence, kv head, key range) and all
 // the query heads of the GQA group (up to GC at a time), so a K/V byte is
 // read once for the group.  A producer warp streams blocks of 32 keys of K
-// and V through a shared-memory ring with TMA (128-byte swizzle); four
-// compute warps take one 16-byte chunk (8 head dims) of a key per lane, so
-// a warp holds 32/(D/8) keys per step.  A lane multiplies its K chunk only
-// if the chunk still holds a kept pair at that key's distance (pruned dims
-// are zeroed); the dot product is a shuffle reduction across the key's lanes.
-// In the [B, L, Hkv, D] cache layout each half of a K row is one 128-byte
-// line and the kept slice touches both, so whole rows move from DRAM either
-// way; the window saves arithmetic here, not bytes.  A second kernel merges
-// the key ranges by their log-sum-exp.
+// and V through a shared-memory ring with TMA (128-byte swizzle); each block
+// is consumed by one of four compute warps.  For the scores a lane owns a
+// key and walks only the groups of 8 pairs still kept in the block; for
+// O += p V a lane owns a 16-byte chunk of the head dim.  In the
+// [B, L, Hkv, D] cache layout each half of a K row is one 128-byte line and
+// the kept slice touches both, so whole rows move from DRAM either way; the
+// window saves arithmetic here, not bytes.  A second kernel merges the key
+// ranges by their log-sum-exp.
 #pragma once
 
 #include "device_util.cuh"
@@ -55,26 +54,33 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
 }
 
 // Shared-memory ring of the split kernel: blocks of KB keys of K and V in
-// the 128-byte-swizzled layout TMA writes (64-dim panels, row = key).
+// the 128-byte-swizzled layout TMA writes (64-dim panels, row = key), plus
+// the pre-scaled query heads, the thresholds and each warp's p row.
+constexpr int kDecodeComputeWarps = 4;
+
 template <int D>
 struct DecodeSmem {
-  static constexpr int KB = 32;                        // keys per block
-  static constexpr int NS = (D == 64) ? 8 : 4;         // ring depth
+  static constexpr int KB = 32;                        // keys per block (one per lane)
+  // ring depth (blocks in flight): a multiple of the compute warps, so that
+  // stage s is only ever consumed by warp s mod W and a warp never waits on a
+  // phase of a stage whose previous phase belongs to another warp (a parity
+  // wait cannot tell phase k from phase k - 2)
+  static constexpr int NS = (D == 64) ? 8 : 4;
   static constexpr int PANEL = KB * 128;               // one 64-dim panel of a block
   static constexpr int TILE = KB * D * 2;              // K or V block
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = NS * TILE;
-  static constexpr int OFF_BAR = 2 * NS * TILE;        // full[NS], empty[NS]
+  static constexpr int OFF_Q = 2 * NS * TILE;          // [8 heads][D] fp32, scaled by scale * log2(e)
+  static constexpr int OFF_T = OFF_Q + 8 * D * 4;      // thresholds (64 x int32)
+  static constexpr int OFF_P = OFF_T + 64 * 4;         // [warps][8 heads][KB] fp32 weights
+  static constexpr int OFF_BAR = OFF_P + kDecodeComputeWarps * 8 * KB * 4;  // full[NS], empty[NS]
   static constexpr int BYTES = OFF_BAR + 2 * NS * 8;
   static constexpr int ALLOC = BYTES + 1024;           // slack to align the ring to 1024 bytes
 };
 
-// compute warps per CTA: more warps (and fewer live values each) for large
-// GQA groups, whose per-lane accumulators limit occupancy
-__host__ __device__ constexpr int decode_compute_warps(int GC) { return GC > 4 ? 8 : 4; }
-
 // 16 bytes of a K or V row from the swizzled ring: row r (key within the
-// block), 16-byte chunk c of the head dim.
+// block), 16-byte chunk c of the head dim.  Eight consecutive rows put a
+// given chunk in eight different 16-byte bank groups.
 template <int D>
 __device__ __forceinline__ uint4 ring_chunk(const uint8_t* tile, int r, int c) {
   using L = DecodeSmem<D>;
@@ -82,28 +88,36 @@ __device__ __forceinline__ uint4 ring_chunk(const uint8_t* tile, int r, int c) {
                                          (((c & 7) ^ (r & 7)) << 4));
 }
 
+// Work split inside a CTA: the producer warp streams blocks of 32 keys; block
+// i goes to compute warp i mod 4.  For the scores a lane owns one key (its
+// whole row): it walks only the groups of 8 pairs that are still kept
+// somewhere in the warp's 32 keys, with the query head dims read from shared
+// memory (broadcast), so the window removes work and no cross-lane reduction
+// is needed.  For O += p V a lane owns one 16-byte chunk of the head dim for
+// 32 / (D / 8) keys at a time.
 template <int D, int GC>
-__global__ void __launch_bounds__((decode_compute_warps(GC) + 1) * 32)
+__global__ void __launch_bounds__((kDecodeComputeWarps + 1) * 32, GC <= 4 ? 3 : 2)
 decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ DecodeParams p) {
   using L = DecodeSmem<D>;
-  constexpr int KB = L::KB, NS = L::NS;
-  constexpr int kDecodeComputeWarps = decode_compute_warps(GC);
-  constexpr int TPK = D / 8;              // lanes per key (one 16-byte chunk each)
-  constexpr int KPW = 32 / TPK;           // keys per warp per step
-  constexpr int SLOTS = kDecodeComputeWarps * KPW;
-  constexpr int U = KB / SLOTS;           // steps per block
-  constexpr int HALF = TPK / 2;           // chunks per half of the head dim
-  static_assert(KB % SLOTS == 0, "block must be a multiple of the key slots");
+  constexpr int KB = L::KB, NS = L::NS, W = kDecodeComputeWarps;
+  constexpr int P = D / 2;
+  constexpr int NG = P / 8;               // groups of 8 pairs (16 dims: 8 in each half)
+  constexpr int TPK = D / 8;              // lanes per key in the PV step (one 16-byte chunk each)
+  constexpr int KPW = 32 / TPK;           // keys per PV step
+  constexpr uint32_t FULL = 0xffffffffu;
+  static_assert(W * GC * D * 4 <= 2 * NS * L::TILE, "merge buffer must fit in the ring");
+  static_assert(NS % W == 0, "each ring stage must belong to one compute warp");
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the swizzled ring starts on a 1024-byte boundary of the shared window
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  __shared__ float sm_m[SLOTS][GC];
-  __shared__ float sm_l[SLOTS][GC];
+  __shared__ float sm_m[W][GC];
+  __shared__ float sm_l[W][GC];
   // the merge's partial outputs reuse the ring once every block is consumed
-  static_assert(SLOTS * GC * D * 4 <= 2 * NS * L::TILE, "merge buffer must fit in the ring");
   float (*sm_o)[GC][D] = reinterpret_cast<float (*)[GC][D]>(smem);
+  float* qs = reinterpret_cast<float*>(smem + L::OFF_Q);
+  int* sT = reinterpret_cast<int*>(smem + L::OFF_T);
 
   const uint32_t sbase = smem_u32(smem);
   auto full = [&](int s) { return sbase + L::OFF_BAR + 8 * s; };
@@ -126,13 +140,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(empty(s), kDecodeComputeWarps);
+      mbar_init(empty(s), 1);   // the one compute warp that owns the block
     }
     fence_barrier_init();
   }
+  if (threadIdx.x < 64) sT[threadIdx.x] = p.T[threadIdx.x];
+  for (int idx = threadIdx.x; idx < GC * D; idx += blockDim.x) {
+    const int hh = idx / D, e = idx % D;
+    qs[idx] = hh < nh ? bf16lo_to_f32(p.q[((size_t)b * p.Hq + h0 + hh) * D + e]) * p.scale_log2 : 0.f;
+  }
   __syncthreads();
 
-  if (warp == kDecodeComputeWarps) {
+  if (warp == W) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&tmK);
@@ -152,28 +171,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   }
 
   // ---------------------------------------------------------------- compute
-  const int c = lane % TPK;               // head-dim chunk [8c, 8c+8)
-  const int slot = warp * KPW + lane / TPK;
-  const int pb = (c % HALF) * 8;          // first pair of this chunk
-  int Tc[8];                              // thresholds of this chunk's 8 pairs
-#pragma unroll
-  for (int e = 0; e < 8; ++e) Tc[e] = p.T[pb + e];
-  const int T_first = Tc[0];
-  const int T_last = Tc[7];
-
-  float qf[GC][8];
-#pragma unroll
-  for (int hh = 0; hh < GC; ++hh) {
-    if (hh < nh) {
-      const uint4 u = *reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + h0 + hh) * D + 8 * c);
-      unpack8(u, qf[hh]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) qf[hh][e] *= p.scale_log2;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) qf[hh][e] = 0.f;
-    }
-  }
+  const int c = lane % TPK;               // PV: head-dim chunk [8c, 8c+8)
+  const int kk = lane / TPK;              // PV: key within a step
+  float* pw = reinterpret_cast<float*>(smem + L::OFF_P) + warp * 8 * KB;  // this warp's p rows
   float m[GC], l[GC], o[GC][8];
 #pragma unroll
   for (int hh = 0; hh < GC; ++hh) {
@@ -183,95 +183,138 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     for (int e = 0; e < 8; ++e) o[hh][e] = 0.f;
   }
 
-  bool ok = true;
-  for (int i = 0; i < nblk; ++i) {
+  for (int i = warp; i < nblk; i += W) {
     const int s = i % NS;
-    if (!__all_sync(0xffffffffu, mbar_wait(full(s), (i / NS) & 1))) { ok = false; break; }
+    if (!__all_sync(FULL, mbar_wait(full(s), (i / NS) & 1))) break;
     const uint8_t* kt = smem + L::OFF_K + s * L::TILE;
     const uint8_t* vt = smem + L::OFF_V + s * L::TILE;
-    float sco[U][GC];
-    float vf[U][8];
+    const int j0 = j_begin + i * KB;
+    const int j = j0 + lane;              // this lane's key
+    const bool valid = j < j_end;
+    const int dist = qpos - j;
+    // smallest distance of a real key in the block: groups whose largest
+    // threshold is below it are pruned for every key of the block
+    const int dmin = qpos - (min(j0 + KB, j_end) - 1);
+    int g0 = 0;
+    while (g0 < NG && sT[8 * g0 + 7] < dmin) ++g0;
+
+    // ---- scores: one key per lane, groups g0 .. NG-1
+    float sc[GC];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int r = u * SLOTS + slot;     // key within the block
-      const int j = j_begin + i * KB + r;
-      const bool valid = j < j_end;
-      const int dist = qpos - j;
-      unpack8(ring_chunk<D>(vt, r, c), vf[u]);
-      float kf[8];
-      if (dist <= T_last) {               // this chunk holds a kept pair
-        unpack8(ring_chunk<D>(kt, r, c), kf);
-        if (dist > T_first) {             // only partly kept at this distance
+    for (int hh = 0; hh < GC; ++hh) sc[hh] = 0.f;
+#pragma unroll 1
+    for (int g = g0; g < NG; ++g) {
+      float kf[16];
+      {
+        float a[8], bb[8];
+        unpack8(ring_chunk<D>(kt, lane, g), a);            // dims 8g .. 8g+7
+        unpack8(ring_chunk<D>(kt, lane, NG + g), bb);      // dims P+8g .. P+8g+7
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            if (dist > Tc[e]) kf[e] = 0.f;
+        for (int e = 0; e < 8; ++e) { kf[e] = a[e]; kf[8 + e] = bb[e]; }
+      }
+      // pairs of the group pruned at this key's distance contribute 0
+      if (__any_sync(FULL, dist > sT[8 * g])) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (dist > sT[8 * g + e]) { kf[e] = 0.f; kf[8 + e] = 0.f; }
         }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) kf[e] = 0.f;
       }
 #pragma unroll
       for (int hh = 0; hh < GC; ++hh) {
+        const float4* qa = reinterpret_cast<const float4*>(qs + hh * D + 8 * g);
+        const float4* qb = reinterpret_cast<const float4*>(qs + hh * D + P + 8 * g);
+        const float4 x0 = qa[0], x1 = qa[1], y0 = qb[0], y1 = qb[1];
         float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; e += 2)
-          fma2(a0, a1, qf[hh][e], qf[hh][e + 1], kf[e], kf[e + 1], a0, a1);
-        float acc = a0 + a1;
-#pragma unroll
-        for (int off = TPK / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        sco[u][hh] = valid ? acc : -INFINITY;
+        fma2(a0, a1, x0.x, x0.y, kf[0], kf[1], a0, a1);
+        fma2(a0, a1, x0.z, x0.w, kf[2], kf[3], a0, a1);
+        fma2(a0, a1, x1.x, x1.y, kf[4], kf[5], a0, a1);
+        fma2(a0, a1, x1.z, x1.w, kf[6], kf[7], a0, a1);
+        fma2(a0, a1, y0.x, y0.y, kf[8], kf[9], a0, a1);
+        fma2(a0, a1, y0.z, y0.w, kf[10], kf[11], a0, a1);
+        fma2(a0, a1, y1.x, y1.y, kf[12], kf[13], a0, a1);
+        fma2(a0, a1, y1.z, y1.w, kf[14], kf[15], a0, a1);
+        sc[hh] += a0 + a1;
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty(s));
+
+    // ---- online softmax over the block (warp-wide max per head)
 #pragma unroll
     for (int hh = 0; hh < GC; ++hh) {
-      float mx = m[hh];
+      const float sv = valid ? sc[hh] : -INFINITY;
+      float bm = sv;
 #pragma unroll
-      for (int u = 0; u < U; ++u) mx = fmaxf(mx, sco[u][hh]);
-      if (mx == -INFINITY) continue;
-      const float corr = ex2_approx(m[hh] - mx);
-      l[hh] *= corr;
+      for (int off = 16; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(FULL, bm, off));
+      const float mn = fmaxf(m[hh], bm);
+      float pv = 0.f;
+      if (mn != -INFINITY) {
+        const float corr = (m[hh] == -INFINITY) ? 0.f : ex2_approx(m[hh] - mn);
+        pv = ex2_approx(sv - mn);
+        l[hh] = l[hh] * corr + pv;        // this lane's key only; summed over lanes at the end
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) mul2(o[hh][e], o[hh][e + 1], o[hh][e], o[hh][e + 1], corr, corr);
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const float pu = ex2_approx(sco[u][hh] - mx);
-        l[hh] += pu;
-#pragma unroll
-        for (int e = 0; e < 8; e += 2)
-          fma2(o[hh][e], o[hh][e + 1], pu, pu, vf[u][e], vf[u][e + 1], o[hh][e], o[hh][e + 1]);
+        for (int e = 0; e < 8; e += 2) mul2(o[hh][e], o[hh][e + 1], o[hh][e], o[hh][e + 1], corr, corr);
+        m[hh] = mn;
       }
-      m[hh] = mx;
+      pw[hh * KB + lane] = pv;
     }
-  }
-  (void)ok;
+    __syncwarp();
 
-  // merge the key slots of this CTA (compute warps only); every block has
-  // been consumed, so the ring is free
-  asm volatile("bar.sync 1, %0;" ::"n"(kDecodeComputeWarps * 32) : "memory");
+    // ---- O += p V: lane (kk, c) takes chunk c of keys kk, kk + KPW, ...
+    // (keys past the sequence end are not read: a cache may hold anything there)
+    const int nvalid = min(KB, j_end - j0);
+#pragma unroll 4
+    for (int r = kk; r < nvalid; r += KPW) {
+      float vf[8];
+      unpack8(ring_chunk<D>(vt, r, c), vf);
+#pragma unroll
+      for (int hh = 0; hh < GC; ++hh) {
+        const float pr = pw[hh * KB + r];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) fma2(o[hh][e], o[hh][e + 1], pr, pr, vf[e], vf[e + 1], o[hh][e], o[hh][e + 1]);
+      }
+    }
+    __syncwarp();  // the p rows are rewritten by the next block
+    if (lane == 0) mbar_arrive(empty(s));
+  }
+
+  // combine this warp's lanes: l over keys (all lanes), o over the KPW key groups
 #pragma unroll
   for (int hh = 0; hh < GC; ++hh) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) sm_o[slot][hh][8 * c + e] = o[hh][e];
-    if (c == 0) {
-      sm_m[slot][hh] = m[hh];
-      sm_l[slot][hh] = l[hh];
+    for (int off = 16; off > 0; off >>= 1) l[hh] += __shfl_xor_sync(FULL, l[hh], off);
+#pragma unroll
+    for (int off = TPK; off < 32; off <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[hh][e] += __shfl_xor_sync(FULL, o[hh][e], off);
     }
   }
-  asm volatile("bar.sync 1, %0;" ::"n"(kDecodeComputeWarps * 32) : "memory");
-  for (int idx = threadIdx.x; idx < nh * D; idx += kDecodeComputeWarps * 32) {
+
+  // merge the warps of this CTA (compute warps only); every block has been
+  // consumed, so the ring is free
+  asm volatile("bar.sync 1, %0;" ::"n"(W * 32) : "memory");
+  if (kk == 0) {
+#pragma unroll
+    for (int hh = 0; hh < GC; ++hh) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sm_o[warp][hh][8 * c + e] = o[hh][e];
+      if (c == 0) {
+        sm_m[warp][hh] = m[hh];
+        sm_l[warp][hh] = l[hh];
+      }
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(W * 32) : "memory");
+  for (int idx = threadIdx.x; idx < nh * D; idx += W * 32) {
     const int hh = idx / D, e = idx % D;
     float M = -INFINITY;
 #pragma unroll
-    for (int s2 = 0; s2 < SLOTS; ++s2) M = fmaxf(M, sm_m[s2][hh]);
+    for (int w2 = 0; w2 < W; ++w2) M = fmaxf(M, sm_m[w2][hh]);
     float Ls = 0.f, Os = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
-      for (int s2 = 0; s2 < SLOTS; ++s2) {
-        const float w = ex2_approx(sm_m[s2][hh] - M);
-        Ls += sm_l[s2][hh] * w;
-        Os += sm_o[s2][hh][e] * w;
+      for (int w2 = 0; w2 < W; ++w2) {
+        const float wt = ex2_approx(sm_m[w2][hh] - M);
+        Ls += sm_l[w2][hh] * wt;
+        Os += sm_o[w2][hh][e] * wt;
       }
     }
     float* rec = p.part + (((size_t)b * p.Hq + h0 + hh) * p.S + split) * (D + 2);
