@@ -384,6 +384,28 @@ def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
                    "parallelism": f"independent problem per GPU x{world}",
                    "l2": "flushed between steps (512 MiB write)"},
     }
+    # the same call with K in the pair-major layout (converted once, outside the timed region):
+    # the window then also cuts the bytes K moves from HBM
+    slabs = wp.kcache_to_pairmajor(kc)
+
+    def step_pm():
+        wp.decode_pairmajor(q, slabs, vc, kv_len, win, scale=w.scale, out=out, lse=lse, workspace=ws)
+
+    pm_ms, pm_per, _ = time_steps(step_pm, args.warmup, steps, flush, world)
+    if wp.device_status() != wp.OK:
+        raise RuntimeError("pair-major decode kernel status: timeout")
+    pm_achieved = alg / (statistics.mean(pm_per) * 1e-3) / 1e9
+    res["pairmajor"] = {
+        "value": round(weak_scaling_value(alg, world, pm_ms / steps) / 1e9, 1), "unit": "GB/s",
+        "ms_per_step": round(pm_ms / steps, 4),
+        "roofline": {"bound": "hbm", "achieved": round(pm_achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(pm_achieved / peaks["hbm_gbs"], 4),
+                     "traffic": None, "peak_source": f"{peaks['source']} HBM copy"},
+        "speedup_vs_window_off": round(off_step / (pm_ms / steps), 3),
+        "layout": "K [B, Hkv, D/16, L, 16] pair-major slabs, V [B, L, Hkv, D]",
+    }
+    res["gpu_launches"] += 2 * steps
+    del slabs
     if primary:
         res["clocks"] = clk
         qh = q.cpu().pin_memory()

@@ -174,6 +174,39 @@ WPATTN_API int wpattn_decode_noalloc(const wpattn_window *w,
 WPATTN_API size_t wpattn_decode_noalloc_max_bytes(void);
 
 /*
+ * Decode with the K cache in the pair-major layout (a variant of this
+ * library, not a layout of the pages; ATFlash Abstract: decode reads K only
+ * over the active head-dim slice of each key block, and here that slice is
+ * contiguous).
+ *   k_slabs: bf16 device [B, Hkv, D/16, Lmax, 16].  Slab g of key j holds head
+ *            dims 8g..8g+7 followed by D/2+8g..D/2+8g+7, i.e. the 8 RoPE pairs
+ *            8g..8g+7 whose window group starts a contraction step.  Build it
+ *            from a [B, Lmax, Hkv, D] cache with wpattn_kcache_to_pairmajor.
+ * Every other argument, the result and the workspace are those of
+ * wpattn_decode (same sizes, same errors); the two calls give the same
+ * output.  A key block (32 keys) loads only the slabs of the groups kept at
+ * some of its distances, so the window also cuts the bytes K moves from HBM.
+ */
+WPATTN_API int wpattn_decode_pairmajor(const wpattn_window *w,
+                  const void *q, const void *k_slabs, const void *v_cache,
+                  const int32_t *kv_len_host, int64_t Lmax,
+                  int32_t B, int32_t Hq, int32_t Hkv, float softmax_scale,
+                  void *out, float *lse,
+                  void *workspace, size_t workspace_bytes,
+                  void *cuda_stream);
+
+/*
+ * Rewrite a K cache [B, Lmax, Hkv, head_dim] (bf16, device) into the
+ * pair-major slabs [B, Hkv, head_dim/16, Lmax, 16] that
+ * wpattn_decode_pairmajor reads (bf16, device, caller-allocated,
+ * B * Lmax * Hkv * head_dim * 2 bytes, must not overlap k_cache).  Both
+ * pointers 16-byte aligned; head_dim in {64, 128} (else WPATTN_EUNSUPPORTED);
+ * asynchronous on `cuda_stream`.  Bit-exact: only moves bytes.
+ */
+WPATTN_API int wpattn_kcache_to_pairmajor(const void *k_cache, void *k_slabs, int64_t Lmax,
+                  int32_t B, int32_t Hkv, int32_t head_dim, void *cuda_stream);
+
+/*
  * Synchronises `cuda_stream`, then reads and clears the current device's
  * kernel status word.  Returns WPATTN_OK, WPATTN_ETIMEOUT (a kernel gave up a
  * bounded wait; its outputs are undefined) or WPATTN_ECUDA.

@@ -8,7 +8,8 @@ fallback path: if the shared library is missing or a call fails, an
 exception is raised.
 
 Entry points (same names as the C ABI, without the ``wpattn_`` prefix):
-``prefill``, ``decode``, ``decode_workspace_size``, ``pruned_fraction``,
+``prefill``, ``decode``, ``decode_pairmajor``, ``kcache_to_pairmajor``,
+``decode_workspace_size``, ``decode_noalloc``, ``pruned_fraction``,
 ``thresholds``, ``device_status``.
 """
 from __future__ import annotations
@@ -70,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.wpattn_decode_workspace_size.argtypes = [wp, i32, i32, i32, i64]
         L.wpattn_decode.argtypes = [wp, vp, vp, vp, ctypes.POINTER(ctypes.c_int32), i64, i32, i32,
                                     i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
+        L.wpattn_decode_pairmajor.argtypes = L.wpattn_decode.argtypes
+        L.wpattn_kcache_to_pairmajor.argtypes = [vp, vp, i64, i32, i32, i32, vp]
         L.wpattn_device_status.argtypes = [vp]
         L.wpattn_strerror.restype = ctypes.c_char_p
         L.wpattn_strerror.argtypes = [ctypes.c_int]
@@ -179,6 +182,46 @@ def decode(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | None = None
                              ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
                              _stream_ptr(stream))
     _check(rc, "wpattn_decode")
+    return out, lse
+
+
+def kcache_to_pairmajor(k_cache, out=None, stream=None):
+    """K cache [B, L, Hkv, D] -> pair-major slabs [B, Hkv, D/16, L, 16] (bf16 CUDA tensors)."""
+    import torch
+    B, L, Hkv, D = k_cache.shape
+    if out is None:
+        out = torch.empty((B, Hkv, D // 16, L, 16), dtype=k_cache.dtype, device=k_cache.device)
+    _check(lib().wpattn_kcache_to_pairmajor(_dev_tensor(k_cache, "k_cache"), _dev_tensor(out, "out"),
+                                            L, B, Hkv, D, _stream_ptr(stream)),
+           "wpattn_kcache_to_pairmajor")
+    return out
+
+
+def decode_pairmajor(q, k_slabs, v_cache, kv_len, w: Window, *, scale: float | None = None,
+                     out=None, lse=None, want_lse: bool = True, workspace=None, stream=None):
+    """Windowed decode with K as pair-major slabs [B, Hkv, D/16, L, 16] (see
+    ``kcache_to_pairmajor``); q, v_cache, kv_len and the results as for ``decode``."""
+    import torch
+    B, Hq, D = q.shape
+    Hkv, L = k_slabs.shape[1], k_slabs.shape[3]
+    kvl = (ctypes.c_int32 * B)(*[int(x) for x in kv_len])
+    if workspace is None:
+        n = decode_workspace_size(w, B, Hq, Hkv, L)
+        if n == 0:
+            raise WpattnError(EINVAL, "wpattn_decode_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    rc = lib().wpattn_decode_pairmajor(ctypes.byref(w._c()), _dev_tensor(q, "q"),
+                                       _dev_tensor(k_slabs, "k_slabs"), _dev_tensor(v_cache, "v_cache"),
+                                       kvl, L, B, Hq, Hkv, float(scale) if scale else 0.0,
+                                       _dev_tensor(out, "out"),
+                                       ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+                                       ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                       _stream_ptr(stream))
+    _check(rc, "wpattn_decode_pairmajor")
     return out, lse
 
 

@@ -73,6 +73,20 @@ int device_info(DeviceInfo** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// bf16 tensor map with explicit byte strides of dims 1..3 (dim 0 contiguous), no swizzle
+int encode_bf16_4d_strided(CUtensorMap* map, const void* base, const cuuint64_t (&dims)[4],
+                           const cuuint64_t (&strides)[3], uint32_t box0, uint32_t box1) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return WPATTN_ECUDA;
+  const cuuint32_t box[4] = {box0, box1, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? WPATTN_OK : WPATTN_ECUDA;
+}
+
 int encode_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                    uint64_t d3, uint32_t box0, uint32_t box1, bool swizzle128) {
   EncodeTiledFn enc = get_encode_fn();
@@ -113,7 +127,7 @@ int launch_prefill(const void* q, const void* k, const void* v, const PrefillPar
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
-template <int D, int GC>
+template <int D, int GC, bool PM>
 int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& prm,
                         cudaStream_t st) {
   constexpr int smem = DecodeSmem<D>::ALLOC;
@@ -121,36 +135,53 @@ int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WPATTN_ECUDA;
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(decode_split_kernel<D, GC>,
+    if (cudaFuncSetAttribute(decode_split_kernel<D, GC, PM>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return WPATTN_ECUDA;
     attr_set[dev] = true;
   }
   dim3 grid(prm.S, prm.Hkv * prm.hchunks, prm.B);
-  decode_split_kernel<D, GC><<<grid, (kDecodeComputeWarps + 1) * 32, smem, st>>>(tk, tv, prm);
+  decode_split_kernel<D, GC, PM><<<grid, (kDecodeComputeWarps + 1) * 32, smem, st>>>(tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
-template <int D>
-int launch_decode(const DecodeParams& prm, int gc, cudaStream_t st) {
-  int rc;
-  CUtensorMap tk, tv;
-  // caches are [B, Lmax, Hkv, D]: dims (fastest first) D, Lmax, Hkv, B; 64-dim x 32-key boxes
-  if ((rc = encode_bf16_4d(&tk, prm.k, D, prm.Lmax, prm.Hkv, prm.B, 64, DecodeSmem<D>::KB, true)) != WPATTN_OK)
-    return rc;
-  if ((rc = encode_bf16_4d(&tv, prm.v, D, prm.Lmax, prm.Hkv, prm.B, 64, DecodeSmem<D>::KB, true)) != WPATTN_OK)
-    return rc;
+template <int D, bool PM>
+int launch_decode_gc(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& prm, int gc,
+                     cudaStream_t st) {
   switch (gc) {
-    case 1: rc = launch_decode_split<D, 1>(tk, tv, prm, st); break;
-    case 2: rc = launch_decode_split<D, 2>(tk, tv, prm, st); break;
-    case 3: rc = launch_decode_split<D, 3>(tk, tv, prm, st); break;
-    case 4: rc = launch_decode_split<D, 4>(tk, tv, prm, st); break;
-    case 5: rc = launch_decode_split<D, 5>(tk, tv, prm, st); break;
-    case 6: rc = launch_decode_split<D, 6>(tk, tv, prm, st); break;
-    case 7: rc = launch_decode_split<D, 7>(tk, tv, prm, st); break;
-    case 8: rc = launch_decode_split<D, 8>(tk, tv, prm, st); break;
+    case 1: return launch_decode_split<D, 1, PM>(tk, tv, prm, st);
+    case 2: return launch_decode_split<D, 2, PM>(tk, tv, prm, st);
+    case 3: return launch_decode_split<D, 3, PM>(tk, tv, prm, st);
+    case 4: return launch_decode_split<D, 4, PM>(tk, tv, prm, st);
+    case 5: return launch_decode_split<D, 5, PM>(tk, tv, prm, st);
+    case 6: return launch_decode_split<D, 6, PM>(tk, tv, prm, st);
+    case 7: return launch_decode_split<D, 7, PM>(tk, tv, prm, st);
+    case 8: return launch_decode_split<D, 8, PM>(tk, tv, prm, st);
     default: return WPATTN_EUNSUPPORTED;
   }
+}
+
+template <int D>
+int launch_decode(const DecodeParams& prm, int gc, bool pm, cudaStream_t st) {
+  int rc;
+  CUtensorMap tk, tv;
+  constexpr uint32_t KB = DecodeSmem<D>::KB;
+  if (pm) {
+    // pair-major K slabs [B, Hkv, D/16, Lmax, 16]: dims (fastest first) 16, Lmax,
+    // Hkv * D/16 (slab planes), B; 16-dim x 32-key boxes
+    const uint64_t planes = static_cast<uint64_t>(prm.Hkv) * (D / 16);
+    const cuuint64_t dims[4] = {16, static_cast<cuuint64_t>(prm.Lmax), planes, static_cast<cuuint64_t>(prm.B)};
+    const cuuint64_t strides[3] = {32, static_cast<cuuint64_t>(prm.Lmax) * 32,
+                                   planes * static_cast<cuuint64_t>(prm.Lmax) * 32};
+    if ((rc = encode_bf16_4d_strided(&tk, prm.k, dims, strides, 16, KB)) != WPATTN_OK) return rc;
+  } else {
+    // caches are [B, Lmax, Hkv, D]: dims (fastest first) D, Lmax, Hkv, B; 64-dim x 32-key boxes
+    if ((rc = encode_bf16_4d(&tk, prm.k, D, prm.Lmax, prm.Hkv, prm.B, 64, KB, true)) != WPATTN_OK)
+      return rc;
+  }
+  if ((rc = encode_bf16_4d(&tv, prm.v, D, prm.Lmax, prm.Hkv, prm.B, 64, KB, true)) != WPATTN_OK)
+    return rc;
+  rc = pm ? launch_decode_gc<D, true>(tk, tv, prm, gc, st) : launch_decode_gc<D, false>(tk, tv, prm, gc, st);
   if (rc != WPATTN_OK) return rc;
   const size_t smem = static_cast<size_t>(prm.S) * 2 * sizeof(float);
   if (smem > 48 * 1024) {
@@ -279,10 +310,15 @@ size_t wpattn_decode_workspace_size(const wpattn_window* w, int32_t B, int32_t H
   return decode_workspace_bytes(B, Hq, plan.D, decode_max_splits(B, Hkv, max_kv_len));
 }
 
-int wpattn_decode(const wpattn_window* w, const void* q, const void* k_cache, const void* v_cache,
-                  const int32_t* kv_len_host, int64_t Lmax, int32_t B, int32_t Hq, int32_t Hkv,
-                  float softmax_scale, void* out, float* lse, void* workspace,
-                  size_t workspace_bytes, void* cuda_stream) {
+}  // extern "C"
+
+namespace {
+// wpattn_decode and wpattn_decode_pairmajor: the same call with the K cache in
+// the [B, Lmax, Hkv, D] layout (pm = false) or as pair-major slabs (pm = true)
+int decode_impl(const wpattn_window* w, const void* q, const void* k_cache, const void* v_cache,
+                const int32_t* kv_len_host, int64_t Lmax, int32_t B, int32_t Hq, int32_t Hkv,
+                float softmax_scale, void* out, float* lse, void* workspace,
+                size_t workspace_bytes, void* cuda_stream, bool pm) {
   WindowPlan plan;
   int rc = make_window_plan(w, &plan);
   if (rc != WPATTN_OK) return rc;
@@ -320,8 +356,50 @@ int wpattn_decode(const wpattn_window* w, const void* q, const void* k_cache, co
   for (int p = 0; p < 64; ++p) prm.T[p] = plan.T[p] > INT32_MAX ? INT32_MAX : static_cast<int>(plan.T[p]);
   for (int b = 0; b < B; ++b) prm.kv_len[b] = kv_len_host[b];
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  if (plan.D == 64) return launch_decode<64>(prm, gc, st);
-  return launch_decode<128>(prm, gc, st);
+  if (plan.D == 64) return launch_decode<64>(prm, gc, pm, st);
+  return launch_decode<128>(prm, gc, pm, st);
+}
+}  // namespace
+
+extern "C" {
+
+int wpattn_decode(const wpattn_window* w, const void* q, const void* k_cache, const void* v_cache,
+                  const int32_t* kv_len_host, int64_t Lmax, int32_t B, int32_t Hq, int32_t Hkv,
+                  float softmax_scale, void* out, float* lse, void* workspace,
+                  size_t workspace_bytes, void* cuda_stream) {
+  return decode_impl(w, q, k_cache, v_cache, kv_len_host, Lmax, B, Hq, Hkv, softmax_scale, out, lse,
+                     workspace, workspace_bytes, cuda_stream, false);
+}
+
+int wpattn_decode_pairmajor(const wpattn_window* w, const void* q, const void* k_slabs,
+                            const void* v_cache, const int32_t* kv_len_host, int64_t Lmax,
+                            int32_t B, int32_t Hq, int32_t Hkv, float softmax_scale, void* out,
+                            float* lse, void* workspace, size_t workspace_bytes,
+                            void* cuda_stream) {
+  return decode_impl(w, q, k_slabs, v_cache, kv_len_host, Lmax, B, Hq, Hkv, softmax_scale, out, lse,
+                     workspace, workspace_bytes, cuda_stream, true);
+}
+
+int wpattn_kcache_to_pairmajor(const void* k_cache, void* k_slabs, int64_t Lmax, int32_t B,
+                               int32_t Hkv, int32_t head_dim, void* cuda_stream) {
+  if (!k_cache || !k_slabs || Lmax <= 0 || B <= 0 || Hkv <= 0) return WPATTN_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(k_slabs)) return WPATTN_EINVAL;
+  if (head_dim != 64 && head_dim != 128) return WPATTN_EUNSUPPORTED;
+  if (Lmax >= (int64_t(1) << 31)) return WPATTN_EUNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  int rc;
+  if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const uint64_t n = static_cast<uint64_t>(B) * Hkv * (head_dim / 16) * static_cast<uint64_t>(Lmax);
+  const uint64_t blocks = (n + 255) / 256;
+  if (blocks > 0x7FFFFFFFull) return WPATTN_EUNSUPPORTED;
+  if (head_dim == 64)
+    kcache_to_pairmajor_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const uint16_t*>(k_cache), static_cast<uint16_t*>(k_slabs), Lmax, B, Hkv);
+  else
+    kcache_to_pairmajor_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const uint16_t*>(k_cache), static_cast<uint16_t*>(k_slabs), Lmax, B, Hkv);
+  return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
 size_t wpattn_decode_noalloc_max_bytes(void) { return kDecodeStaticScratchBytes; }

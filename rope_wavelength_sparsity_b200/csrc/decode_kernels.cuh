@@ -95,7 +95,13 @@ __device__ __forceinline__ uint4 ring_chunk(const uint8_t* tile, int r, int c) {
 // memory (broadcast), so the window removes work and no cross-lane reduction
 // is needed.  For O += p V a lane owns one 16-byte chunk of the head dim for
 // 32 / (D / 8) keys at a time.
-template <int D, int GC>
+//
+// PM (pair-major K cache): K is stored as [B, Hkv, D/16, Lmax, 16], slab g
+// holding dims 8g..8g+7 and P+8g..P+8g+7 of every key (the 8 pairs of one
+// group).  The producer then loads only the slabs still kept for the block
+// (1 KB each, from the first kept group on), so the window cuts DRAM bytes;
+// in the ring, slab g of a block sits at 1 KB * g, key r at 32 bytes * r.
+template <int D, int GC, bool PM>
 __global__ void __launch_bounds__((kDecodeComputeWarps + 1) * 32, GC <= 4 ? 3 : 2)
 decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ DecodeParams p) {
@@ -136,6 +142,15 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   const int nblk = j_end > j_begin ? (j_end - j_begin + KB - 1) / KB : 0;
   const int qpos = Lb - 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // first group of 8 pairs kept for some key of the block starting at j0:
+  // groups whose largest threshold is below the block's smallest distance
+  // (that of its last real key) are pruned for every key of the block
+  auto first_kept_group = [&](int j0) -> int {
+    const int dmin = qpos - (min(j0 + KB, j_end) - 1);
+    int g0 = 0;
+    while (g0 < NG && sT[8 * g0 + 7] < dmin) ++g0;
+    return g0;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -159,11 +174,20 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       for (int i = 0; i < nblk; ++i) {
         const int s = i % NS;
         if (i >= NS && !mbar_wait(empty(s), ((i / NS) & 1) ^ 1)) break;
-        mbar_arrive_expect_tx(full(s), 2 * L::TILE);
         const int j0 = j_begin + i * KB;
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_4d(sbase + L::OFF_K + s * L::TILE + c * L::PANEL, &tmK, full(s), 64 * c, j0, kvh, b);
-          tma_load_4d(sbase + L::OFF_V + s * L::TILE + c * L::PANEL, &tmV, full(s), 64 * c, j0, kvh, b);
+        if (PM) {
+          const int g0 = first_kept_group(j0);
+          mbar_arrive_expect_tx(full(s), (NG - g0) * KB * 32 + L::TILE);
+          for (int g = g0; g < NG; ++g)
+            tma_load_4d(sbase + L::OFF_K + s * L::TILE + g * KB * 32, &tmK, full(s), 0, j0, kvh * NG + g, b);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(sbase + L::OFF_V + s * L::TILE + c * L::PANEL, &tmV, full(s), 64 * c, j0, kvh, b);
+        } else {
+          mbar_arrive_expect_tx(full(s), 2 * L::TILE);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_4d(sbase + L::OFF_K + s * L::TILE + c * L::PANEL, &tmK, full(s), 64 * c, j0, kvh, b);
+            tma_load_4d(sbase + L::OFF_V + s * L::TILE + c * L::PANEL, &tmV, full(s), 64 * c, j0, kvh, b);
+          }
         }
       }
     }
@@ -192,11 +216,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     const int j = j0 + lane;              // this lane's key
     const bool valid = j < j_end;
     const int dist = qpos - j;
-    // smallest distance of a real key in the block: groups whose largest
-    // threshold is below it are pruned for every key of the block
-    const int dmin = qpos - (min(j0 + KB, j_end) - 1);
-    int g0 = 0;
-    while (g0 < NG && sT[8 * g0 + 7] < dmin) ++g0;
+    const int g0 = first_kept_group(j0);
 
     // ---- scores: one key per lane, groups g0 .. NG-1
     float sc[GC];
@@ -207,8 +227,14 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       float kf[16];
       {
         float a[8], bb[8];
-        unpack8(ring_chunk<D>(kt, lane, g), a);            // dims 8g .. 8g+7
-        unpack8(ring_chunk<D>(kt, lane, NG + g), bb);      // dims P+8g .. P+8g+7
+        if (PM) {  // this key's 32-byte row of slab g
+          const uint4* row = reinterpret_cast<const uint4*>(kt + g * KB * 32 + lane * 32);
+          unpack8(row[0], a);
+          unpack8(row[1], bb);
+        } else {
+          unpack8(ring_chunk<D>(kt, lane, g), a);            // dims 8g .. 8g+7
+          unpack8(ring_chunk<D>(kt, lane, NG + g), bb);      // dims P+8g .. P+8g+7
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) { kf[e] = a[e]; kf[8 + e] = bb[e]; }
       }
@@ -324,6 +350,31 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       rec[D + 1] = Ls;
     }
   }
+}
+
+// K cache [B, Lmax, Hkv, D] -> pair-major slabs [B, Hkv, D/16, Lmax, 16]:
+// slab g of a key holds dims 8g..8g+7 then D/2+8g..D/2+8g+7 (the 8 pairs of
+// group g).  One thread per (batch, kv head, slab, key), in slab order, so
+// consecutive threads write consecutive 32-byte rows.
+template <int D>
+__global__ void __launch_bounds__(256)
+kcache_to_pairmajor_kernel(const uint16_t* __restrict__ k, uint16_t* __restrict__ slabs, int64_t Lmax,
+                           int B, int Hkv) {
+  constexpr int NG = D / 16, P = D / 2;
+  const uint64_t idx = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const uint64_t n = static_cast<uint64_t>(B) * Hkv * NG * static_cast<uint64_t>(Lmax);
+  if (idx >= n) return;
+  const uint64_t j = idx % static_cast<uint64_t>(Lmax);
+  const uint64_t plane = idx / static_cast<uint64_t>(Lmax);   // (b * Hkv + h) * NG + g
+  const int g = static_cast<int>(plane % NG);
+  const uint64_t bh = plane / NG;                              // b * Hkv + h
+  const uint64_t b = bh / Hkv, h = bh % Hkv;
+  const uint16_t* row = k + ((b * static_cast<uint64_t>(Lmax) + j) * Hkv + h) * D;
+  const uint4 lo = *reinterpret_cast<const uint4*>(row + 8 * g);
+  const uint4 hi = *reinterpret_cast<const uint4*>(row + P + 8 * g);
+  uint4* dst = reinterpret_cast<uint4*>(slabs + idx * 16);
+  dst[0] = lo;
+  dst[1] = hi;
 }
 
 // Merge the S key ranges of each (sequence, query head): out = sum_s w_s o_s
