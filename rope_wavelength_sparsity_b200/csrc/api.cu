@@ -103,17 +103,19 @@ int encode_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
 }
 
 template <int D, bool G8>
-int launch_prefill(const void* q, const void* k, const void* v, const PrefillParams& prm,
+int launch_prefill(const void* q, const void* k, const void* v, PrefillParams prm,
                    DeviceInfo* dev, cudaStream_t st) {
+  using Shape = PrefillShape<D>;
   CUtensorMap tq, tk, tv;
   int rc;
+  prm.num_ctas_q = (prm.Nq + Shape::QT * kBM - 1) / (Shape::QT * kBM);
   // tensors are [B, N, H, D]: dims (fastest first) D, N, H, B
   if ((rc = encode_bf16_4d(&tq, q, D, prm.Nq, prm.Hq, prm.B, 8, kBM, false)) != WPATTN_OK) return rc;
   // with no key the kernel issues no K/V load; the maps only need to be valid
   const uint64_t nk = prm.Nk > 0 ? prm.Nk : prm.Nq;
   const uint64_t hk = prm.Nk > 0 ? prm.Hkv : prm.Hq;
-  if ((rc = encode_bf16_4d(&tk, k, D, nk, hk, prm.B, 8, kBN, false)) != WPATTN_OK) return rc;
-  if ((rc = encode_bf16_4d(&tv, v, D, nk, hk, prm.B, 64, kBN, true)) != WPATTN_OK) return rc;
+  if ((rc = encode_bf16_4d(&tk, k, D, nk, hk, prm.B, 8, Shape::BN, false)) != WPATTN_OK) return rc;
+  if ((rc = encode_bf16_4d(&tv, v, D, nk, hk, prm.B, 64, Shape::BN, true)) != WPATTN_OK) return rc;
   constexpr int smem = PrefillSmem<D>::ALLOC;
   const int slot = (D == 64 ? 0 : 2) + (G8 ? 1 : 0);
   if (!dev->prefill_attr[slot]) {
@@ -123,7 +125,7 @@ int launch_prefill(const void* q, const void* k, const void* v, const PrefillPar
     dev->prefill_attr[slot] = true;
   }
   dim3 grid(prm.num_ctas_q, prm.Hq, prm.B);
-  prefill_kernel<D, G8><<<grid, kPrefillThreads, smem, st>>>(tq, tk, tv, prm);
+  prefill_kernel<D, G8><<<grid, Shape::THREADS, smem, st>>>(tq, tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
@@ -281,7 +283,6 @@ int wpattn_prefill(const wpattn_window* w, const void* q, const void* k, const v
   prm.out = static_cast<uint16_t*>(out);
   prm.lse = lse;
   prm.B = B; prm.Nq = Nq; prm.Nk = Nk; prm.Hq = Hq; prm.Hkv = Hkv; prm.G = Hq / Hkv;
-  prm.num_ctas_q = (Nq + kQT * kBM - 1) / (kQT * kBM);
   // the kernel works in positions relative to k_pos0, in 32-bit integers
   const int64_t qk_off = q_pos0 - k_pos0;
   if (qk_off < -(int64_t(1) << 30) || qk_off > (int64_t(1) << 30) || Nq > (1 << 30) ||

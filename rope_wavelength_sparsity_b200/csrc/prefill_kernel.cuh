@@ -42,15 +42,25 @@
 namespace wpattn {
 
 constexpr int kBM = 128;              // query rows per tile (TMEM lanes)
-constexpr int kBN = 128;              // keys per tile
-constexpr int kQT = 2;                // query tiles per CTA
-constexpr int kPrefillThreads = 384;  // 8 softmax warps + producer + MMA + 2 idle
-// Registers: launched at 168 per thread (384 x 168 = 64512); the softmax
-// warpgroups grow to 224 and warpgroup 2 (producer, MMA, idle) shrinks to 56:
-// 256 x 224 + 128 x 56 = 64512.
-constexpr uint32_t kRegsSoftmax = 224;
-constexpr uint32_t kRegsOther = 56;
 constexpr int kCT = 16;               // pairs per batch of the per-warp K transpose (g = 1)
+
+// Tile shape.  TMEM (128 lanes x 512 columns) holds, per query tile, S (BN
+// fp32 columns) and O (D columns).  Two query tiles on 128-key tiles fit
+// both head dims (2 x (128 + 128) = 512 columns at D = 128).  The kernel
+// also supports three query tiles on 96-key tiles (3 x (96 + 64) = 480
+// columns at D = 64); measured slower there (its 152-register softmax
+// warpgroups spill), so it is not selected.
+template <int D>
+struct PrefillShape {
+  static constexpr int QT = 2;                        // query tiles per CTA = softmax warpgroups
+  static constexpr int BN = 128;                      // keys per tile
+  static constexpr int THREADS = (QT + 1) * 128;      // + producer, MMA issuer, 2 idle warps
+  // Registers: launched at 65536 / THREADS per thread; the softmax warpgroups
+  // grow and the last warpgroup shrinks to 56:
+  //   QT = 2: 256 x 224 + 128 x 56 = 64512;  QT = 3: 384 x 152 + 128 x 56 = 65536.
+  static constexpr uint32_t REGS_SOFTMAX = (QT == 3) ? 152 : 224;
+  static constexpr uint32_t REGS_OTHER = 56;
+};
 
 struct PrefillParams {
   uint16_t* out;      // [B, Nq, Hq, D] bf16
@@ -65,19 +75,23 @@ struct PrefillParams {
 
 template <int D>
 struct PrefillSmem {
+  static constexpr int QT = PrefillShape<D>::QT, BN = PrefillShape<D>::BN;
   static constexpr int NS = (D == 64) ? 4 : 2;       // K/V ring depth
   static constexpr int NPOLY = 0;                    // of every 8 column pairs, exp2 on the FMA pipe
-  static constexpr int TILE = kBM * D * 2;           // one Q, K or V tile in bytes
+  static constexpr int QTILE = kBM * D * 2;          // one Q tile in bytes
+  static constexpr int KTILE = BN * D * 2;           // one K or V tile in bytes
+  static constexpr int PANEL_Q = kBM * 16;           // one 8-dim panel of a Q tile
+  static constexpr int PANEL_K = BN * 16;            // one 8-dim panel of a K tile
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + kQT * TILE;
-  static constexpr int OFF_V = OFF_K + NS * TILE;
-  static constexpr int OFF_QM = OFF_V + NS * TILE;        // masked first k-step of Q, per tile
-  static constexpr int OFF_CT = OFF_QM + kQT * 2 * kBM * 16;  // per-warp transposed K pairs
-  static constexpr int OFF_T = OFF_CT + 8 * kCT * 32 * 4;     // thresholds (64 x int32)
+  static constexpr int OFF_K = OFF_Q + QT * QTILE;
+  static constexpr int OFF_V = OFF_K + NS * KTILE;
+  static constexpr int OFF_QM = OFF_V + NS * KTILE;          // masked first k-step of Q, per tile
+  static constexpr int OFF_CT = OFF_QM + QT * 2 * PANEL_Q;    // per-warp transposed K pairs
+  static constexpr int OFF_T = OFF_CT + 4 * QT * kCT * 32 * 4;  // thresholds (64 x int32)
   static constexpr int OFF_BAR = OFF_T + 64 * 4;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
-  //           s_full[2], p_full[2], o_final[2], qm_init[2]
-  static constexpr int NBAR = 1 + 4 * NS + 8;
+  //           s_full[QT], p_full[QT], o_final[QT], qm_init[QT]
+  static constexpr int NBAR = 1 + 4 * NS + 4 * QT;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_TMEM + 16;
   static constexpr int ALLOC = BYTES;
@@ -95,15 +109,20 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 // G8: pairs share thresholds in groups of 8 (a compile-time switch, so the
 // two correction paths do not share a register allocation)
 template <int D, bool G8>
-__global__ void __launch_bounds__(kPrefillThreads, 1)
+__global__ void __launch_bounds__(PrefillShape<D>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ PrefillParams p) {
   using L = PrefillSmem<D>;
   constexpr int NS = L::NS;
+  constexpr int QT = PrefillShape<D>::QT;   // query tiles per CTA
+  constexpr int BN = PrefillShape<D>::BN;   // keys per tile
   constexpr int P = D / 2;
   constexpr int KS = D / 16;          // k-steps of the QK contraction (8 pairs each)
-  constexpr int PANEL = kBM * 16;     // bytes of one 8-dim column panel
-  constexpr uint32_t TMEM_O = 256;
+  constexpr int PANEL_Q = L::PANEL_Q;
+  constexpr int PANEL_K = L::PANEL_K;
+  constexpr int W_PROD = 4 * QT;      // producer warp (after the softmax warpgroups)
+  constexpr int W_MMA = 4 * QT + 1;   // MMA issuer warp
+  constexpr uint32_t TMEM_O = QT * BN;  // S_t at t * BN, O_t at TMEM_O + t * D
   constexpr uint32_t FULL = 0xffffffffu;
 
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -118,9 +137,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   auto v_full = [&](int s) { return bar + 8 * (1 + 2 * NS + s); };
   auto v_empty = [&](int s) { return bar + 8 * (1 + 3 * NS + s); };
   auto s_full = [&](int t) { return bar + 8 * (1 + 4 * NS + t); };
-  auto p_full = [&](int t) { return bar + 8 * (3 + 4 * NS + t); };
-  auto o_final = [&](int t) { return bar + 8 * (5 + 4 * NS + t); };
-  auto qm_init = [&](int t) { return bar + 8 * (7 + 4 * NS + t); };
+  auto p_full = [&](int t) { return bar + 8 * (1 + 4 * NS + QT + t); };
+  auto o_final = [&](int t) { return bar + 8 * (1 + 4 * NS + 2 * QT + t); };
+  auto qm_init = [&](int t) { return bar + 8 * (1 + 4 * NS + 3 * QT + t); };
 
   const uint32_t sQM = sbase + L::OFF_QM;
   int* sT = reinterpret_cast<int*>(smem + L::OFF_T);  // per-pair thresholds, read by every role
@@ -135,24 +154,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int cq = p.num_ctas_q - 1 - blockIdx.x;  // longest rows first
   const int h = blockIdx.y, b = blockIdx.z;
   const int kvh = h / p.G;
-  const int nkt = (p.Nk + kBN - 1) / kBN;
+  const int nkt = (p.Nk + BN - 1) / BN;
 
   // key tiles of query tile t: positions <= its last row, iterated from kt_top down
   auto last_key_tile = [&](int t) -> int {
-    const int row0 = (kQT * cq + t) * kBM;
+    const int row0 = (QT * cq + t) * kBM;
     if (row0 >= p.Nq || p.Nk <= 0) return -1;
     const int i_max = p.qk_off + min(row0 + kBM - 1, p.Nq - 1);
     if (i_max < 0) return -1;
-    return min(i_max / kBN, nkt - 1);
+    return min(i_max / BN, nkt - 1);
   };
-  const int kt_last0 = last_key_tile(0), kt_last1 = last_key_tile(1);
-  const int kt_top = max(kt_last0, kt_last1);
+  int kt_last[QT];
+#pragma unroll
+  for (int t = 0; t < QT; ++t) kt_last[t] = last_key_tile(t);
+  int kt_top = kt_last[0];
+#pragma unroll
+  for (int t = 1; t < QT; ++t) kt_top = max(kt_top, kt_last[t]);
   const int n_iter = kt_top + 1;  // shared K/V iterations j: key tile kt_top - j
   // Smallest distance of query tile t in key tile kt (negative on the diagonal).
   // Going down the key tiles it grows by 128, so the first kept pair of the
   // tile (p_min of that distance) only moves forward: advance it in place.
   auto advance_plo = [&](int t, int kt, int& plo) {
-    const int dlo = p.qk_off + (kQT * cq + t) * kBM - (kBN * kt + kBN - 1);
+    const int dlo = p.qk_off + (QT * cq + t) * kBM - (BN * kt + BN - 1);
     while (plo < P && sT[plo] < dlo) ++plo;
   };
   // Split pair of the tile: pairs plo .. ps-1 (kept somewhere in the tile) are
@@ -166,7 +189,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // (psr, carried by the caller) is advanced in place like plo.
   auto split_pair = [&](int t, int kt, int plo, int& psr) -> int {
     if (plo >= P) return plo;
-    const int dc = max(p.qk_off + (kQT * cq + t) * kBM - kBN * kt, 0);  // row 0 to key 0
+    const int dc = max(p.qk_off + (QT * cq + t) * kBM - BN * kt, 0);  // row 0 to key 0
     const int target = dc > 0x7FFFFFDF ? 0x7FFFFFFF : dc + 32;
     while (psr < P && sT[psr] < target) ++psr;
     return min(max(psr, plo), P - (G8 ? 8 : 1));
@@ -177,11 +200,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     mbar_init(q_full, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(k_full(s), 1);
-      mbar_init(k_empty(s), 1 + 8);  // MMA commit + 8 softmax warps (they read K for corrections)
+      mbar_init(k_empty(s), 1 + 4 * QT);  // MMA commit + every softmax warp (they read K for corrections)
       mbar_init(v_full(s), 1);
       mbar_init(v_empty(s), 1);
     }
-    for (int t = 0; t < kQT; ++t) {
+    for (int t = 0; t < QT; ++t) {
       mbar_init(s_full(t), 1);
       mbar_init(p_full(t), 4);
       mbar_init(o_final(t), 1);
@@ -190,7 +213,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == W_MMA) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -199,9 +222,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= 8) {
-  regs_decrease<kRegsOther>();
-  if (warp == 8) {
+  if (warp >= W_PROD) {
+  regs_decrease<PrefillShape<D>::REGS_OTHER>();
+  if (warp == W_PROD) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_iter > 0) {
       prefetch_tensormap(&tmQ);
@@ -209,72 +232,74 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       prefetch_tensormap(&tmV);
       // a query tile wholly past Nq is not loaded (its rows are never used)
       int nq_tiles = 0;
-      for (int t = 0; t < kQT; ++t) nq_tiles += ((kQT * cq + t) * kBM < p.Nq) ? 1 : 0;
-      mbar_arrive_expect_tx(q_full, nq_tiles * L::TILE);
+      for (int t = 0; t < QT; ++t) nq_tiles += ((QT * cq + t) * kBM < p.Nq) ? 1 : 0;
+      mbar_arrive_expect_tx(q_full, nq_tiles * L::QTILE);
       for (int t = 0; t < nq_tiles; ++t)
         for (int c = 0; c < D / 8; ++c)
-          tma_load_4d(sQ + t * L::TILE + c * PANEL, &tmQ, q_full, 8 * c, (kQT * cq + t) * kBM, h, b);
+          tma_load_4d(sQ + t * L::QTILE + c * PANEL_Q, &tmQ, q_full, 8 * c, (QT * cq + t) * kBM, h, b);
       for (int j = 0; j < n_iter; ++j) {
         const int kt = kt_top - j;
         const int s = j % NS;
         const uint32_t ph = (j / NS) & 1;
         if (j >= NS && !mbar_wait(k_empty(s), ph ^ 1)) break;
-        mbar_arrive_expect_tx(k_full(s), L::TILE);
+        mbar_arrive_expect_tx(k_full(s), L::KTILE);
         for (int c = 0; c < D / 8; ++c)
-          tma_load_4d(sK + s * L::TILE + c * PANEL, &tmK, k_full(s), 8 * c, kBN * kt, kvh, b);
+          tma_load_4d(sK + s * L::KTILE + c * PANEL_K, &tmK, k_full(s), 8 * c, BN * kt, kvh, b);
         if (j >= NS && !mbar_wait(v_empty(s), ph ^ 1)) break;
-        mbar_arrive_expect_tx(v_full(s), L::TILE);
+        mbar_arrive_expect_tx(v_full(s), L::KTILE);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sV + s * L::TILE + c * (kBN * 128), &tmV, v_full(s), 64 * c, kBN * kt, kvh, b);
+          tma_load_4d(sV + s * L::KTILE + c * (BN * 128), &tmV, v_full(s), 64 * c, BN * kt, kvh, b);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == W_MMA) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && n_iter > 0) {
-      constexpr uint32_t idesc_qk = make_idesc_bf16(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc_qk = make_idesc_bf16(kBM, BN, 0, 0);
       constexpr uint32_t idesc_pv = make_idesc_bf16(kBM, D, 0, 1);
-      constexpr uint32_t LBO_QK = (D / 16) * PANEL;  // first half -> second half of a pair
       bool ok = mbar_wait(q_full, 0);
-      int cnt0 = 0, cnt1 = 0;  // tiles processed so far by query tile 0 / 1
-      bool qm_seen0 = false, qm_seen1 = false;
-      int plo0 = 0, plo1 = 0, psr0 = 0, psr1 = 0;
-      // descriptors: start addresses advance by adding (byte offset >> 4)
-      const uint64_t qdesc0 = make_sdesc(sQ, LBO_QK, 128, 0);
-      const uint64_t qmdesc0 = make_sdesc(sQM, PANEL, 128, 0);
-      const uint64_t kdesc0 = make_sdesc(sK, LBO_QK, 128, 0);
-      const uint64_t vdesc0 = make_sdesc(sV, kBN * 128, 1024, 2);
+      // per query tile (indices are compile-time after unrolling): PVs issued,
+      // masked-Q barrier seen, planner state
+      int cnt[QT], plo[QT], psr[QT];
+      bool qm_seen[QT];
+#pragma unroll
+      for (int t = 0; t < QT; ++t) { cnt[t] = 0; plo[t] = 0; psr[t] = 0; qm_seen[t] = false; }
+      // descriptors: start addresses advance by adding (byte offset >> 4);
+      // LBO = D/16 panels: first half -> second half of a pair
+      const uint64_t qdesc0 = make_sdesc(sQ, (D / 16) * PANEL_Q, 128, 0);
+      const uint64_t qmdesc0 = make_sdesc(sQM, PANEL_Q, 128, 0);
+      const uint64_t kdesc0 = make_sdesc(sK, (D / 16) * PANEL_K, 128, 0);
+      const uint64_t vdesc0 = make_sdesc(sV, BN * 128, 1024, 2);
       // split pair of QK_t(j): planned ahead of the wait for P_t(j - 1)
       auto plan_qk = [&](int t, int j) -> int {
         const int kt = kt_top - j;
-        int& plo = t ? plo1 : plo0;
-        advance_plo(t, kt, plo);
-        return split_pair(t, kt, plo, t ? psr1 : psr0);
+        advance_plo(t, kt, plo[t]);
+        return split_pair(t, kt, plo[t], psr[t]);
       };
       auto issue_qk = [&](int t, int j, int ps) -> bool {
-        bool& seen = t ? qm_seen1 : qm_seen0;
-        if (!seen) {  // the softmax warps prepared the masked k-step of tile t's first tile
+        if (!qm_seen[t]) {  // the softmax warps prepared the masked k-step of tile t's first tile
           if (!mbar_wait(qm_init(t), 0)) return false;
-          seen = true;
+          qm_seen[t] = true;
         }
         const int k0 = ps >> 3;
-        const uint64_t kbase = kdesc0 + (uint64_t)(((j % NS) * L::TILE) >> 4);
-        const uint64_t qbase = qdesc0 + (uint64_t)((t * L::TILE) >> 4);
-        const uint32_t d_tmem = tmem + t * kBN;
+        const uint64_t kbase = kdesc0 + (uint64_t)(((j % NS) * L::KTILE) >> 4);
+        const uint64_t qbase = qdesc0 + (uint64_t)((t * L::QTILE) >> 4);
+        const uint32_t d_tmem = tmem + t * BN;
         for (int ks = k0; ks < KS; ++ks) {
           // pairs 8*k0 .. ps-1 are not contracted: the first step reads a
           // copy of Q with those pairs zeroed
           const uint64_t ad = (ks == k0 && (ps & 7))
-                                  ? qmdesc0 + (uint64_t)((t * 2 * PANEL) >> 4)
-                                  : qbase + (uint64_t)((ks * PANEL) >> 4);
-          umma_ss(d_tmem, ad, kbase + (uint64_t)((ks * PANEL) >> 4), idesc_qk, ks > k0 ? 1u : 0u);
+                                  ? qmdesc0 + (uint64_t)((t * 2 * PANEL_Q) >> 4)
+                                  : qbase + (uint64_t)((ks * PANEL_Q) >> 4);
+          umma_ss(d_tmem, ad, kbase + (uint64_t)((ks * PANEL_K) >> 4), idesc_qk, ks > k0 ? 1u : 0u);
         }
         umma_commit(s_full(t));
         return true;
       };
       if (ok && mbar_wait(k_full(0), 0)) {
         tc_fence_after();
-        if (kt_last0 >= kt_top && !issue_qk(0, 0, plan_qk(0, 0))) ok = false;
-        if (ok && kt_last1 >= kt_top && !issue_qk(1, 0, plan_qk(1, 0))) ok = false;
+#pragma unroll
+        for (int t = 0; t < QT; ++t)
+          if (ok && kt_last[t] >= kt_top && !issue_qk(t, 0, plan_qk(t, 0))) ok = false;
         umma_commit(k_empty(0));
       } else {
         ok = false;
@@ -284,22 +309,21 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const bool next = j + 1 < n_iter;
         if (next && !mbar_wait(k_full((j + 1) % NS), ((j + 1) / NS) & 1)) { ok = false; break; }
         if (!mbar_wait(v_full(j % NS), (j / NS) & 1)) { ok = false; break; }
-        const uint64_t vbase = vdesc0 + (uint64_t)(((j % NS) * L::TILE) >> 4);
+        const uint64_t vbase = vdesc0 + (uint64_t)(((j % NS) * L::KTILE) >> 4);
 #pragma unroll
-        for (int t = 0; t < kQT; ++t) {
-          const int ktl = t ? kt_last1 : kt_last0;
-          int& cnt = t ? cnt1 : cnt0;
+        for (int t = 0; t < QT; ++t) {
+          const int ktl = kt_last[t];
           const bool do_qk = ok && next && kt - 1 <= ktl;
           const int ps_n = do_qk ? plan_qk(t, j + 1) : 0;
           if (ok && kt <= ktl) {
-            if (!mbar_wait(p_full(t), cnt & 1)) { ok = false; }
+            if (!mbar_wait(p_full(t), cnt[t] & 1)) { ok = false; }
             if (ok) {
               tc_fence_after();
 #pragma unroll
-              for (int ks = 0; ks < kBN / 16; ++ks)
-                umma_ts(tmem + TMEM_O + t * D, tmem + t * kBN + ks * 8,
-                        vbase + (uint64_t)((ks * 2048) >> 4), idesc_pv, (cnt > 0 || ks > 0) ? 1u : 0u);
-              ++cnt;
+              for (int ks = 0; ks < BN / 16; ++ks)
+                umma_ts(tmem + TMEM_O + t * D, tmem + t * BN + ks * 8,
+                        vbase + (uint64_t)((ks * 2048) >> 4), idesc_pv, (cnt[t] > 0 || ks > 0) ? 1u : 0u);
+              ++cnt[t];
             }
           }
           if (ok && do_qk && !issue_qk(t, j + 1, ps_n)) ok = false;
@@ -309,25 +333,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (next) umma_commit(k_empty((j + 1) % NS));
       }
       // O_t final: every MMA issued so far has completed once this arrives
-      for (int t = 0; t < kQT; ++t) umma_commit(o_final(t));
+      for (int t = 0; t < QT; ++t) umma_commit(o_final(t));
       if (!ok) mbar_wait(o_final(0), 0);
     }
   }
   } else {
-    regs_increase<kRegsSoftmax>();
+    regs_increase<PrefillShape<D>::REGS_SOFTMAX>();
     // ------------------------------------------------------------- softmax
     const int t = warp >> 2;                   // query tile of this warpgroup
     const int wq = warp & 3;                   // TMEM lane quarter
     const int r = wq * 32 + lane;              // row within the tile = TMEM lane
-    const int row = (kQT * cq + t) * kBM + r;  // query index
+    const int row = (QT * cq + t) * kBM + r;   // query index
     const int i_pos = p.qk_off + row;          // relative position of this row
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const uint32_t tS = lane_base + t * kBN;
+    const uint32_t tS = lane_base + t * BN;
     const uint32_t tO = lane_base + TMEM_O + t * D;
-    const uint8_t* smem_q = smem + L::OFF_Q + t * L::TILE;
-    uint8_t* smem_qm = smem + L::OFF_QM + t * 2 * PANEL;
-    const int i_tile0 = p.qk_off + (kQT * cq + t) * kBM;  // relative position of the first row
-    const int my_kt_last = t ? kt_last1 : kt_last0;
+    const uint8_t* smem_q = smem + L::OFF_Q + t * L::QTILE;
+    uint8_t* smem_qm = smem + L::OFF_QM + t * 2 * PANEL_Q;
+    const int i_tile0 = p.qk_off + (QT * cq + t) * kBM;  // relative position of the first row
+    const int my_kt_last = last_key_tile(t);
     float m_ref = -INFINITY;   // exponent reference of O and l (log2 units)
     float l_run = 0.f;
     int cnt = 0;
@@ -338,8 +362,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     auto write_masked_q = [&](int ps) {
       const int rz = ps & 7;
       if (rz == 0 || (ps >> 3) >= KS) return;
-      uint4 lo = *reinterpret_cast<const uint4*>(smem_q + (ps >> 3) * PANEL + r * 16);
-      uint4 hi = *reinterpret_cast<const uint4*>(smem_q + (P / 8 + (ps >> 3)) * PANEL + r * 16);
+      uint4 lo = *reinterpret_cast<const uint4*>(smem_q + (ps >> 3) * PANEL_Q + r * 16);
+      uint4 hi = *reinterpret_cast<const uint4*>(smem_q + (P / 8 + (ps >> 3)) * PANEL_Q + r * 16);
       const uint32_t m0 = (rz > 0 ? 0u : 0xFFFFu) | (rz > 1 ? 0u : 0xFFFF0000u);
       const uint32_t m1 = (rz > 2 ? 0u : 0xFFFFu) | (rz > 3 ? 0u : 0xFFFF0000u);
       const uint32_t m2 = (rz > 4 ? 0u : 0xFFFFu) | (rz > 5 ? 0u : 0xFFFF0000u);
@@ -347,7 +371,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       lo.x &= m0; lo.y &= m1; lo.z &= m2; lo.w &= m3;
       hi.x &= m0; hi.y &= m1; hi.z &= m2; hi.w &= m3;
       *reinterpret_cast<uint4*>(smem_qm + r * 16) = lo;
-      *reinterpret_cast<uint4*>(smem_qm + PANEL + r * 16) = hi;
+      *reinterpret_cast<uint4*>(smem_qm + PANEL_Q + r * 16) = hi;
       fence_proxy_async_smem();
     };
 
@@ -373,7 +397,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (lane == 0) mbar_arrive(k_empty(s));
         continue;
       }
-      const int kp0 = kBN * kt;
+      const int kp0 = BN * kt;
       const int d_row = i_pos - kp0;         // distance to the tile's first key
       const int plo = plo_next, ps = ps_next;
       const bool all_pruned = plo >= P;
@@ -392,16 +416,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // is ready; for g = 8 they are applied to S in TMEM before it is read.
       const bool need_sub = !all_pruned && __any_sync(FULL, d_row > sT[ps]);
       const bool need_add = !all_pruned && ps > plo &&
-                            __any_sync(FULL, d_row >= 0 && d_row - (kBN - 1) <= sT[ps - 1]);
+                            __any_sync(FULL, d_row >= 0 && d_row - (BN - 1) <= sT[ps - 1]);
       const bool corr = need_sub || need_add;
       // K stage s is released below; waiting for its fill first makes the
       // arrival count towards iteration j (the stage's previous phase is over)
       if (!__all_sync(FULL, mbar_wait(k_full(s), (j / NS) & 1))) { ok = false; break; }
-      float sc[kBN];
+      float sc[BN];
       if (corr && !G8) {
-        const uint8_t* kb = smem + L::OFF_K + s * L::TILE;
+        const uint8_t* kb = smem + L::OFF_K + s * L::KTILE;
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) sc[c] = 0.f;
+        for (int c = 0; c < BN; ++c) sc[c] = 0.f;
         // the chunk loops are not unrolled (this path runs on few tiles and
         // must stay small in the instruction cache): a chunk's terms are
         // summed into dl and added to sc by a switch on the chunk index
@@ -416,7 +440,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint32_t* ct = reinterpret_cast<uint32_t*>(smem + L::OFF_CT) + warp * (kCT * 32);
         const int T_lo = ps > plo ? sT[ps - 1] : 0;
 #pragma unroll 1
-        for (int cc = 0; cc < kBN / 32; ++cc) {
+        for (int cc = 0; cc < BN / 32; ++cc) {
           const int dc = d_row - 32 * cc;                  // distance at the chunk's first column
           const int dmax = __shfl_sync(FULL, dc, 31);      // largest distance of the block
           const int dmin = max(__shfl_sync(FULL, dc, 0) - 31, 0);
@@ -439,9 +463,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             const uint8_t* krow = kb + (32 * cc + lane) * 16;
 #pragma unroll 1
             for (int pp = p0; pp < p1; ++pp) {
-              const int o = (pp >> 3) * PANEL + (pp & 7) * 2;
+              const int o = (pp >> 3) * PANEL_K + (pp & 7) * 2;
               const uint32_t klo = *reinterpret_cast<const uint16_t*>(krow + o);
-              const uint32_t khi = *reinterpret_cast<const uint16_t*>(krow + o + (P / 8) * PANEL);
+              const uint32_t khi = *reinterpret_cast<const uint16_t*>(krow + o + (P / 8) * PANEL_K);
               ct[(pp - p0) * 32 + lane] = klo | (khi << 16);
             }
             __syncwarp();
@@ -459,9 +483,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 hi = min(dc, 31);
                 sgn = 1.f;
               }
-              const int o = (pp >> 3) * PANEL + (pp & 7) * 2 + r * 16;
+              const int o = (pp >> 3) * PANEL_Q + (pp & 7) * 2 + r * 16;
               const float qa = sgn * __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + o)) << 16);
-              const float qb = sgn * __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + o + (P / 8) * PANEL)) << 16);
+              const float qb = sgn * __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + o + (P / 8) * PANEL_Q)) << 16);
               const uint4* w4 = reinterpret_cast<const uint4*>(ct + (pp - p0) * 32);
 #pragma unroll
               for (int c4 = 0; c4 < 8; ++c4) {
@@ -481,7 +505,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             WPATTN_ADD_CHUNK(0)
             WPATTN_ADD_CHUNK(1)
             WPATTN_ADD_CHUNK(2)
-            WPATTN_ADD_CHUNK(3)
+            default:  // chunk 3 (128-key tiles only)
+              if constexpr (BN > 96) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) sc[96 + c] += dl[c];
+              }
+              break;
           }
         }
 #undef WPATTN_ADD_CHUNK
@@ -494,7 +523,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!__all_sync(FULL, mbar_wait(s_full(t), cnt & 1))) { ok = false; break; }
       tc_fence_after();
       if (corr && G8) {
-        const uint8_t* kb = smem + L::OFF_K + s * L::TILE;
+        const uint8_t* kb = smem + L::OFF_K + s * L::KTILE;
         // whole groups of 8 pairs share a threshold: one 16-dim dot product per element
 #pragma unroll 1
         for (int gp = plo; gp < P; gp += 8) {
@@ -503,22 +532,21 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           int c_lo, c_hi;  // columns of this row that take the group's term
           if (sub) {
             c_lo = 0;
-            c_hi = d_row > T ? min(d_row - T - 1, kBN - 1) : -1;
+            c_hi = d_row > T ? min(d_row - T - 1, BN - 1) : -1;
           } else {
             c_lo = T >= d_row ? 0 : d_row - T;
-            c_hi = min(d_row, kBN - 1);
+            c_hi = min(d_row, BN - 1);
           }
           if (!__any_sync(FULL, c_lo <= c_hi)) {
             if (sub) break;  // later groups are pruned at even fewer columns
             continue;
           }
           const float sgn = sub ? -1.f : 1.f;
-          const int off_lo = (gp >> 3) * PANEL;
-          const int off_hi = (P / 8 + (gp >> 3)) * PANEL;
+          const int grp = gp >> 3;
           float qv[16];
           {
-            const uint4 a = *reinterpret_cast<const uint4*>(smem_q + off_lo + r * 16);
-            const uint4 c = *reinterpret_cast<const uint4*>(smem_q + off_hi + r * 16);
+            const uint4 a = *reinterpret_cast<const uint4*>(smem_q + grp * PANEL_Q + r * 16);
+            const uint4 c = *reinterpret_cast<const uint4*>(smem_q + (P / 8 + grp) * PANEL_Q + r * 16);
             qv[0] = bf16lo_to_f32(a.x); qv[1] = bf16hi_to_f32(a.x);
             qv[2] = bf16lo_to_f32(a.y); qv[3] = bf16hi_to_f32(a.y);
             qv[4] = bf16lo_to_f32(a.z); qv[5] = bf16hi_to_f32(a.z);
@@ -529,7 +557,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             qv[14] = bf16lo_to_f32(c.w); qv[15] = bf16hi_to_f32(c.w);
           }
 #pragma unroll 1
-          for (int cc = 0; cc < kBN / 32; ++cc) {
+          for (int cc = 0; cc < BN / 32; ++cc) {
             const int lo = c_lo - 32 * cc, hi = c_hi - 32 * cc;  // chunk-local range
             if (!__any_sync(FULL, lo <= 31 && hi >= 0 && lo <= hi)) continue;
             float v[32];
@@ -537,8 +565,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tmem_ld_wait();
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              const uint4 a = *reinterpret_cast<const uint4*>(kb + off_lo + (32 * cc + c) * 16);
-              const uint4 b2 = *reinterpret_cast<const uint4*>(kb + off_hi + (32 * cc + c) * 16);
+              const uint4 a = *reinterpret_cast<const uint4*>(kb + grp * PANEL_K + (32 * cc + c) * 16);
+              const uint4 b2 = *reinterpret_cast<const uint4*>(kb + (P / 8 + grp) * PANEL_K + (32 * cc + c) * 16);
               float d0 = 0.f, d1 = 0.f;
               fma2(d0, d1, qv[0], qv[1], bf16lo_to_f32(a.x), bf16hi_to_f32(a.x), d0, d1);
               fma2(d0, d1, qv[2], qv[3], bf16lo_to_f32(a.y), bf16hi_to_f32(a.y), d0, d1);
@@ -559,7 +587,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       if (corr && !G8) {
 #pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) {
+        for (int cc = 0; cc < BN / 32; ++cc) {
           float v[32];
           tmem_ld32(tS + 32 * cc, v);
           tmem_ld_wait();
@@ -568,29 +596,40 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
       } else {
 #pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) tmem_ld32(tS + 32 * cc, &sc[32 * cc]);
+        for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(tS + 32 * cc, &sc[32 * cc]);
         tmem_ld_wait();
       }
 
       if (all_pruned) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) sc[c] = 0.f;   // every pair pruned: score 0
+        for (int c = 0; c < BN; ++c) sc[c] = 0.f;   // every pair pruned: score 0
       }
 
       // causal mask (d < 0) and the ragged key tail: columns c > cm
-      const bool need_mask = (i_tile0 - (kp0 + kBN - 1) < 0) || (kp0 + kBN > p.Nk);
-      int cm = kBN - 1;
+      const bool need_mask = (i_tile0 - (kp0 + BN - 1) < 0) || (kp0 + BN > p.Nk);
+      int cm = BN - 1;
       if (need_mask) {
         // last column with d >= 0, and the last real key
-        cm = min(max(min(d_row, p.Nk - 1 - kp0), -1), kBN);
+        cm = min(max(min(d_row, p.Nk - 1 - kp0), -1), BN);
 #pragma unroll
-        for (int c = 0; c < kBN; ++c)
+        for (int c = 0; c < BN; ++c)
           if (c > cm) sc[c] = -INFINITY;
       }
 
       // Row max first, then the exponentials against the (lazily moved) reference.
       const float sl = p.scale_log2;
       auto tile_max = [&]() -> float {
+        if constexpr (BN == 96) {
+          float a12[12];
+#pragma unroll
+          for (int k = 0; k < 12; ++k)
+            a12[k] = max3(max3(sc[8 * k], sc[8 * k + 1], sc[8 * k + 2]),
+                          max3(sc[8 * k + 3], sc[8 * k + 4], sc[8 * k + 5]),
+                          fmaxf(sc[8 * k + 6], sc[8 * k + 7]));
+          const float b0 = max3(a12[0], a12[1], a12[2]), b1 = max3(a12[3], a12[4], a12[5]);
+          const float b2 = max3(a12[6], a12[7], a12[8]), b3 = max3(a12[9], a12[10], a12[11]);
+          return fmaxf(max3(b0, b1, b2), b3) * sl;
+        }
         float a16[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
@@ -604,15 +643,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         return max3(max3(b6[0], b6[1], b6[2]), max3(b6[3], b6[4], b6[5]), -INFINITY) * sl;
       };
       // p for every column against reference m, packed to bf16 pairs in pk;
-      // returns the row sum of p
-      uint32_t pk[kBN / 2];
+      // returns the row sum of p.  With 96-key tiles P is stored 16 columns
+      // at a time as it is produced (fewer live registers).
+      uint32_t pk[BN / 2];
       auto exps = [&](float m) -> float {
         const float nm = (m == -INFINITY) ? 0.f : -m;
         float acc[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[k] = 0.f;
 #pragma unroll
-        for (int i = 0; i < kBN / 2; ++i) {
+        for (int i = 0; i < BN / 2; ++i) {
           const int c = 2 * i;
           float x0, x1, e0, e1;
           fma2(x0, x1, sc[c], sc[c + 1], sl, sl, nm, nm);
@@ -624,6 +664,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           add2(acc[2 * (i & 3)], acc[2 * (i & 3) + 1], acc[2 * (i & 3)], acc[2 * (i & 3) + 1], e0, e1);
           pk[i] = pack_bf16x2(e0, e1);
+          if constexpr (BN == 96) {
+            if ((i & 15) == 15) tmem_st16u(tS + (i - 15), &pk[i - 15]);
+          }
         }
         return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
       };
@@ -651,8 +694,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       const float rowsum = exps(m_ref);
       l_run = l_run * f + rowsum;
-      tmem_st32u(tS, &pk[0]);       // P overwrites the first 64 columns of S
-      tmem_st32u(tS + 32, &pk[32]);
+      if constexpr (BN == 128) {     // P overwrites the first 64 columns of S
+        tmem_st32u(tS, &pk[0]);
+        tmem_st32u(tS + 32, &pk[32]);
+      }
       // the next tile's masked Q step, before P is released to the MMA warp
       if (kt > 0) write_masked_q(ps_next);
       tmem_st_wait();
