@@ -48,8 +48,8 @@ FLUSH_BYTES = 512 << 20
 # that kernel's sources at capture time: a changed kernel reports null until
 # it is captured again.
 NCU_TRAFFIC = {
-    # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.152832 MB read + 25.150464 MB written
-    ("qwen2.5-0.5b-32k", "91a245467242c9f1"): 101303296,
+    # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.134912 MB read + 23.742208 MB written
+    ("qwen2.5-0.5b-32k", "78ae9ff5d51882a2"): 76134912 + 23742208,
     # profiles/decode_split_kernel_llama3.2-3b-decode-32k.md: 536.926464 MB read + 5.638144 MB
     # written for B=4, L=32768, scaled by the 16x keys x heads of the B=16, L=131072 call
     ("llama3.2-3b-decode-128k", "247125b8d0a5fc28"): 16 * (536926464 + 5638144),
