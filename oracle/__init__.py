@@ -58,6 +58,10 @@ def _load():
             lib.oracle_scores.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
                                           ctypes.c_int64, ctypes.c_double, ctypes.c_double,
                                           ctypes.c_int, vp]
+            lib.oracle_decode_positions.argtypes = [
+                vp, vp, vp, vp, vp, vp, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                ctypes.c_int, ctypes.c_double, ctypes.c_int64, vp, vp, vp]
             for name in ("oracle_count_bruteforce", "oracle_count_rows"):
                 getattr(lib, name).argtypes = [ctypes.c_int, ctypes.c_double, ctypes.c_double,
                                                ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
@@ -140,6 +144,38 @@ def decode_rows(q, k_cache, v_cache, kv_len, *, Hq, Hkv, base, alpha, g, scale, 
         outs.append(o[0])
         lses.append(l[0])
     return np.stack(outs), np.array(lses)
+
+
+def decode_positions(q, k_cache, v_cache, kv_len, q_pos, k_pos, *, Hq, Hkv, base, alpha, g,
+                     scale, rows=None):
+    """Decode with explicit positions: the query of sequence b sits at q_pos[b] and
+    its key j < kv_len[b] at k_pos[b, j]; keys past the query are excluded.
+
+    q: uint16 [B, Hq, D]; caches uint16 [B, Lmax, Hkv, D]; k_pos int [B, >= max kv_len].
+    ATFlash Abstract: the window is a function of the relative position q_pos - k_pos.
+    """
+    lib = _load()
+    q, k_cache, v_cache = _u16(q), _u16(k_cache), _u16(v_cache)
+    B, _, D = q.shape
+    Lmax = k_cache.shape[1]
+    kvl = np.ascontiguousarray(np.asarray(kv_len, dtype=np.int64).reshape(B))
+    qp = np.ascontiguousarray(np.asarray(q_pos, dtype=np.int64).reshape(B))
+    kp = np.ascontiguousarray(np.asarray(k_pos, dtype=np.int64).reshape(B, -1))
+    if kp.shape[1] < int(kvl.max(initial=0)):
+        raise ValueError("k_pos has fewer columns than the longest sequence")
+    if rows is None:
+        rows = [(b, h) for b in range(B) for h in range(Hq)]
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 2))
+    n = rows.shape[0]
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros(n, dtype=np.float64)
+    rc = lib.oracle_decode_positions(
+        q.ctypes.data, k_cache.ctypes.data, v_cache.ctypes.data, kvl.ctypes.data,
+        qp.ctypes.data, kp.ctypes.data, kp.shape[1], B, Lmax, Hq, Hkv, D, base, alpha, g,
+        scale, n, rows.ctypes.data, out.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_decode_positions failed ({rc})")
+    return out, lse
 
 
 def scores(qrow, keys, *, q_pos, k_pos0=0, base, alpha, g):

@@ -278,3 +278,108 @@ def test_decode_rows_match_causal_sdpa_when_window_off():
             np.testing.assert_allclose(out[n], want.numpy(), atol=1e-10)
             assert abs(lse[n] - float(torch.logsumexp(z, 0))) < 1e-10
             n += 1
+
+
+# ---------------------------------------------------------------------------
+# decode with explicit key positions (ATFlash Abstract: the kept pair set is a
+# function of the relative position q_pos - k_pos alone)
+# ---------------------------------------------------------------------------
+
+def test_positions_hand_case():
+    """D = 4, base 100, alpha 1 (T = (6, 62)), query (1, 2, 3, 4) at position 107.
+    Key A = (1, 1, 1, 1) at 100 (d = 7): pair 0 pruned, s = 2 + 4 = 6.
+    Key B = (0.5, 0, 0.25, 1) at 0 (d = 107 > 62): both pairs pruned, s = 0.
+    Key C = (1, 0, 0, 0) at 107 (d = 0): s = 1.  Key D at 108 is in the future:
+    excluded.  Weights (e^6, 1, e, 0) / Z with scale 1."""
+    q = _bf16_bits(np.array([1.0, 2.0, 3.0, 4.0]).reshape(1, 1, 4))
+    kk = np.zeros((1, 4, 1, 4))
+    vv = np.zeros((1, 4, 1, 4))
+    kk[0, 0, 0] = [1.0, 1.0, 1.0, 1.0]
+    kk[0, 1, 0] = [0.5, 0.0, 0.25, 1.0]
+    kk[0, 2, 0] = [1.0, 0.0, 0.0, 0.0]
+    kk[0, 3, 0] = [9.0, 9.0, 9.0, 9.0]
+    vv[0, 0, 0] = [1.0, 0.0, 0.0, 0.0]
+    vv[0, 1, 0] = [0.0, 1.0, 0.0, 0.0]
+    vv[0, 2, 0] = [0.0, 0.0, 1.0, 0.0]
+    vv[0, 3, 0] = [0.0, 0.0, 0.0, 1.0]
+    out, lse = oracle.decode_positions(q, _bf16_bits(kk), _bf16_bits(vv), [4], [107],
+                                       [[100, 0, 107, 108]], Hq=1, Hkv=1, base=100.0,
+                                       alpha=1.0, g=1, scale=1.0)
+    z = math.exp(6.0) + 1.0 + math.exp(1.0)
+    np.testing.assert_allclose(out[0], [math.exp(6.0) / z, 1.0 / z, math.e / z, 0.0],
+                               rtol=0, atol=1e-12)
+    assert abs(lse[0] - math.log(z)) < 1e-12
+
+
+def test_positions_alpha_inf_is_masked_sdpa():
+    """alpha = inf: ordinary attention under the mask k_pos <= q_pos."""
+    B, Hq, Hkv, D, L = 2, 4, 2, 16, 30
+    q = _rand((B, Hq, D), 61)
+    kc = _rand((B, L, Hkv, D), 62)
+    vc = _rand((B, L, Hkv, D), 63)
+    rng = np.random.default_rng(5)
+    kv_len = [30, 19]
+    k_pos = rng.integers(0, 500, size=(B, L))
+    q_pos = [400, 250]
+    out, lse = oracle.decode_positions(inputs.bits(q), inputs.bits(kc), inputs.bits(vc), kv_len,
+                                       q_pos, k_pos, Hq=Hq, Hkv=Hkv, base=1e4,
+                                       alpha=float("inf"), g=1, scale=0.25)
+    n = 0
+    for b in range(B):
+        keep = torch.tensor(k_pos[b, :kv_len[b]] <= q_pos[b])
+        for h in range(Hq):
+            kk = kc[b, :kv_len[b], h // (Hq // Hkv)].double()
+            vv = vc[b, :kv_len[b], h // (Hq // Hkv)].double()
+            z = 0.25 * (kk @ q[b, h].double())
+            z = torch.where(keep, z, torch.tensor(-math.inf, dtype=torch.float64))
+            want = torch.softmax(z, 0) @ vv
+            np.testing.assert_allclose(out[n], want.numpy(), atol=1e-10)
+            assert abs(lse[n] - float(torch.logsumexp(z, 0))) < 1e-10
+            n += 1
+
+
+def test_positions_contiguous_equal_decode_rows():
+    """k_pos = 0..n-1 with the query at n-1 is plain decode."""
+    B, Hq, Hkv, D, L = 3, 4, 1, 32, 300
+    q = _rand((B, Hq, D), 71)
+    kc = _rand((B, L, Hkv, D), 72)
+    vc = _rand((B, L, Hkv, D), 73)
+    kv_len = [300, 1, 137]
+    k_pos = np.tile(np.arange(L), (B, 1))
+    a = oracle.decode_positions(inputs.bits(q), inputs.bits(kc), inputs.bits(vc), kv_len,
+                                [n - 1 for n in kv_len], k_pos, Hq=Hq, Hkv=Hkv, base=1e4,
+                                alpha=1.0, g=1, scale=0.2)
+    b = oracle.decode_rows(inputs.bits(q), inputs.bits(kc), inputs.bits(vc), kv_len, Hq=Hq,
+                           Hkv=Hkv, base=1e4, alpha=1.0, g=1, scale=0.2)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("g", [1, 8])
+def test_positions_joint_permutation_invariance(g):
+    """Reordering the cache rows together with their positions changes nothing
+    but the summation order; a position-only shift of everything by the same
+    offset changes nothing at all (relative positions are unchanged)."""
+    B, Hq, Hkv, D, L = 1, 2, 1, 32, 400
+    q = _rand((B, Hq, D), 81)
+    kc = _rand((B, L, Hkv, D), 82)
+    vc = _rand((B, L, Hkv, D), 83)
+    rng = np.random.default_rng(9)
+    k_pos = np.sort(rng.choice(5000, size=L, replace=False))[None, :]
+    q_pos = [int(k_pos[0, -1]) + 3]
+    kw = dict(Hq=Hq, Hkv=Hkv, base=1e4, alpha=1.0, g=g, scale=0.3)
+    o1, l1 = oracle.decode_positions(inputs.bits(q), inputs.bits(kc), inputs.bits(vc), [L],
+                                     q_pos, k_pos, **kw)
+    perm = rng.permutation(L)
+    o2, l2 = oracle.decode_positions(inputs.bits(q), inputs.bits(kc)[:, perm],
+                                     inputs.bits(vc)[:, perm], [L], q_pos, k_pos[:, perm], **kw)
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l2, l1, rtol=0, atol=1e-12)
+    o3, l3 = oracle.decode_positions(inputs.bits(q), inputs.bits(kc), inputs.bits(vc), [L],
+                                     [q_pos[0] + 12345], k_pos + 12345, **kw)
+    np.testing.assert_array_equal(o3, o1)
+    np.testing.assert_array_equal(l3, l1)
+    # and the windowed result differs from the window-off one (the pin is not vacuous)
+    o4, _ = oracle.decode_positions(inputs.bits(q), inputs.bits(kc), inputs.bits(vc), [L],
+                                    q_pos, k_pos, **dict(kw, alpha=float("inf")))
+    assert np.abs(o4 - o1).max() > 1e-3
