@@ -50,9 +50,9 @@ FLUSH_BYTES = 512 << 20
 NCU_TRAFFIC = {
     # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.134912 MB read + 23.742208 MB written
     ("qwen2.5-0.5b-32k", "78ae9ff5d51882a2"): 76134912 + 23742208,
-    # profiles/decode_split_kernel_llama3.2-3b-decode-32k.md: 536.926464 MB read + 5.638144 MB
+    # profiles/decode_split_kernel_llama3.2-3b-decode-32k.md: 537.025280 MB read + 6.628608 MB
     # written for B=4, L=32768, scaled by the 16x keys x heads of the B=16, L=131072 call
-    ("llama3.2-3b-decode-128k", "247125b8d0a5fc28"): 16 * (536926464 + 5638144),
+    ("llama3.2-3b-decode-128k", "f05ba464b5fd744d"): 16 * (537025280 + 6628608),
 }
 
 KERNEL_SOURCES = {"prefill": ("prefill_kernel.cuh", "device_util.cuh"),
@@ -406,6 +406,34 @@ def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
     }
     res["gpu_launches"] += 2 * steps
     del slabs
+    # the same call from a paged cache (16-row pages in shuffled pool order, the
+    # page size serving engines default to), scattered once outside the timed region
+    page = 16
+    table, num_pages = inputs.page_layout(kv_len, page, seed=rank + 100)
+    kp = inputs.scatter_to_pages(kc, kv_len, table, page, num_pages)
+    vp = inputs.scatter_to_pages(vc, kv_len, table, page, num_pages)
+    table = table.to(dev)
+    ws_pg = torch.empty(wp.decode_workspace_size(win, w.B, w.Hq, w.Hkv, table.shape[1] * page),
+                        dtype=torch.uint8, device=dev)
+
+    def step_pg():
+        wp.decode_paged(q, kp, vp, table, kv_len, win, scale=w.scale, out=out, lse=lse,
+                        workspace=ws_pg)
+
+    pg_ms, pg_per, _ = time_steps(step_pg, args.warmup, steps, flush, world)
+    if wp.device_status() != wp.OK:
+        raise RuntimeError("paged decode kernel status: not ok")
+    pg_achieved = alg / (statistics.mean(pg_per) * 1e-3) / 1e9
+    res["paged"] = {
+        "value": round(weak_scaling_value(alg, world, pg_ms / steps) / 1e9, 1), "unit": "GB/s",
+        "ms_per_step": round(pg_ms / steps, 4),
+        "roofline": {"bound": "hbm", "achieved": round(pg_achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(pg_achieved / peaks["hbm_gbs"], 4),
+                     "traffic": None, "peak_source": f"{peaks['source']} HBM copy"},
+        "layout": f"K, V page pools [{num_pages}, {page}, Hkv, D], shuffled block table",
+    }
+    res["gpu_launches"] += 2 * steps
+    del kp, vp, ws_pg
     if primary:
         res["clocks"] = clk
         qh = q.cpu().pin_memory()

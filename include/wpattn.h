@@ -53,7 +53,9 @@ enum {
     WPATTN_EUNSUPPORTED = 2,  /* valid but not supported here (head_dim, device arch, size limit) */
     WPATTN_ECUDA = 3,         /* a CUDA runtime call or a kernel launch failed */
     WPATTN_ETIMEOUT = 4,      /* a kernel's bounded wait ran out (see wpattn_device_status) */
-    WPATTN_EWORKSPACE = 5     /* workspace null or smaller than wpattn_decode_workspace_size */
+    WPATTN_EWORKSPACE = 5,    /* workspace null or smaller than wpattn_decode_workspace_size */
+    WPATTN_EINDEX = 6         /* a device-side index was out of range (block-table entry outside
+                                 the pool, negative key position); see wpattn_device_status */
 };
 
 /*
@@ -207,9 +209,71 @@ WPATTN_API int wpattn_kcache_to_pairmajor(const void *k_cache, void *k_slabs, in
                   int32_t B, int32_t Hkv, int32_t head_dim, void *cuda_stream);
 
 /*
+ * Decode with explicit positions: the keys of a sequence need not sit at
+ * positions 0..kv_len-1 with the query right after them (a cache that evicted
+ * or reordered tokens, a query at a position of its own).  ATFlash Abstract:
+ * whether a pair is kept depends only on the relative position, so the
+ * window is applied to d = q_pos[b] - k_pos[b, j].
+ *   q_pos_host: host int32 [B], 0 <= q_pos < 2^31 - 1 (else WPATTN_EINVAL).
+ *   k_pos:      device int32, k_pos[b * k_pos_stride + j] is the position of
+ *               cache row j of sequence b (j < kv_len[b]); 4-byte aligned;
+ *               k_pos_stride >= max kv_len (else WPATTN_EINVAL).  Positions
+ *               need not be sorted or distinct.  A key whose position is
+ *               after q_pos[b] is left out (causality).  A negative position
+ *               is an error found on the device: the key is left out and
+ *               WPATTN_EINDEX is recorded for wpattn_device_status.
+ * Every other argument, the result and the workspace are those of
+ * wpattn_decode.  A sequence with no key at or before its query gets out = 0
+ * and lse = -inf.  With k_pos[b, j] = j and q_pos[b] = kv_len[b] - 1 the
+ * call gives wpattn_decode's output bit for bit.
+ */
+WPATTN_API int wpattn_decode_positions(const wpattn_window *w,
+                  const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *kv_len_host, int64_t Lmax,
+                  const int32_t *q_pos_host, const int32_t *k_pos, int64_t k_pos_stride,
+                  int32_t B, int32_t Hq, int32_t Hkv, float softmax_scale,
+                  void *out, float *lse,
+                  void *workspace, size_t workspace_bytes,
+                  void *cuda_stream);
+
+/*
+ * Decode from a paged KV cache (the page-table layout serving engines use;
+ * not a layout of the pages, whose decode reads a contiguous cache).
+ *   k_pages, v_pages: bf16 device pools [num_pages, page_size, Hkv, D],
+ *               16-byte aligned.
+ *   page_size:  8, 16 or a multiple of 32 (else WPATTN_EUNSUPPORTED).
+ *   block_table: device int32 [B, max_pages_per_seq], 4-byte aligned: cache
+ *               row j of sequence b is row j % page_size of page
+ *               block_table[b * max_pages_per_seq + j / page_size].  Only the
+ *               entries that cover rows j < kv_len[b] are read.  An entry
+ *               outside [0, num_pages) is an error found on the device: page
+ *               0 is read in its place and WPATTN_EINDEX is recorded.
+ *   kv_len_host: host int32 [B], 1 <= kv_len <= max_pages_per_seq * page_size.
+ *   q_pos_host, k_pos, k_pos_stride: both null (keys at 0..kv_len-1, query at
+ *               kv_len-1) or both given, as for wpattn_decode_positions
+ *               (k_pos is indexed by the logical row j, not by page).
+ * The workspace is sized by wpattn_decode_workspace_size with max_kv_len =
+ * max_pages_per_seq * page_size.  Result and errors as for wpattn_decode; the
+ * output equals, bit for bit, that of wpattn_decode (or
+ * wpattn_decode_positions) on the [B, max_pages_per_seq * page_size, Hkv, D]
+ * cache gathered through the block table.
+ */
+WPATTN_API int wpattn_decode_paged(const wpattn_window *w,
+                  const void *q, const void *k_pages, const void *v_pages,
+                  int32_t num_pages, int32_t page_size,
+                  const int32_t *block_table, int32_t max_pages_per_seq,
+                  const int32_t *kv_len_host, const int32_t *q_pos_host,
+                  const int32_t *k_pos, int64_t k_pos_stride,
+                  int32_t B, int32_t Hq, int32_t Hkv, float softmax_scale,
+                  void *out, float *lse,
+                  void *workspace, size_t workspace_bytes,
+                  void *cuda_stream);
+
+/*
  * Synchronises `cuda_stream`, then reads and clears the current device's
  * kernel status word.  Returns WPATTN_OK, WPATTN_ETIMEOUT (a kernel gave up a
- * bounded wait; its outputs are undefined) or WPATTN_ECUDA.
+ * bounded wait; its outputs are undefined), WPATTN_EINDEX (a kernel met an
+ * out-of-range device-side index; its outputs are undefined) or WPATTN_ECUDA.
  */
 WPATTN_API int wpattn_device_status(void *cuda_stream);
 

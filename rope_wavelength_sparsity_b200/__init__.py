@@ -9,6 +9,7 @@ exception is raised.
 
 Entry points (same names as the C ABI, without the ``wpattn_`` prefix):
 ``prefill``, ``decode``, ``decode_pairmajor``, ``kcache_to_pairmajor``,
+``decode_positions``, ``decode_paged``,
 ``decode_workspace_size``, ``decode_noalloc``, ``pruned_fraction``,
 ``thresholds``, ``device_status``.
 """
@@ -22,7 +23,7 @@ from dataclasses import dataclass
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libwpattn.so")
 
-OK, EINVAL, EUNSUPPORTED, ECUDA, ETIMEOUT, EWORKSPACE = range(6)
+OK, EINVAL, EUNSUPPORTED, ECUDA, ETIMEOUT, EWORKSPACE, EINDEX = range(7)
 
 
 class WpattnError(RuntimeError):
@@ -73,6 +74,11 @@ def lib() -> ctypes.CDLL:
                                     i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
         L.wpattn_decode_pairmajor.argtypes = L.wpattn_decode.argtypes
         L.wpattn_kcache_to_pairmajor.argtypes = [vp, vp, i64, i32, i32, i32, vp]
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        L.wpattn_decode_positions.argtypes = [wp, vp, vp, vp, i32p, i64, i32p, vp, i64, i32, i32,
+                                              i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
+        L.wpattn_decode_paged.argtypes = [wp, vp, vp, vp, i32, i32, vp, i32, i32p, i32p, vp, i64,
+                                          i32, i32, i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
         L.wpattn_device_status.argtypes = [vp]
         L.wpattn_strerror.restype = ctypes.c_char_p
         L.wpattn_strerror.argtypes = [ctypes.c_int]
@@ -222,6 +228,81 @@ def decode_pairmajor(q, k_slabs, v_cache, kv_len, w: Window, *, scale: float | N
                                        ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
                                        _stream_ptr(stream))
     _check(rc, "wpattn_decode_pairmajor")
+    return out, lse
+
+
+def _decode_outputs(q, w, B, Hq, Hkv, cap, out, lse, want_lse, workspace):
+    import torch
+    if workspace is None:
+        n = decode_workspace_size(w, B, Hq, Hkv, cap)
+        if n == 0:
+            raise WpattnError(EINVAL, "wpattn_decode_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    return out, lse, workspace
+
+
+def _int32_dev(t, name):
+    """Device pointer of a 2-D int32 CUDA tensor whose rows are contiguous."""
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.int32:
+        raise TypeError(f"{name} must be an int32 CUDA tensor")
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise TypeError(f"{name} must be 2-D with contiguous rows")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def decode_positions(q, k_cache, v_cache, kv_len, q_pos, k_pos, w: Window, *,
+                     scale: float | None = None, out=None, lse=None, want_lse: bool = True,
+                     workspace=None, stream=None):
+    """Decode with explicit positions: the query of sequence b at q_pos[b] (host
+    ints), cache row j at k_pos[b, j] (int32 CUDA tensor [B, >= max kv_len]).
+    Caches, kv_len and results as for ``decode``."""
+    B, Hq, D = q.shape
+    L, Hkv = k_cache.shape[1], k_cache.shape[2]
+    kvl = (ctypes.c_int32 * B)(*[int(x) for x in kv_len])
+    qp = (ctypes.c_int32 * B)(*[int(x) for x in q_pos])
+    out, lse, workspace = _decode_outputs(q, w, B, Hq, Hkv, L, out, lse, want_lse, workspace)
+    rc = lib().wpattn_decode_positions(ctypes.byref(w._c()), _dev_tensor(q, "q"),
+                                       _dev_tensor(k_cache, "k_cache"), _dev_tensor(v_cache, "v_cache"),
+                                       kvl, L, qp, _int32_dev(k_pos, "k_pos"), k_pos.stride(0), B,
+                                       Hq, Hkv, float(scale) if scale else 0.0, _dev_tensor(out, "out"),
+                                       ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+                                       ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                       _stream_ptr(stream))
+    _check(rc, "wpattn_decode_positions")
+    return out, lse
+
+
+def decode_paged(q, k_pages, v_pages, block_table, kv_len, w: Window, *, q_pos=None, k_pos=None,
+                 scale: float | None = None, out=None, lse=None, want_lse: bool = True,
+                 workspace=None, stream=None):
+    """Decode from page pools k_pages, v_pages [num_pages, page_size, Hkv, D] (bf16
+    CUDA) through block_table (int32 CUDA [B, max_pages_per_seq]); optional
+    explicit positions as for ``decode_positions``.  Results as for ``decode``."""
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    if not block_table.is_contiguous():
+        raise TypeError("block_table must be contiguous")
+    max_pages = block_table.shape[1]
+    kvl = (ctypes.c_int32 * B)(*[int(x) for x in kv_len])
+    qp = (ctypes.c_int32 * B)(*[int(x) for x in q_pos]) if q_pos is not None else None
+    out, lse, workspace = _decode_outputs(q, w, B, Hq, Hkv, max_pages * page_size, out, lse,
+                                          want_lse, workspace)
+    rc = lib().wpattn_decode_paged(ctypes.byref(w._c()), _dev_tensor(q, "q"),
+                                   _dev_tensor(k_pages, "k_pages"), _dev_tensor(v_pages, "v_pages"),
+                                   num_pages, page_size, _int32_dev(block_table, "block_table"),
+                                   max_pages, kvl, qp,
+                                   _int32_dev(k_pos, "k_pos") if k_pos is not None else None,
+                                   k_pos.stride(0) if k_pos is not None else 0, B, Hq, Hkv,
+                                   float(scale) if scale else 0.0, _dev_tensor(out, "out"),
+                                   ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+                                   ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                   _stream_ptr(stream))
+    _check(rc, "wpattn_decode_paged")
     return out, lse
 
 

@@ -2,6 +2,7 @@
 // include/wpattn.h).  Host side: argument checks, the planner, TMA tensor
 // maps and kernel launches.  Every step of the computation runs in the
 // kernels of decode_kernels.cuh and prefill_kernel.cuh.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -176,12 +177,21 @@ int launch_decode(const DecodeParams& prm, int gc, bool pm, cudaStream_t st) {
     const cuuint64_t strides[3] = {32, static_cast<cuuint64_t>(prm.Lmax) * 32,
                                    planes * static_cast<cuuint64_t>(prm.Lmax) * 32};
     if ((rc = encode_bf16_4d_strided(&tk, prm.k, dims, strides, 16, KB)) != WPATTN_OK) return rc;
+  } else if (prm.block_table) {
+    // page pools [num_pages, page_size, Hkv, D]: dims D, page_size, Hkv, num_pages;
+    // boxes of 64 dims x min(page_size, 32) rows (a copy never crosses a page)
+    const uint32_t R = prm.page_size < static_cast<int>(KB) ? prm.page_size : KB;
+    if ((rc = encode_bf16_4d(&tk, prm.k, D, prm.page_size, prm.Hkv, prm.num_pages, 64, R, true)) != WPATTN_OK)
+      return rc;
+    if ((rc = encode_bf16_4d(&tv, prm.v, D, prm.page_size, prm.Hkv, prm.num_pages, 64, R, true)) != WPATTN_OK)
+      return rc;
   } else {
     // caches are [B, Lmax, Hkv, D]: dims (fastest first) D, Lmax, Hkv, B; 64-dim x 32-key boxes
     if ((rc = encode_bf16_4d(&tk, prm.k, D, prm.Lmax, prm.Hkv, prm.B, 64, KB, true)) != WPATTN_OK)
       return rc;
   }
-  if ((rc = encode_bf16_4d(&tv, prm.v, D, prm.Lmax, prm.Hkv, prm.B, 64, KB, true)) != WPATTN_OK)
+  if (!prm.block_table &&
+      (rc = encode_bf16_4d(&tv, prm.v, D, prm.Lmax, prm.Hkv, prm.B, 64, KB, true)) != WPATTN_OK)
     return rc;
   rc = pm ? launch_decode_gc<D, true>(tk, tv, prm, gc, st) : launch_decode_gc<D, false>(tk, tv, prm, gc, st);
   if (rc != WPATTN_OK) return rc;
@@ -218,6 +228,7 @@ const char* wpattn_strerror(int code) {
     case WPATTN_ECUDA: return "CUDA runtime or launch error";
     case WPATTN_ETIMEOUT: return "a kernel gave up a bounded wait";
     case WPATTN_EWORKSPACE: return "workspace missing or too small";
+    case WPATTN_EINDEX: return "a device-side index (page or position) was out of range";
     default: return "unknown status code";
   }
 }
@@ -314,12 +325,23 @@ size_t wpattn_decode_workspace_size(const wpattn_window* w, int32_t B, int32_t H
 }  // extern "C"
 
 namespace {
-// wpattn_decode and wpattn_decode_pairmajor: the same call with the K cache in
-// the [B, Lmax, Hkv, D] layout (pm = false) or as pair-major slabs (pm = true)
+// How the decode call finds its keys: the [B, Lmax, Hkv, D] cache (the
+// default), pair-major K slabs, or page pools with a block table; and where
+// they sit: at positions 0..kv_len-1 with the query last (the default), or at
+// explicit positions.
+struct DecodeLayout {
+  bool pm = false;
+  const int32_t* block_table = nullptr;   // device [B, max_pages]
+  int max_pages = 0, page_size = 0, num_pages = 0;
+  const int32_t* q_pos_host = nullptr;    // host [B]
+  const int32_t* k_pos = nullptr;         // device [B, k_pos_stride]
+  int64_t k_pos_stride = 0;
+};
+
 int decode_impl(const wpattn_window* w, const void* q, const void* k_cache, const void* v_cache,
                 const int32_t* kv_len_host, int64_t Lmax, int32_t B, int32_t Hq, int32_t Hkv,
                 float softmax_scale, void* out, float* lse, void* workspace,
-                size_t workspace_bytes, void* cuda_stream, bool pm) {
+                size_t workspace_bytes, void* cuda_stream, const DecodeLayout& lay) {
   WindowPlan plan;
   int rc = make_window_plan(w, &plan);
   if (rc != WPATTN_OK) return rc;
@@ -333,6 +355,15 @@ int decode_impl(const wpattn_window* w, const void* q, const void* k_cache, cons
   if (G > 16 || B > kDecodeMaxB || Lmax >= (int64_t(1) << 31)) return WPATTN_EUNSUPPORTED;
   for (int b = 0; b < B; ++b)
     if (kv_len_host[b] < 1 || kv_len_host[b] > Lmax) return WPATTN_EINVAL;
+  if (lay.q_pos_host)
+    for (int b = 0; b < B; ++b)
+      if (lay.q_pos_host[b] < 0 || lay.q_pos_host[b] == INT32_MAX) return WPATTN_EINVAL;
+  if (lay.k_pos) {
+    int32_t longest = 0;
+    for (int b = 0; b < B; ++b) longest = std::max(longest, kv_len_host[b]);
+    if (lay.k_pos_stride < longest || (reinterpret_cast<uintptr_t>(lay.k_pos) & 3u) != 0)
+      return WPATTN_EINVAL;
+  }
   DeviceInfo* dev = nullptr;
   if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
   const int S = decode_splits(B, Hkv, Lmax, dev->num_sms);
@@ -355,10 +386,19 @@ int decode_impl(const wpattn_window* w, const void* q, const void* k_cache, cons
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(plan.D));
   prm.scale_log2 = scale * 1.44269504088896340736f;
   for (int p = 0; p < 64; ++p) prm.T[p] = plan.T[p] > INT32_MAX ? INT32_MAX : static_cast<int>(plan.T[p]);
-  for (int b = 0; b < B; ++b) prm.kv_len[b] = kv_len_host[b];
+  for (int b = 0; b < B; ++b) {
+    prm.kv_len[b] = kv_len_host[b];
+    prm.q_pos[b] = lay.q_pos_host ? lay.q_pos_host[b] : kv_len_host[b] - 1;
+  }
+  prm.block_table = lay.block_table;
+  prm.max_pages = lay.max_pages;
+  prm.page_size = lay.page_size;
+  prm.num_pages = lay.num_pages;
+  prm.k_pos = lay.k_pos;
+  prm.k_pos_stride = lay.k_pos_stride;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  if (plan.D == 64) return launch_decode<64>(prm, gc, pm, st);
-  return launch_decode<128>(prm, gc, pm, st);
+  if (plan.D == 64) return launch_decode<64>(prm, gc, lay.pm, st);
+  return launch_decode<128>(prm, gc, lay.pm, st);
 }
 }  // namespace
 
@@ -369,7 +409,7 @@ int wpattn_decode(const wpattn_window* w, const void* q, const void* k_cache, co
                   float softmax_scale, void* out, float* lse, void* workspace,
                   size_t workspace_bytes, void* cuda_stream) {
   return decode_impl(w, q, k_cache, v_cache, kv_len_host, Lmax, B, Hq, Hkv, softmax_scale, out, lse,
-                     workspace, workspace_bytes, cuda_stream, false);
+                     workspace, workspace_bytes, cuda_stream, DecodeLayout{});
 }
 
 int wpattn_decode_pairmajor(const wpattn_window* w, const void* q, const void* k_slabs,
@@ -377,8 +417,52 @@ int wpattn_decode_pairmajor(const wpattn_window* w, const void* q, const void* k
                             int32_t B, int32_t Hq, int32_t Hkv, float softmax_scale, void* out,
                             float* lse, void* workspace, size_t workspace_bytes,
                             void* cuda_stream) {
+  DecodeLayout lay;
+  lay.pm = true;
   return decode_impl(w, q, k_slabs, v_cache, kv_len_host, Lmax, B, Hq, Hkv, softmax_scale, out, lse,
-                     workspace, workspace_bytes, cuda_stream, true);
+                     workspace, workspace_bytes, cuda_stream, lay);
+}
+
+int wpattn_decode_positions(const wpattn_window* w, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* kv_len_host, int64_t Lmax,
+                            const int32_t* q_pos_host, const int32_t* k_pos, int64_t k_pos_stride,
+                            int32_t B, int32_t Hq, int32_t Hkv, float softmax_scale, void* out,
+                            float* lse, void* workspace, size_t workspace_bytes,
+                            void* cuda_stream) {
+  if (!q_pos_host || !k_pos) return WPATTN_EINVAL;
+  DecodeLayout lay;
+  lay.q_pos_host = q_pos_host;
+  lay.k_pos = k_pos;
+  lay.k_pos_stride = k_pos_stride;
+  return decode_impl(w, q, k_cache, v_cache, kv_len_host, Lmax, B, Hq, Hkv, softmax_scale, out, lse,
+                     workspace, workspace_bytes, cuda_stream, lay);
+}
+
+int wpattn_decode_paged(const wpattn_window* w, const void* q, const void* k_pages,
+                        const void* v_pages, int32_t num_pages, int32_t page_size,
+                        const int32_t* block_table, int32_t max_pages_per_seq,
+                        const int32_t* kv_len_host, const int32_t* q_pos_host,
+                        const int32_t* k_pos, int64_t k_pos_stride, int32_t B, int32_t Hq,
+                        int32_t Hkv, float softmax_scale, void* out, float* lse, void* workspace,
+                        size_t workspace_bytes, void* cuda_stream) {
+  if (!block_table || num_pages <= 0 || max_pages_per_seq <= 0) return WPATTN_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) != 0) return WPATTN_EINVAL;
+  // a 32-key block is one page, a part of one page, or a whole number of pages
+  if (!(page_size == 8 || page_size == 16 || (page_size > 0 && page_size % 32 == 0)))
+    return WPATTN_EUNSUPPORTED;
+  if ((q_pos_host == nullptr) != (k_pos == nullptr)) return WPATTN_EINVAL;
+  const int64_t cap = static_cast<int64_t>(max_pages_per_seq) * page_size;
+  if (static_cast<int64_t>(num_pages) * page_size >= (int64_t(1) << 40)) return WPATTN_EUNSUPPORTED;
+  DecodeLayout lay;
+  lay.block_table = block_table;
+  lay.max_pages = max_pages_per_seq;
+  lay.page_size = page_size;
+  lay.num_pages = num_pages;
+  lay.q_pos_host = q_pos_host;
+  lay.k_pos = k_pos;
+  lay.k_pos_stride = k_pos_stride;
+  return decode_impl(w, q, k_pages, v_pages, kv_len_host, cap, B, Hq, Hkv, softmax_scale, out, lse,
+                     workspace, workspace_bytes, cuda_stream, lay);
 }
 
 int wpattn_kcache_to_pairmajor(const void* k_cache, void* k_slabs, int64_t Lmax, int32_t B,

@@ -35,7 +35,17 @@ struct DecodeParams {
   int hchunks;         // ceil(G / GC)
   float scale_log2;    // softmax scale * log2(e)
   int T[64];           // per-pair thresholds, clamped to int32
+  // paged cache (block_table != null): k and v are page pools
+  // [num_pages, page_size, Hkv, D]; key j of sequence b is row j % page_size of
+  // page block_table[b * max_pages + j / page_size]
+  const int32_t* block_table;
+  int max_pages, page_size, num_pages;
+  // explicit key positions (k_pos != null): key j of sequence b sits at
+  // k_pos[b * k_pos_stride + j]; otherwise at position j
+  const int32_t* k_pos;
+  int64_t k_pos_stride;
   int kv_len[kDecodeMaxB];
+  int q_pos[kDecodeMaxB];  // position of each sequence's query
 };
 
 __device__ __forceinline__ uint4 ldg_stream(const void* ptr) {
@@ -140,7 +150,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   const int j_begin = split * chunk;
   const int j_end = min(Lb, j_begin + chunk);
   const int nblk = j_end > j_begin ? (j_end - j_begin + KB - 1) / KB : 0;
-  const int qpos = Lb - 1;
+  const int qpos = p.q_pos[b];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // first group of 8 pairs kept for some key of the block starting at j0:
   // groups whose largest threshold is below the block's smallest distance
@@ -168,20 +178,81 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 
   if (warp == W) {
     // ------------------------------------------------------------ producer
+    // The whole warp walks the blocks (lane 0 issues the copies) so that, for
+    // a paged cache, the lanes can fetch 32 page numbers at a time.
     if (lane == 0) {
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      for (int i = 0; i < nblk; ++i) {
-        const int s = i % NS;
-        if (i >= NS && !mbar_wait(empty(s), ((i / NS) & 1) ^ 1)) break;
-        const int j0 = j_begin + i * KB;
+    }
+    // paged: rows per copy (one page, at most one block), copies per block
+    const int R = p.block_table ? min(p.page_size, KB) : KB;
+    const int U = KB / R;
+    // page of copy unit u (R rows from j_begin + u * R): lane l holds unit
+    // 32 k + l of the current batch k and, loaded one batch ahead so that its
+    // latency is hidden, of the next
+    auto fetch_page = [&](int unit) -> int {
+      const long long jl = j_begin + static_cast<long long>(unit) * R;
+      if (!p.block_table || jl >= j_end) return 0;
+      const int pg = p.block_table[(size_t)b * p.max_pages + static_cast<int>(jl / p.page_size)];
+      if (pg < 0 || pg >= p.num_pages) {
+        record_status(6 /* WPATTN_EINDEX */);
+        return 0;                         // read a real page; the output is flagged
+      }
+      return pg;
+    };
+    int my_page = 0, next_page = 0;
+    const bool paged = !PM && p.block_table != nullptr;
+    if (paged) {
+      my_page = fetch_page(lane);
+      next_page = fetch_page(32 + lane);
+    }
+    // addressing of the next block, worked out while its ring stage drains
+    int pg[4], row0 = 0, nsub = 0;
+    auto plan_block = [&](int i) {
+      const int unit0 = i * U;            // copy units of this CTA's range, R rows each
+      if (unit0 > 0 && (unit0 & 31) == 0) {
+        my_page = next_page;
+        next_page = fetch_page(unit0 + 32 + lane);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) pg[u] = __shfl_sync(FULL, my_page, (unit0 + u) & 31);
+      const int j0 = j_begin + i * KB;
+      row0 = R < KB ? 0 : j0 % p.page_size;  // R < KB: one page per unit, from its row 0
+      nsub = (min(j0 + KB, j_end) - j0 + R - 1) / R;
+    };
+    if (paged && nblk > 0) plan_block(0);
+    // pair-major: first slab of the next block, found while its stage drains
+    int g0_next = (PM && nblk > 0) ? first_kept_group(j_begin) : 0;
+    for (int i = 0; i < nblk; ++i) {
+      const int s = i % NS;
+      if (i >= NS && !__all_sync(FULL, mbar_wait(empty(s), ((i / NS) & 1) ^ 1))) break;
+      const int j0 = j_begin + i * KB;
+      if (paged) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(full(s), nsub * R * D * 2 * 2);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (u >= nsub) break;
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+              const uint32_t off = s * L::TILE + c * L::PANEL + u * R * 128;
+              tma_load_4d(sbase + L::OFF_K + off, &tmK, full(s), 64 * c, row0, kvh, pg[u]);
+              tma_load_4d(sbase + L::OFF_V + off, &tmV, full(s), 64 * c, row0, kvh, pg[u]);
+            }
+          }
+        }
+        if (i + 1 < nblk) plan_block(i + 1);
+        continue;
+      }
+      if (lane == 0) {
         if (PM) {
-          const int g0 = first_kept_group(j0);
+          const int g0 = g0_next;
           mbar_arrive_expect_tx(full(s), (NG - g0) * KB * 32 + L::TILE);
           for (int g = g0; g < NG; ++g)
             tma_load_4d(sbase + L::OFF_K + s * L::TILE + g * KB * 32, &tmK, full(s), 0, j0, kvh * NG + g, b);
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sbase + L::OFF_V + s * L::TILE + c * L::PANEL, &tmV, full(s), 64 * c, j0, kvh, b);
+          if (i + 1 < nblk) g0_next = first_kept_group(j0 + KB);
         } else {
           mbar_arrive_expect_tx(full(s), 2 * L::TILE);
           for (int c = 0; c < D / 64; ++c) {
@@ -209,14 +280,29 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 
   for (int i = warp; i < nblk; i += W) {
     const int s = i % NS;
+    const int j0 = j_begin + i * KB;
+    const int j = j0 + lane;              // this lane's key
+    // explicit positions: fetched before the wait so the load overlaps it
+    int kpos = j;
+    if (p.k_pos && j < j_end) kpos = p.k_pos[(size_t)b * p.k_pos_stride + j];
+    // contiguous positions: the block's first kept group is known before its data
+    int g0 = p.k_pos ? 0 : first_kept_group(j0);
     if (!__all_sync(FULL, mbar_wait(full(s), (i / NS) & 1))) break;
     const uint8_t* kt = smem + L::OFF_K + s * L::TILE;
     const uint8_t* vt = smem + L::OFF_V + s * L::TILE;
-    const int j0 = j_begin + i * KB;
-    const int j = j0 + lane;              // this lane's key
-    const bool valid = j < j_end;
-    const int dist = qpos - j;
-    const int g0 = first_kept_group(j0);
+    bool valid = j < j_end;
+    int dist = qpos - kpos;
+    if (p.k_pos) {
+      if (valid && kpos < 0) {
+        record_status(6 /* WPATTN_EINDEX */);
+        kpos = qpos + 1;                  // treated as a future key
+        dist = -1;
+      }
+      valid = valid && kpos <= qpos;      // keys after the query are causally excluded
+      // smallest distance over the block's attended keys (positions need not be sorted)
+      const int dmin = __reduce_min_sync(FULL, valid ? dist : 0x7fffffff);
+      while (g0 < NG && sT[8 * g0 + 7] < dmin) ++g0;
+    }
 
     // ---- scores: one key per lane, groups g0 .. NG-1
     float sc[GC];

@@ -165,3 +165,87 @@ def decode_inputs(w: Workload, seed: int = 0, device="cpu"):
 def bits(t: torch.Tensor):
     """bf16 tensor -> numpy uint16 bit patterns (CPU), the form the oracle reads."""
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view("uint16")
+
+
+def page_layout(kv_len, page_size: int, seed: int, spare_pages: int = 3):
+    """(block_table int32 [B, max_pages], num_pages) of a shuffled page pool.
+
+    Sequence b gets ceil(kv_len[b] / page_size) distinct pages drawn in random
+    order from a pool with ``spare_pages`` pages nobody uses; entries past a
+    sequence's last page are -1 (a reader that touched them would be caught).
+    """
+    kv = [int(x) for x in kv_len]
+    need = [(n + page_size - 1) // page_size for n in kv]
+    max_pages = max(need)
+    num_pages = sum(need) + spare_pages
+    perm = torch.randperm(num_pages, generator=_gen(seed, "cpu")).to(torch.int32)
+    table = torch.full((len(kv), max_pages), -1, dtype=torch.int32)
+    at = 0
+    for b, n in enumerate(need):
+        table[b, :n] = perm[at:at + n]
+        at += n
+    return table, num_pages
+
+
+def _page_rows(n: int, table_row: torch.Tensor, page_size: int, device) -> torch.Tensor:
+    """Pool row (page * page_size + row in page) of cache rows 0..n-1 of one sequence."""
+    j = torch.arange(n, device=device)
+    return table_row.to(device).long()[j // page_size] * page_size + j % page_size
+
+
+def scatter_to_pages(cache: torch.Tensor, kv_len, block_table: torch.Tensor, page_size: int,
+                     num_pages: int) -> torch.Tensor:
+    """[B, L, Hkv, D] cache -> pool [num_pages, page_size, Hkv, D] on the cache's
+    device: rows j < kv_len[b] go to their page; every other row of the pool
+    (unused pages, the tail of a sequence's last page) is NaN, so a kernel that
+    read one would show it."""
+    B, L, Hkv, D = cache.shape
+    pool = torch.full((num_pages * page_size, Hkv, D), float("nan"), dtype=cache.dtype,
+                      device=cache.device)
+    for b in range(B):
+        n = int(kv_len[b])
+        pool[_page_rows(n, block_table[b], page_size, cache.device)] = cache[b, :n]
+    return pool.view(num_pages, page_size, Hkv, D)
+
+
+def gather_pages(pool: torch.Tensor, kv_len, block_table: torch.Tensor) -> torch.Tensor:
+    """The [B, max_pages * page_size, Hkv, D] cache a block table describes, on the
+    pool's device (rows past a sequence's last page are NaN)."""
+    num_pages, page_size, Hkv, D = pool.shape
+    B, max_pages = block_table.shape
+    out = torch.full((B, max_pages * page_size, Hkv, D), float("nan"), dtype=pool.dtype,
+                     device=pool.device)
+    flat = pool.reshape(num_pages * page_size, Hkv, D)
+    for b in range(B):
+        n = (int(kv_len[b]) + page_size - 1) // page_size * page_size
+        out[b, :n] = flat[_page_rows(n, block_table[b], page_size, pool.device)]
+    return out
+
+
+def key_positions(kv_len, seed: int, mode: str = "evicted", span: float = 4.0):
+    """(q_pos [B] ints, k_pos int32 [B, max kv_len]) for caches that dropped tokens.
+
+    ``evicted``: each sequence keeps kv_len[b] of the first round(span * kv_len[b])
+    positions (a random subset, sorted); the query comes right after the last
+    kept key, so the most recent key is always kept.  ``shuffled``: the same
+    positions in random cache order.  ``future``: as ``shuffled`` but about a
+    tenth of the keys sit after the query (they must be left out).
+    Unused columns are -1 (never read).
+    """
+    g = _gen(seed, "cpu")
+    kv = [int(x) for x in kv_len]
+    k_pos = torch.full((len(kv), max(kv)), -1, dtype=torch.int32)
+    q_pos = []
+    for b, n in enumerate(kv):
+        total = max(n, int(round(span * n)))
+        keep = torch.randperm(total, generator=g)[:n].sort().values.to(torch.int32)
+        qp = int(keep[-1]) + 1
+        if mode in ("shuffled", "future"):
+            keep = keep[torch.randperm(n, generator=g)]
+        if mode == "future":
+            late = torch.rand(n, generator=g) < 0.1
+            keep = torch.where(late, qp + 1 + torch.randint(0, 1000, (n,), generator=g,
+                                                            dtype=torch.int32), keep)
+        k_pos[b, :n] = keep
+        q_pos.append(qp)
+    return q_pos, k_pos
