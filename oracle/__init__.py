@@ -58,6 +58,11 @@ def _load():
             lib.oracle_scores.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
                                           ctypes.c_int64, ctypes.c_double, ctypes.c_double,
                                           ctypes.c_int, vp]
+            lib.oracle_attention_rows_masked.argtypes = [
+                vp, vp, vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                ctypes.c_double, ctypes.c_int, ctypes.c_double, vp, ctypes.c_int64,
+                ctypes.c_int64, ctypes.c_int64, vp, vp, vp]
             lib.oracle_decode_positions.argtypes = [
                 vp, vp, vp, vp, vp, vp, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double,
@@ -120,6 +125,35 @@ def attention_rows(q, k, v, *, Hq, Hkv, q_pos0=0, k_pos0=0, base, alpha, g, scal
         rows.ctypes.data, out.ctypes.data, lse.ctypes.data)
     if rc != 0:
         raise ValueError(f"oracle_attention_rows failed ({rc})")
+    return out, lse
+
+
+def attention_rows_masked(q, k, v, block_mask, *, Hq, Hkv, q_pos0=0, k_pos0=0, base, alpha, g,
+                          scale, rows, block_q=128, block_k=128):
+    """As ``attention_rows``, with key j of row t attended only where
+    block_mask[b, h, t // block_q, j // block_k] is nonzero.
+
+    block_mask: [B, Hq, ceil(Nq / block_q), ceil(Nk / block_k)], any integer or
+    bool dtype.  ATFlash Abstract: the window composes with token selection.
+    """
+    lib = _load()
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    B, Nq, _, D = q.shape
+    Nk = k.shape[1]
+    nqb, nkb = -(-Nq // block_q), -(-Nk // block_k)
+    m = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
+    if m.shape != (B, Hq, nqb, nkb):
+        raise ValueError(f"block_mask shape {m.shape}, want {(B, Hq, nqb, nkb)}")
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    n = rows.shape[0]
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros(n, dtype=np.float64)
+    rc = lib.oracle_attention_rows_masked(
+        q.ctypes.data, k.ctypes.data, v.ctypes.data, B, Nq, Nk, Hq, Hkv, D, q_pos0, k_pos0,
+        base, alpha, g, scale, m.ctypes.data, block_q, block_k, n, rows.ctypes.data,
+        out.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_attention_rows_masked failed ({rc})")
     return out, lse
 
 

@@ -383,3 +383,83 @@ def test_positions_joint_permutation_invariance(g):
     o4, _ = oracle.decode_positions(inputs.bits(q), inputs.bits(kc), inputs.bits(vc), [L],
                                     q_pos, k_pos, **dict(kw, alpha=float("inf")))
     assert np.abs(o4 - o1).max() > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# block mask stacked on the window (ATFlash Abstract: the window composes with
+# token-level selection)
+# ---------------------------------------------------------------------------
+
+def test_block_mask_hand_case():
+    """The 2-pair case of test_two_pair_softmax_by_hand (query at 7, T = (6, 62)) with
+    4-key blocks.  Mask (0, 1): keys 4..7 remain, scores (0, 0, 0, 5.25).  Mask (1, 0):
+    keys 0..3 remain, scores (6, 0, 0, 0) (the row's own key is masked out)."""
+    q = _bf16_bits(np.array([1.0, 2.0, 3.0, 4.0]).reshape(1, 1, 1, 4))
+    kk = np.zeros((1, 8, 1, 4))
+    vv = np.zeros((1, 8, 1, 4))
+    kk[0, 0, 0] = [1.0, 1.0, 1.0, 1.0]
+    kk[0, 7, 0] = [0.5, 0.0, 0.25, 1.0]
+    vv[0, 0, 0] = [1.0, 0.0, 0.0, 0.0]
+    vv[0, 7, 0] = [0.0, 1.0, 0.0, 0.0]
+    vv[0, 1:7, 0, 2] = 1.0
+    kw = dict(Hq=1, Hkv=1, q_pos0=7, k_pos0=0, base=100.0, alpha=1.0, g=1, scale=1.0,
+              rows=[(0, 0, 0)], block_q=1, block_k=4)
+    out, lse = oracle.attention_rows_masked(q, _bf16_bits(kk), _bf16_bits(vv),
+                                            np.array([0, 1]).reshape(1, 1, 1, 2), **kw)
+    z = 3.0 + math.exp(5.25)
+    np.testing.assert_allclose(out[0], [0.0, math.exp(5.25) / z, 3.0 / z, 0.0], rtol=0, atol=1e-12)
+    assert abs(lse[0] - math.log(z)) < 1e-12
+    out, lse = oracle.attention_rows_masked(q, _bf16_bits(kk), _bf16_bits(vv),
+                                            np.array([1, 0]).reshape(1, 1, 1, 2), **kw)
+    z = math.exp(6.0) + 3.0
+    np.testing.assert_allclose(out[0], [math.exp(6.0) / z, 0.0, 3.0 / z, 0.0], rtol=0, atol=1e-12)
+    assert abs(lse[0] - math.log(z)) < 1e-12
+    out, lse = oracle.attention_rows_masked(q, _bf16_bits(kk), _bf16_bits(vv),
+                                            np.zeros((1, 1, 1, 2)), **kw)
+    assert (out == 0).all() and lse[0] == -math.inf
+
+
+def test_block_mask_all_ones_is_attention_rows():
+    q = _rand((2, 70, 2, 16), 91)
+    k = _rand((2, 70, 1, 16), 92)
+    v = _rand((2, 70, 1, 16), 93)
+    rows = [(b, h, t) for b in range(2) for h in range(2) for t in range(0, 70, 3)]
+    kw = dict(Hq=2, Hkv=1, base=1e4, alpha=1.0, g=1, scale=0.25, rows=rows)
+    a = oracle.attention_rows(inputs.bits(q), inputs.bits(k), inputs.bits(v), **kw)
+    m = np.ones((2, 2, 3, 5), dtype=np.uint8)
+    b = oracle.attention_rows_masked(inputs.bits(q), inputs.bits(k), inputs.bits(v), m,
+                                     block_q=32, block_k=16, **kw)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_block_mask_alpha_inf_is_masked_sdpa():
+    """alpha = inf: ordinary attention under (causal AND block mask), by a library routine."""
+    B, Nq, Nk, Hq, Hkv, D, q0, k0 = 2, 40, 56, 2, 1, 16, 16, 0
+    q = _rand((B, Nq, Hq, D), 94)
+    k = _rand((B, Nk, Hkv, D), 95)
+    v = _rand((B, Nk, Hkv, D), 96)
+    bq, bk = 8, 8
+    rng = np.random.default_rng(3)
+    m = (rng.random((B, Hq, Nq // bq, Nk // bk)) < 0.5).astype(np.uint8)
+    rows = [(b, h, t) for b in range(B) for h in range(Hq) for t in range(Nq)]
+    out, lse = oracle.attention_rows_masked(inputs.bits(q), inputs.bits(k), inputs.bits(v), m,
+                                            Hq=Hq, Hkv=Hkv, q_pos0=q0, k_pos0=k0, base=1e4,
+                                            alpha=float("inf"), g=1, scale=0.25, rows=rows,
+                                            block_q=bq, block_k=bk)
+    qf = q.double().permute(0, 2, 1, 3)
+    kf = k.double().repeat_interleave(Hq // Hkv, dim=2).permute(0, 2, 1, 3)
+    vf = v.double().repeat_interleave(Hq // Hkv, dim=2).permute(0, 2, 1, 3)
+    causal = (k0 + torch.arange(Nk))[None, :] <= (q0 + torch.arange(Nq))[:, None]
+    blk = torch.tensor(m, dtype=torch.bool).repeat_interleave(bq, 2).repeat_interleave(bk, 3)
+    allowed = causal[None, None] & blk
+    z = 0.25 * qf @ kf.transpose(-1, -2)
+    z = torch.where(allowed, z, torch.tensor(-math.inf, dtype=torch.float64))
+    for n, (b, h, t) in enumerate(rows):
+        if not allowed[b, h, t].any():
+            assert lse[n] == -math.inf and (out[n] == 0).all()
+            continue
+        want = torch.softmax(z[b, h, t], 0) @ vf[b, h]
+        np.testing.assert_allclose(out[n], want.numpy(), atol=1e-10)
+        assert abs(lse[n] - float(torch.logsumexp(z[b, h, t], 0))) < 1e-10
+    assert (~allowed.reshape(-1, Nk).any(1)).any()     # some rows are empty: the case is covered
