@@ -50,9 +50,9 @@ FLUSH_BYTES = 512 << 20
 NCU_TRAFFIC = {
     # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.134912 MB read + 23.742208 MB written
     ("qwen2.5-0.5b-32k", "78ae9ff5d51882a2"): 76134912 + 23742208,
-    # profiles/decode_split_kernel_llama3.2-3b-decode-32k.md: 537.025280 MB read + 6.628608 MB
+    # profiles/decode_split_kernel_llama3.2-3b-decode-32k.md: 536.942080 MB read + 7.402752 MB
     # written for B=4, L=32768, scaled by the 16x keys x heads of the B=16, L=131072 call
-    ("llama3.2-3b-decode-128k", "f05ba464b5fd744d"): 16 * (537025280 + 6628608),
+    ("llama3.2-3b-decode-128k", "fd8fb0cb72b0635b"): 16 * (536942080 + 7402752),
 }
 
 KERNEL_SOURCES = {"prefill": ("prefill_kernel.cuh", "device_util.cuh"),

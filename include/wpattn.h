@@ -117,6 +117,42 @@ WPATTN_API int wpattn_prefill(const wpattn_window *w,
                    void *cuda_stream);
 
 /*
+ * Prefill with a block mask stacked on the window (token-level block
+ * sparsity of the MInference kind; ATFlash Abstract: the window is orthogonal
+ * to token selection and composes with it).  Same arguments and results as
+ * wpattn_prefill, plus:
+ *   block_mask: device uint32 [B, Hq, ceil(Nq / 128), mask_words], 4-byte
+ *               aligned.  Query rows 128 qb .. 128 qb + 127 of head h attend
+ *               keys 128 kb .. 128 kb + 127 only if bit kb % 32 of word
+ *               kb / 32 of row (b, h, qb) is set; the window and causality
+ *               then apply to the attended keys.  Bits past ceil(Nk / 128)
+ *               are ignored.  Build it from a byte mask with
+ *               wpattn_pack_block_mask.
+ *   mask_words: words per row, >= ceil(ceil(Nk / 128) / 32) (else
+ *               WPATTN_EINVAL).
+ * Key tiles that no query tile of a CTA attends are neither loaded nor
+ * computed.  A query left with no key gets out = 0 and lse = -inf.  An
+ * all-ones mask gives wpattn_prefill's output bit for bit.
+ */
+WPATTN_API int wpattn_prefill_masked(const wpattn_window *w,
+                  const void *q, const void *k, const void *v,
+                  void *out, float *lse,
+                  int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
+                  int64_t q_pos0, int64_t k_pos0, float softmax_scale,
+                  const uint32_t *block_mask, int32_t mask_words,
+                  void *cuda_stream);
+
+/*
+ * Pack a byte block mask (device uint8 [rows, nkb], nonzero = attended) into
+ * the bit rows wpattn_prefill_masked reads (device uint32 [rows, mask_words],
+ * caller-allocated, 4-byte aligned; bit kb % 32 of word kb / 32, zero past
+ * nkb).  mask_words >= ceil(nkb / 32) (else WPATTN_EINVAL).  Asynchronous on
+ * `cuda_stream`; bit-exact.
+ */
+WPATTN_API int wpattn_pack_block_mask(const uint8_t *mask, uint32_t *words, int64_t rows,
+                  int32_t nkb, int32_t mask_words, void *cuda_stream);
+
+/*
  * Bytes of device workspace wpattn_decode needs for up to B sequences of up
  * to max_kv_len keys (0 on bad arguments).  The split of each sequence into
  * key ranges depends only on (B, Hkv, max_kv_len) and the device's SM count.

@@ -9,7 +9,7 @@ exception is raised.
 
 Entry points (same names as the C ABI, without the ``wpattn_`` prefix):
 ``prefill``, ``decode``, ``decode_pairmajor``, ``kcache_to_pairmajor``,
-``decode_positions``, ``decode_paged``,
+``decode_positions``, ``decode_paged``, ``prefill_masked``, ``pack_block_mask``,
 ``decode_workspace_size``, ``decode_noalloc``, ``pruned_fraction``,
 ``thresholds``, ``device_status``.
 """
@@ -68,6 +68,9 @@ def lib() -> ctypes.CDLL:
                                              ctypes.POINTER(ctypes.c_double)]
         L.wpattn_prefill.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64, i64,
                                      f32, vp]
+        L.wpattn_prefill_masked.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64,
+                                            i64, f32, vp, i32, vp]
+        L.wpattn_pack_block_mask.argtypes = [vp, vp, i64, i32, i32, vp]
         L.wpattn_decode_workspace_size.restype = ctypes.c_size_t
         L.wpattn_decode_workspace_size.argtypes = [wp, i32, i32, i32, i64]
         L.wpattn_decode.argtypes = [wp, vp, vp, vp, ctypes.POINTER(ctypes.c_int32), i64, i32, i32,
@@ -154,6 +157,61 @@ def prefill(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0, scale: floa
                               B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0,
                               float(scale) if scale else 0.0, _stream_ptr(stream))
     _check(rc, "wpattn_prefill")
+    return out, lse
+
+
+MASK_BLOCK = 128  # rows and keys covered by one block-mask entry
+
+
+def pack_block_mask(mask, stream=None):
+    """Block mask [B, Hq, ceil(Nq/128), ceil(Nk/128)] (bool or uint8 CUDA, nonzero =
+    attended) -> the packed bit rows ``prefill_masked`` reads: int32 [B, Hq, nqb,
+    ceil(nkb/32)], bit kb % 32 of word kb // 32."""
+    import torch
+    if not isinstance(mask, torch.Tensor) or not mask.is_cuda or mask.dim() != 4:
+        raise TypeError("mask must be a 4-D CUDA tensor")
+    if mask.dtype == torch.bool:
+        mask = mask.view(torch.uint8)
+    if mask.dtype != torch.uint8 or not mask.is_contiguous():
+        raise TypeError("mask must be a contiguous bool or uint8 tensor")
+    B, Hq, nqb, nkb = mask.shape
+    nw = (nkb + 31) // 32
+    words = torch.empty((B, Hq, nqb, nw), dtype=torch.int32, device=mask.device)
+    _check(lib().wpattn_pack_block_mask(ctypes.c_void_p(mask.data_ptr()),
+                                        ctypes.c_void_p(words.data_ptr()), B * Hq * nqb, nkb, nw,
+                                        _stream_ptr(stream)), "wpattn_pack_block_mask")
+    return words
+
+
+def prefill_masked(q, k, v, block_mask, w: Window, *, q_pos0: int = 0, k_pos0: int = 0,
+                   scale: float | None = None, out=None, lse=None, want_lse: bool = True,
+                   stream=None):
+    """``prefill`` with a 128 x 128 block mask on top of the window and causality.
+
+    block_mask: bool / uint8 [B, Hq, ceil(Nq/128), ceil(Nk/128)] (packed here), or the
+    packed int32 words from ``pack_block_mask``.
+    """
+    import torch
+    B, Nq, Hq, D = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    if block_mask.dtype != torch.int32:
+        block_mask = pack_block_mask(block_mask, stream=stream)
+    nqb = (Nq + MASK_BLOCK - 1) // MASK_BLOCK
+    if (block_mask.dim() != 4 or tuple(block_mask.shape[:3]) != (B, Hq, nqb)
+            or not block_mask.is_cuda or not block_mask.is_contiguous()):
+        raise TypeError(f"packed block mask must be a contiguous CUDA int32 [B, Hq, {nqb}, words]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = lib().wpattn_prefill_masked(ctypes.byref(w._c()), _dev_tensor(q, "q"), _dev_tensor(k, "k"),
+                                     _dev_tensor(v, "v"), _dev_tensor(out, "out"),
+                                     ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+                                     B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0,
+                                     float(scale) if scale else 0.0,
+                                     ctypes.c_void_p(block_mask.data_ptr()), block_mask.shape[3],
+                                     _stream_ptr(stream))
+    _check(rc, "wpattn_prefill_masked")
     return out, lse
 
 

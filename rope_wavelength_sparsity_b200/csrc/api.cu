@@ -46,7 +46,7 @@ struct DeviceInfo {
   bool init = false;
   bool supported = false;
   int num_sms = 0;
-  bool prefill_attr[4] = {false, false, false, false};  // (D 64, 128) x (g 1, 8)
+  bool prefill_attr[8] = {};  // (D 64, 128) x (g 1, 8) x (no mask, block mask)
   void* static_scratch = nullptr;  // device address of g_decode_static_scratch
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -103,7 +103,7 @@ int encode_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
   return r == CUDA_SUCCESS ? WPATTN_OK : WPATTN_ECUDA;
 }
 
-template <int D, bool G8>
+template <int D, bool G8, bool MASK>
 int launch_prefill(const void* q, const void* k, const void* v, PrefillParams prm,
                    DeviceInfo* dev, cudaStream_t st) {
   using Shape = PrefillShape<D>;
@@ -118,16 +118,25 @@ int launch_prefill(const void* q, const void* k, const void* v, PrefillParams pr
   if ((rc = encode_bf16_4d(&tk, k, D, nk, hk, prm.B, 8, Shape::BN, false)) != WPATTN_OK) return rc;
   if ((rc = encode_bf16_4d(&tv, v, D, nk, hk, prm.B, 64, Shape::BN, true)) != WPATTN_OK) return rc;
   constexpr int smem = PrefillSmem<D>::ALLOC;
-  const int slot = (D == 64 ? 0 : 2) + (G8 ? 1 : 0);
+  const int slot = (D == 64 ? 0 : 2) + (G8 ? 1 : 0) + (MASK ? 4 : 0);
+  // a mask bit covers one 128-row query tile x one 128-key tile
+  if (MASK && (Shape::BN != 128 || kBM != 128)) return WPATTN_EUNSUPPORTED;
   if (!dev->prefill_attr[slot]) {
-    if (cudaFuncSetAttribute(prefill_kernel<D, G8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(prefill_kernel<D, G8, MASK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
       return WPATTN_ECUDA;
     dev->prefill_attr[slot] = true;
   }
   dim3 grid(prm.num_ctas_q, prm.Hq, prm.B);
-  prefill_kernel<D, G8><<<grid, Shape::THREADS, smem, st>>>(tq, tk, tv, prm);
+  prefill_kernel<D, G8, MASK><<<grid, Shape::THREADS, smem, st>>>(tq, tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
+}
+
+template <int D, bool MASK>
+int launch_prefill_g(const void* q, const void* k, const void* v, const PrefillParams& prm,
+                     DeviceInfo* dev, cudaStream_t st) {
+  return prm.g8 ? launch_prefill<D, true, MASK>(q, k, v, prm, dev, st)
+                : launch_prefill<D, false, MASK>(q, k, v, prm, dev, st);
 }
 
 template <int D, int GC, bool PM>
@@ -268,9 +277,14 @@ int wpattn_pruned_fraction(const wpattn_window* w, int64_t Nq, int64_t Nk, int64
   return WPATTN_OK;
 }
 
-int wpattn_prefill(const wpattn_window* w, const void* q, const void* k, const void* v, void* out,
-                   float* lse, int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
-                   int64_t q_pos0, int64_t k_pos0, float softmax_scale, void* cuda_stream) {
+}  // extern "C"
+
+namespace {
+// wpattn_prefill and wpattn_prefill_masked: block_mask null = no mask
+int prefill_impl(const wpattn_window* w, const void* q, const void* k, const void* v, void* out,
+                 float* lse, int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
+                 int64_t q_pos0, int64_t k_pos0, float softmax_scale, const uint32_t* block_mask,
+                 int32_t mask_words, void* cuda_stream) {
   WindowPlan plan;
   int rc = make_window_plan(w, &plan);
   if (rc != WPATTN_OK) return rc;
@@ -303,15 +317,58 @@ int wpattn_prefill(const wpattn_window* w, const void* q, const void* k, const v
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(plan.D));
   prm.scale_log2 = scale * 1.44269504088896340736f;
   prm.g8 = plan.g == 8 ? 1 : 0;
+  if (block_mask) {
+    const int64_t nkt = (static_cast<int64_t>(Nk) + 127) / 128;
+    if (mask_words < (nkt + 31) / 32 || (reinterpret_cast<uintptr_t>(block_mask) & 3u) != 0)
+      return WPATTN_EINVAL;
+    prm.block_mask = block_mask;
+    prm.mask_words = mask_words;
+  }
   for (int p = 0; p < 64; ++p) prm.T[p] = plan.T[p] > INT32_MAX ? INT32_MAX : static_cast<int>(plan.T[p]);
   const void* kk = Nk > 0 ? k : q;
   const void* vv = Nk > 0 ? v : q;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   if (plan.D == 64)
-    return prm.g8 ? launch_prefill<64, true>(q, kk, vv, prm, dev, st)
-                  : launch_prefill<64, false>(q, kk, vv, prm, dev, st);
-  return prm.g8 ? launch_prefill<128, true>(q, kk, vv, prm, dev, st)
-                : launch_prefill<128, false>(q, kk, vv, prm, dev, st);
+    return prm.block_mask ? launch_prefill_g<64, true>(q, kk, vv, prm, dev, st)
+                          : launch_prefill_g<64, false>(q, kk, vv, prm, dev, st);
+  return prm.block_mask ? launch_prefill_g<128, true>(q, kk, vv, prm, dev, st)
+                        : launch_prefill_g<128, false>(q, kk, vv, prm, dev, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int wpattn_prefill(const wpattn_window* w, const void* q, const void* k, const void* v, void* out,
+                   float* lse, int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
+                   int64_t q_pos0, int64_t k_pos0, float softmax_scale, void* cuda_stream) {
+  return prefill_impl(w, q, k, v, out, lse, B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0, softmax_scale,
+                      nullptr, 0, cuda_stream);
+}
+
+int wpattn_prefill_masked(const wpattn_window* w, const void* q, const void* k, const void* v,
+                          void* out, float* lse, int32_t B, int32_t Nq, int32_t Nk, int32_t Hq,
+                          int32_t Hkv, int64_t q_pos0, int64_t k_pos0, float softmax_scale,
+                          const uint32_t* block_mask, int32_t mask_words, void* cuda_stream) {
+  if (!block_mask) return WPATTN_EINVAL;
+  return prefill_impl(w, q, k, v, out, lse, B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0, softmax_scale,
+                      block_mask, mask_words, cuda_stream);
+}
+
+int wpattn_pack_block_mask(const uint8_t* mask, uint32_t* words, int64_t rows, int32_t nkb,
+                           int32_t mask_words, void* cuda_stream) {
+  if (rows < 0 || nkb < 0 || mask_words < (nkb + 31) / 32) return WPATTN_EINVAL;
+  if (rows == 0 || mask_words == 0) return WPATTN_OK;
+  if (!mask || !words || (reinterpret_cast<uintptr_t>(words) & 3u) != 0) return WPATTN_EINVAL;
+  DeviceInfo* dev = nullptr;
+  int rc;
+  if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
+  const uint64_t n = static_cast<uint64_t>(rows) * static_cast<uint64_t>(mask_words);
+  const uint64_t blocks = (n + 255) / 256;
+  if (blocks > 0x7FFFFFFFull) return WPATTN_EUNSUPPORTED;
+  pack_block_mask_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
+      mask, words, rows, nkb, mask_words);
+  return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
 size_t wpattn_decode_workspace_size(const wpattn_window* w, int32_t B, int32_t Hq, int32_t Hkv,

@@ -71,6 +71,11 @@ struct PrefillParams {
   float scale_log2;   // softmax scale * log2(e)
   int g8;             // 1: pairs share thresholds in groups of 8
   int T[64];          // per-pair thresholds (nondecreasing), clamped to INT32_MAX
+  // block mask, or null: query tile qt (rows 128 qt ..) attends key tile kt
+  // (keys 128 kt ..) iff bit kt % 32 of word kt / 32 of row (b, h, qt) is set;
+  // rows of mask_words words, [B, Hq, ceil(Nq / 128), mask_words]
+  const uint32_t* block_mask;
+  int mask_words;
 };
 
 template <int D>
@@ -107,8 +112,10 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 }
 
 // G8: pairs share thresholds in groups of 8 (a compile-time switch, so the
-// two correction paths do not share a register allocation)
-template <int D, bool G8>
+// two correction paths do not share a register allocation).  MASK: a block
+// mask selects the key tiles (compile-time too, so that the plain causal walk
+// keeps its registers).
+template <int D, bool G8, bool MASK>
 __global__ void __launch_bounds__(PrefillShape<D>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ PrefillParams p) {
@@ -167,10 +174,54 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   int kt_last[QT];
 #pragma unroll
   for (int t = 0; t < QT; ++t) kt_last[t] = last_key_tile(t);
-  int kt_top = kt_last[0];
+  // Key tiles query tile t attends: at most its causal limit lim, and with a
+  // block mask only those whose bit is set.  Largest such tile <= kt, or -1.
+  const int nqt = (p.Nq + kBM - 1) / kBM;
+  auto attended_below = [&](int t, int kt, int lim) -> int {
+    kt = min(kt, lim);
+    if (kt < 0) return -1;
+    if constexpr (!MASK) return kt;
+    const uint32_t* row =
+        p.block_mask + ((size_t)(b * p.Hq + h) * nqt + (QT * cq + t)) * p.mask_words;
+    while (kt >= 0) {
+      const uint32_t w = __ldg(row + (kt >> 5)) & (0xFFFFFFFFu >> (31 - (kt & 31)));
+      if (w) return (kt & ~31) + 31 - __clz(w);
+      kt = (kt & ~31) - 1;
+    }
+    return -1;
+  };
+  // The CTA's K/V stream: the key tiles some of its query tiles attend, from the
+  // top down.  Step j of the stream is key tile kt_j; bit t of *mem says whether
+  // query tile t attends it.  Every role walks the same stream.
+  auto stream_below = [&](int kt, uint32_t* mem) -> int {
+    if constexpr (!MASK) {  // every tile up to the causal limit: the stream is a countdown
+      int top = -1;
 #pragma unroll
-  for (int t = 1; t < QT; ++t) kt_top = max(kt_top, kt_last[t]);
-  const int n_iter = kt_top + 1;  // shared K/V iterations j: key tile kt_top - j
+      for (int t = 0; t < QT; ++t) top = max(top, kt_last[t]);
+      const int u = min(kt, top);
+      uint32_t bits = 0;
+#pragma unroll
+      for (int t = 0; t < QT; ++t) bits |= (u >= 0 && u <= kt_last[t]) ? (1u << t) : 0u;
+      *mem = bits;
+      return u < 0 ? -1 : u;
+    }
+    int a[QT], u = -1;
+#pragma unroll
+    for (int t = 0; t < QT; ++t) { a[t] = attended_below(t, kt, kt_last[t]); u = max(u, a[t]); }
+    uint32_t bits = 0;
+#pragma unroll
+    for (int t = 0; t < QT; ++t) bits |= (u >= 0 && a[t] == u) ? (1u << t) : 0u;
+    *mem = bits;
+    return u;
+  };
+  uint32_t mem_top;
+  const int kt_top = stream_below(nkt - 1, &mem_top);  // first step of the stream, -1 if none
+  // the step after key tile kt (for the roles that do not need the bits)
+  auto stream_next = [&](int kt) -> int {
+    if constexpr (!MASK) return kt - 1;
+    uint32_t unused;
+    return stream_below(kt - 1, &unused);
+  };
   // Smallest distance of query tile t in key tile kt (negative on the diagonal).
   // Going down the key tiles it grows by 128, so the first kept pair of the
   // tile (p_min of that distance) only moves forward: advance it in place.
@@ -226,7 +277,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   regs_decrease<PrefillShape<D>::REGS_OTHER>();
   if (warp == W_PROD) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n_iter > 0) {
+    if (lane == 0 && kt_top >= 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
@@ -237,8 +288,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int t = 0; t < nq_tiles; ++t)
         for (int c = 0; c < D / 8; ++c)
           tma_load_4d(sQ + t * L::QTILE + c * PANEL_Q, &tmQ, q_full, 8 * c, (QT * cq + t) * kBM, h, b);
-      for (int j = 0; j < n_iter; ++j) {
-        const int kt = kt_top - j;
+      for (int j = 0, kt = kt_top; kt >= 0; ++j, kt = stream_next(kt)) {
         const int s = j % NS;
         const uint32_t ph = (j / NS) & 1;
         if (j >= NS && !mbar_wait(k_empty(s), ph ^ 1)) break;
@@ -253,7 +303,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
   } else if (warp == W_MMA) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0 && n_iter > 0) {
+    if (lane == 0 && kt_top >= 0) {
       constexpr uint32_t idesc_qk = make_idesc_bf16(kBM, BN, 0, 0);
       constexpr uint32_t idesc_pv = make_idesc_bf16(kBM, D, 0, 1);
       bool ok = mbar_wait(q_full, 0);
@@ -269,9 +319,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint64_t qmdesc0 = make_sdesc(sQM, PANEL_Q, 128, 0);
       const uint64_t kdesc0 = make_sdesc(sK, (D / 16) * PANEL_K, 128, 0);
       const uint64_t vdesc0 = make_sdesc(sV, BN * 128, 1024, 2);
-      // split pair of QK_t(j): planned ahead of the wait for P_t(j - 1)
-      auto plan_qk = [&](int t, int j) -> int {
-        const int kt = kt_top - j;
+      // split pair of QK_t on key tile kt: planned ahead of the wait for P_t
+      auto plan_qk = [&](int t, int kt) -> int {
         advance_plo(t, kt, plo[t]);
         return split_pair(t, kt, plo[t], psr[t]);
       };
@@ -299,23 +348,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_after();
 #pragma unroll
         for (int t = 0; t < QT; ++t)
-          if (ok && kt_last[t] >= kt_top && !issue_qk(t, 0, plan_qk(t, 0))) ok = false;
+          if (ok && (MASK ? ((mem_top >> t) & 1u) != 0 : kt_last[t] >= kt_top) &&
+              !issue_qk(t, 0, plan_qk(t, kt_top)))
+            ok = false;
         umma_commit(k_empty(0));
       } else {
         ok = false;
       }
-      for (int j = 0; ok && j < n_iter; ++j) {
-        const int kt = kt_top - j;
-        const bool next = j + 1 < n_iter;
+      // without a mask, query tile t attends step kt iff kt <= kt_last[t] (no bits carried)
+      uint32_t mem = MASK ? mem_top : 0u;
+      for (int j = 0, kt = kt_top; ok && kt >= 0; ++j) {
+        uint32_t mem_n = 0;
+        int kt_n;
+        if constexpr (MASK) kt_n = stream_below(kt - 1, &mem_n);
+        else kt_n = kt - 1;
+        const bool next = kt_n >= 0;
         if (next && !mbar_wait(k_full((j + 1) % NS), ((j + 1) / NS) & 1)) { ok = false; break; }
         if (!mbar_wait(v_full(j % NS), (j / NS) & 1)) { ok = false; break; }
         const uint64_t vbase = vdesc0 + (uint64_t)(((j % NS) * L::KTILE) >> 4);
 #pragma unroll
         for (int t = 0; t < QT; ++t) {
-          const int ktl = kt_last[t];
-          const bool do_qk = ok && next && kt - 1 <= ktl;
-          const int ps_n = do_qk ? plan_qk(t, j + 1) : 0;
-          if (ok && kt <= ktl) {
+          const bool in_n = MASK ? ((mem_n >> t) & 1u) != 0 : kt_n <= kt_last[t];
+          const bool in_j = MASK ? ((mem >> t) & 1u) != 0 : kt <= kt_last[t];
+          const bool do_qk = ok && next && in_n;
+          const int ps_n = do_qk ? plan_qk(t, kt_n) : 0;
+          if (ok && in_j) {
             if (!mbar_wait(p_full(t), cnt[t] & 1)) { ok = false; }
             if (ok) {
               tc_fence_after();
@@ -331,6 +388,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!ok) break;
         umma_commit(v_empty(j % NS));
         if (next) umma_commit(k_empty((j + 1) % NS));
+        kt = kt_n;
+        if constexpr (MASK) mem = mem_n;
       }
       // O_t final: every MMA issued so far has completed once this arrives
       for (int t = 0; t < QT; ++t) umma_commit(o_final(t));
@@ -352,6 +411,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     uint8_t* smem_qm = smem + L::OFF_QM + t * 2 * PANEL_Q;
     const int i_tile0 = p.qk_off + (QT * cq + t) * kBM;  // relative position of the first row
     const int my_kt_last = last_key_tile(t);
+    int my_next = attended_below(t, my_kt_last, my_kt_last);  // this tile's next key tile, -1 when done
     float m_ref = -INFINITY;   // exponent reference of O and l (log2 units)
     float l_run = 0.f;
     int cnt = 0;
@@ -376,22 +436,23 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     };
 
     // Q is read from shared memory for the masked copy and the corrections
-    ok = __all_sync(FULL, mbar_wait(q_full, 0));
+    // (it is loaded only when the CTA's stream has a key tile)
+    ok = kt_top < 0 || __all_sync(FULL, mbar_wait(q_full, 0));
     int plo_next = 0;
-    if (my_kt_last >= 0) advance_plo(t, my_kt_last, plo_next); else plo_next = P;
+    if (my_next >= 0) advance_plo(t, my_next, plo_next); else plo_next = P;
     int psr = 0;
-    int ps_next = my_kt_last >= 0 ? split_pair(t, my_kt_last, plo_next, psr) : P;
-    if (ok && my_kt_last >= 0) write_masked_q(ps_next);
+    int ps_next = my_next >= 0 ? split_pair(t, my_next, plo_next, psr) : P;
+    if (ok && my_next >= 0) write_masked_q(ps_next);
     __syncwarp();
     if (lane == 0) mbar_arrive(qm_init(t));
 
-    for (int j = 0; ok && j < n_iter; ++j) {
-      const int kt = kt_top - j;
+    for (int j = 0, kt = kt_top; ok && kt >= 0; ++j, kt = stream_next(kt)) {
       const int s = j % NS;
-      if (kt > my_kt_last) {
-        // no key of this tile is causal for us: only release K.  Wait for the
-        // stage's fill first, so that this arrival counts towards iteration j
-        // and not towards an earlier phase of the same stage.
+      if (MASK ? kt != my_next : kt > my_kt_last) {
+        // a key tile this query tile does not attend (past its rows, or
+        // masked out): only release K.  Wait for the stage's fill first, so
+        // that this arrival counts towards step j and not towards an earlier
+        // phase of the same stage.
         if (!__all_sync(FULL, mbar_wait(k_full(s), (j / NS) & 1))) { ok = false; break; }
         __syncwarp();
         if (lane == 0) mbar_arrive(k_empty(s));
@@ -401,9 +462,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int d_row = i_pos - kp0;         // distance to the tile's first key
       const int plo = plo_next, ps = ps_next;
       const bool all_pruned = plo >= P;
-      if (kt > 0) {
-        advance_plo(t, kt - 1, plo_next);
-        ps_next = split_pair(t, kt - 1, plo_next, psr);
+      if constexpr (MASK) my_next = attended_below(t, kt - 1, my_kt_last);
+      else my_next = kt - 1;  // below the first attended tile, every tile is attended
+      if (my_next >= 0) {
+        advance_plo(t, my_next, plo_next);
+        ps_next = split_pair(t, my_next, plo_next, psr);
       }
 
       // Per-element corrections, d = d_row - c for column c of the tile:
@@ -699,7 +762,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tmem_st32u(tS + 32, &pk[32]);
       }
       // the next tile's masked Q step, before P is released to the MMA warp
-      if (kt > 0) write_masked_q(ps_next);
+      if (MASK ? my_next >= 0 : kt > 0) write_masked_q(ps_next);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -746,6 +809,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+// Byte block mask [rows, nkb] (nonzero = attended) -> the kernel's bit rows of
+// mask_words words: bit kb % 32 of word kb / 32, zero past nkb.  One thread
+// per word.
+__global__ void __launch_bounds__(256)
+pack_block_mask_kernel(const uint8_t* __restrict__ mask, uint32_t* __restrict__ words, int64_t rows,
+                       int nkb, int mask_words) {
+  const uint64_t idx = static_cast<uint64_t>(blockIdx.x) * 256u + threadIdx.x;
+  if (idx >= static_cast<uint64_t>(rows) * static_cast<uint64_t>(mask_words)) return;
+  const uint64_t r = idx / static_cast<uint64_t>(mask_words);
+  const int wi = static_cast<int>(idx % static_cast<uint64_t>(mask_words));
+  const uint8_t* src = mask + r * static_cast<uint64_t>(nkb);
+  uint32_t w = 0;
+  for (int i = 0; i < 32; ++i) {
+    const int kb = wi * 32 + i;
+    if (kb < nkb && src[kb]) w |= 1u << i;
+  }
+  words[idx] = w;
 }
 
 }  // namespace wpattn

@@ -22,8 +22,9 @@ def check_rows(o_gpu, l_gpu, o_ref, l_ref, what):
     if empty.any():
         assert (o_gpu[empty] == 0).all(), f"{what}: empty rows must be 0"
     ok = ~empty
-    err_o = np.where(ok[:, None], np.abs(o_gpu - o_ref), 0.0).max(axis=1)
-    err_l = np.where(ok, np.abs(l_gpu - l_ref), 0.0)
+    with np.errstate(invalid="ignore"):  # empty rows: -inf - -inf, masked out below
+        err_o = np.where(ok[:, None], np.abs(o_gpu - o_ref), 0.0).max(axis=1)
+        err_l = np.where(ok, np.abs(l_gpu - l_ref), 0.0)
     d_out, d_lse = float(err_o.max()), float(err_l.max())
     bad = np.nonzero((err_o > ATOL_OUT) | (err_l > ATOL_LSE))[0]
     assert d_out <= ATOL_OUT and d_lse <= ATOL_LSE, (
