@@ -92,6 +92,25 @@ def prefill_flops(w, win, wp):
     return w.B * w.Hq * per_head, w.B * w.Hq * off
 
 
+def masked_flops(w, win, wp, mask):
+    """Effective FLOPs of one prefill under a block mask (bool [B, Hq, nqb, nkb], 128 x 128
+    blocks): the kept QK pair-terms and PV of the causal (query, key) pairs of each attended
+    block, counted block by block with the closed-form count."""
+    P, blk = w.D // 2, wp.MASK_BLOCK
+    cache = {}
+    total = 0
+    for idx in mask.nonzero().tolist():
+        qb, kb = idx[2], idx[3]
+        nq = min(blk, w.Nq - qb * blk)
+        nk = min(blk, w.Nk - kb * blk)
+        key = (nq, nk, w.q_pos0 + qb * blk - (w.k_pos0 + kb * blk))
+        if key not in cache:
+            pr, tot, _ = wp.pruned_fraction(win, nq, nk, key[2], 0)
+            cache[key] = 4 * (tot - pr) + 2 * w.D * (tot // P)
+        total += cache[key]
+    return total
+
+
 def decode_bytes(w, win, wp, kv_len):
     """(algorithmic bytes, window-off bytes) of one decode step."""
     P = w.D // 2
@@ -267,6 +286,38 @@ def gpu_arm(args):
         off_ms, _, _ = time_steps(step_off, args.warmup, max(3, args.steps // 4), flush, world)
         off_ms_step = off_ms / max(3, args.steps // 4)
         ms_step = total_ms / args.steps
+        masked = None
+        if not args.only_primary:
+            # the same call under a MInference-shaped block mask (vertical + slash tiles)
+            mask = inputs.vertical_slash_mask(w.B, w.Hq, w.Nq, w.Nk, seed=rank, q_pos0=w.q_pos0,
+                                              k_pos0=w.k_pos0)
+            words = wp.pack_block_mask(mask.to(dev))
+            m_eff = masked_flops(w, win, wp, mask)
+
+            def step_masked():
+                wp.prefill_masked(q, k, v, words, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0,
+                                  scale=w.scale, out=out, lse=lse)
+
+            n_m = max(3, args.steps // 2)
+            m_ms, m_per, _ = time_steps(step_masked, args.warmup, n_m, flush, world)
+            if wp.device_status() != wp.OK:
+                raise RuntimeError("masked prefill kernel status: not ok")
+            m_kernel = statistics.mean(m_per)
+            causal_tiles = sum(1 for qb in range(mask.shape[2]) for kb in range(mask.shape[3])
+                               if kb * 128 + w.k_pos0 <= w.q_pos0 + qb * 128 + 127)
+            masked = {
+                "value": round(weak_scaling_value(m_eff, world, m_ms / n_m) / 1e12, 2),
+                "unit": "TFLOP/s", "ms_per_step": round(m_ms / n_m, 4),
+                "roofline": {"bound": "tensor", "achieved": round(m_eff / (m_kernel * 1e-3) / 1e12, 2),
+                             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": round(m_eff / (m_kernel * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                             "traffic": None},
+                "speedup_vs_unmasked": round(ms_step / (m_ms / n_m), 3),
+                "ideal_speedup": round(eff / m_eff, 3),
+                "attended_tile_fraction": round(float(mask.sum()) / (w.B * w.Hq * causal_tiles), 4),
+                "mask": "vertical-slash: sink + 3 random key tiles per head, 16-tile diagonal band",
+            }
+            del words, mask
         value = weak_scaling_value(eff, world, ms_step) / 1e12
         kernel_ms = statistics.mean(per)
         achieved = eff / (kernel_ms * 1e-3) / 1e12
@@ -290,6 +341,9 @@ def gpu_arm(args):
             "gpu_launches": args.steps,
             "clocks": clk,
         })
+        if masked is not None:
+            result["block_sparse"] = masked
+            result["gpu_launches"] += max(3, args.steps // 2)
         # end to end through the public API with pinned host buffers
         qh = q.cpu().pin_memory()
         kh = k.cpu().pin_memory()

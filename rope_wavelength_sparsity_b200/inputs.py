@@ -249,3 +249,24 @@ def key_positions(kv_len, seed: int, mode: str = "evicted", span: float = 4.0):
         k_pos[b, :n] = keep
         q_pos.append(qp)
     return q_pos, k_pos
+
+
+def vertical_slash_mask(B: int, Hq: int, Nq: int, Nk: int, seed: int, q_pos0: int = 0,
+                        k_pos0: int = 0, n_vertical: int = 4, band: int = 16, block: int = 128):
+    """bool [B, Hq, ceil(Nq/block), ceil(Nk/block)] block mask of the MInference
+    'vertical-slash' shape: per head, key tile 0 (the sink) and n_vertical - 1
+    other key tiles drawn at random, attended by every query tile, plus a band
+    of ``band`` key tiles ending at each query tile's diagonal tile."""
+    g = _gen(seed, "cpu")
+    nqb, nkb = -(-Nq // block), -(-Nk // block)
+    m = torch.zeros((B, Hq, nqb, nkb), dtype=torch.bool)
+    for b in range(B):
+        for h in range(Hq):
+            cols = [0] + torch.randint(0, nkb, (max(0, n_vertical - 1),), generator=g).tolist()
+            m[b, h, :, cols] = True
+            for qb in range(nqb):
+                diag = (q_pos0 - k_pos0 + qb * block + block - 1) // block
+                lo, hi = max(0, diag - band + 1), min(nkb - 1, diag)
+                if hi >= lo:
+                    m[b, h, qb, lo:hi + 1] = True
+    return m
