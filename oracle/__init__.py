@@ -63,6 +63,8 @@ def _load():
                 ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
                 ctypes.c_double, ctypes.c_int, ctypes.c_double, vp, ctypes.c_int64,
                 ctypes.c_int64, ctypes.c_int64, vp, vp, vp]
+            lib.oracle_rope.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_double, vp, vp]
             lib.oracle_decode_positions.argtypes = [
                 vp, vp, vp, vp, vp, vp, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double,
@@ -210,6 +212,28 @@ def decode_positions(q, k_cache, v_cache, kv_len, q_pos, k_pos, *, Hq, Hkv, base
     if rc != 0:
         raise ValueError(f"oracle_decode_positions failed ({rc})")
     return out, lse
+
+
+def rope(x, positions, *, base, exact=False):
+    """RoPE of bf16 vectors x [n, H, D] (uint16 bits), token i at positions[i].
+
+    Pair p = dims (p, p + D/2) turns by positions[i] * base^(-2p/D) (WavePrune,
+    Original abstract).  Returns uint16 bf16 bits rounded to nearest-even from the
+    exact result, or with ``exact`` the float64 result itself.
+    """
+    lib = _load()
+    x = _u16(x)
+    n, H, D = x.shape
+    pos = np.ascontiguousarray(np.asarray(positions, dtype=np.int64).reshape(n))
+    if exact:
+        out = np.zeros((n, H, D), dtype=np.float64)
+        rc = lib.oracle_rope(x.ctypes.data, pos.ctypes.data, n, H, D, base, None, out.ctypes.data)
+    else:
+        out = np.zeros((n, H, D), dtype=np.uint16)
+        rc = lib.oracle_rope(x.ctypes.data, pos.ctypes.data, n, H, D, base, out.ctypes.data, None)
+    if rc != 0:
+        raise ValueError("oracle_rope: bad arguments")
+    return out
 
 
 def scores(qrow, keys, *, q_pos, k_pos0=0, base, alpha, g):

@@ -301,6 +301,72 @@ int oracle_decode_positions(const uint16_t *q, const uint16_t *k, const uint16_t
 }
 
 /*
+ * Round a double to bf16 bits, to nearest with ties to even, in one step from
+ * the exact value (no intermediate float).  Values below the smallest normal
+ * float go through a float first (their bf16 has fewer than 8 significant
+ * bits); the inputs here never produce them except exact zeros.
+ */
+static uint16_t double_to_bf16(double x)
+{
+    if (isnan(x)) return 0x7FC0;
+    const uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    if (a == 0.0) return sign;
+    if (a < ldexp(1.0, -126)) {
+        float f = (float)x;
+        uint32_t u;
+        memcpy(&u, &f, 4);
+        const uint32_t lsb = (u >> 16) & 1u;
+        u += 0x7FFFu + lsb;
+        return (uint16_t)(u >> 16);
+    }
+    int e;
+    const double m = frexp(a, &e);              /* a = m * 2^e, m in [0.5, 1) */
+    double r = nearbyint(ldexp(m, 8));          /* 8 significant bits, ties to even */
+    const double y = ldexp(r, e - 8);
+    if (y >= ldexp(1.0, 128)) return sign | 0x7F80;   /* overflow: inf */
+    const float f = (float)y;                   /* exact: y has 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFFu));
+}
+
+/*
+ * RoPE (WavePrune, Original abstract: each 2-D channel of a query or key is
+ * rotated at a channel-specific frequency, so logits depend on the position
+ * difference only).  Pair p = dims (p, p + D/2) turns by pos * theta_p with
+ * theta_p = base^(-2p/D) (the wavelength 2*pi*base^(2p/D) of the Length
+ * Extrapolation formula):
+ *   y_p       = x_p cos(a) - x_{p+D/2} sin(a)
+ *   y_{p+D/2} = x_p sin(a) + x_{p+D/2} cos(a),   a = pos * theta_p.
+ * x: bf16 [n, H, D] (token i at position pos[i]).  out_bf16 (optional): the
+ * result rounded to bf16; out_f64 (optional): the exact double result.
+ */
+int oracle_rope(const uint16_t *x, const int64_t *pos, int64_t n, int H, int D, double base,
+                uint16_t *out_bf16, double *out_f64)
+{
+    if (n < 0 || H <= 0 || D <= 0 || (D % 2) != 0 || !(base > 1.0)) return -1;
+    const int P = D / 2;
+    for (int64_t i = 0; i < n; ++i) {
+        for (int h = 0; h < H; ++h) {
+            const uint16_t *xr = x + (i * H + h) * (int64_t)D;
+            for (int p = 0; p < P; ++p) {
+                const double theta = pow(base, -(2.0 * p) / D);
+                const double a = (double)pos[i] * theta;
+                const double c = cos(a), sn = sin(a);
+                const double x0 = bf16_to_double(xr[p]), x1 = bf16_to_double(xr[p + P]);
+                const double y0 = x0 * c - x1 * sn;
+                const double y1 = x0 * sn + x1 * c;
+                const int64_t o = (i * H + h) * (int64_t)D;
+                if (out_f64) { out_f64[o + p] = y0; out_f64[o + p + P] = y1; }
+                if (out_bf16) { out_bf16[o + p] = double_to_bf16(y0); out_bf16[o + p + P] = double_to_bf16(y1); }
+            }
+        }
+    }
+    return 0;
+}
+
+/*
  * Windowed scores (before scale) of one query row against keys [0, nkeys):
  * used by tests that check the score formula itself on hand-worked inputs.
  * Causally excluded keys get NaN.

@@ -463,3 +463,71 @@ def test_block_mask_alpha_inf_is_masked_sdpa():
         np.testing.assert_allclose(out[n], want.numpy(), atol=1e-10)
         assert abs(lse[n] - float(torch.logsumexp(z[b, h, t], 0))) < 1e-10
     assert (~allowed.reshape(-1, Nk).any(1)).any()     # some rows are empty: the case is covered
+
+
+# ---------------------------------------------------------------------------
+# RoPE (WavePrune, Original abstract: 2-D channels rotated at channel-specific
+# frequencies; logits depend on the position difference only)
+# ---------------------------------------------------------------------------
+
+def _bf16_values(bits):
+    return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def test_rope_hand_cases():
+    # D = 2: one pair, theta_0 = 1 whatever the base
+    x = _bf16_bits(np.array([[[1.0, 0.0]], [[0.0, 1.0]]]))
+    y = oracle.rope(x, [1, 2], base=1e4, exact=True)
+    np.testing.assert_allclose(y[0, 0], [math.cos(1.0), math.sin(1.0)], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(y[1, 0], [-math.sin(2.0), math.cos(2.0)], rtol=0, atol=1e-15)
+    # D = 4, base 100: theta = (1, 0.1); position 10 turns pair 0 by 10 rad and pair 1 by 1 rad
+    x = _bf16_bits(np.array([[[1.0, 2.0, 0.0, 0.0]]]))
+    y = oracle.rope(x, [10], base=100.0, exact=True)
+    np.testing.assert_allclose(y[0, 0], [math.cos(10.0), 2 * math.cos(1.0), math.sin(10.0),
+                                         2 * math.sin(1.0)], rtol=0, atol=1e-14)
+
+
+def test_rope_position_zero_is_identity_and_pairs_are_half_split():
+    x = _rand((5, 3, 64), 201)
+    xb = inputs.bits(x)
+    assert np.array_equal(oracle.rope(xb, [0] * 5, base=1e4), xb)
+    e = np.zeros((1, 1, 16)); e[0, 0, 0] = 1.0
+    y = oracle.rope(_bf16_bits(e), [3], base=1e4, exact=True)[0, 0]
+    assert (y[[i for i in range(16) if i not in (0, 8)]] == 0).all()
+    assert y[0] != 0 and y[8] != 0
+
+
+def test_rope_preserves_pair_norms_and_depends_on_relative_position():
+    D, n = 64, 6
+    q = inputs.bits(_rand((n, 1, D), 202))
+    k = inputs.bits(_rand((n, 1, D), 203))
+    P = D // 2
+    rng = np.random.default_rng(4)
+    m = rng.integers(0, 100000, n)
+    nn = rng.integers(0, 100000, n)
+    shift = 123457
+    yq = oracle.rope(q, m, base=5e5, exact=True)
+    yk = oracle.rope(k, nn, base=5e5, exact=True)
+    yq2 = oracle.rope(q, m + shift, base=5e5, exact=True)
+    yk2 = oracle.rope(k, nn + shift, base=5e5, exact=True)
+    xq = _bf16_values(q)
+    np.testing.assert_allclose(yq[..., :P] ** 2 + yq[..., P:] ** 2,
+                               xq[..., :P] ** 2 + xq[..., P:] ** 2, rtol=1e-12)
+    # per pair: the rotated product depends on m - n only
+    s1 = yq[..., :P] * yk[..., :P] + yq[..., P:] * yk[..., P:]
+    s2 = yq2[..., :P] * yk2[..., :P] + yq2[..., P:] * yk2[..., P:]
+    np.testing.assert_allclose(s1, s2, rtol=0, atol=1e-9)
+
+
+def test_rope_rounds_to_nearest_bf16():
+    """Each bf16 output is the representable value nearest the exact result."""
+    x = inputs.bits(_rand((64, 4, 128), 204))
+    pos = np.arange(64) * 977
+    yb = oracle.rope(x, pos, base=1e6).astype(np.uint32)
+    ye = oracle.rope(x, pos, base=1e6, exact=True)
+    b = _bf16_values(yb)
+    up = _bf16_values((yb + 1) & 0xFFFF)       # next magnitude up (same sign)
+    dn = _bf16_values(np.where((yb & 0x7FFF) == 0, yb, yb - 1))
+    err = np.abs(ye - b)
+    assert (err <= np.abs(ye - up)).all() and (err <= np.abs(ye - dn)).all()
+    assert (np.sign(b) == np.sign(ye))[ye != 0].all()
