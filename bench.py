@@ -48,15 +48,15 @@ FLUSH_BYTES = 512 << 20
 # that kernel's sources at capture time: a changed kernel reports null until
 # it is captured again.
 NCU_TRAFFIC = {
-    # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.134912 MB read + 23.742208 MB written
-    ("qwen2.5-0.5b-32k", "78ae9ff5d51882a2"): 76134912 + 23742208,
-    # profiles/decode_split_kernel_llama3.2-3b-decode-32k.md: 536.942080 MB read + 7.402752 MB
+    # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.173824 MB read + 24.261376 MB written
+    ("qwen2.5-0.5b-32k", "47ecbacf478e94f7"): 76173824 + 24261376,
+    # profiles/decode_split_kernel_llama3.2-3b-decode-32k.md: 536.953600 MB read + 4.430336 MB
     # written for B=4, L=32768, scaled by the 16x keys x heads of the B=16, L=131072 call
-    ("llama3.2-3b-decode-128k", "fd8fb0cb72b0635b"): 16 * (536942080 + 7402752),
+    ("llama3.2-3b-decode-128k", "3731a04bcf2deee4"): 16 * (536953600 + 4430336),
 }
 
 KERNEL_SOURCES = {"prefill": ("prefill_kernel.cuh", "device_util.cuh"),
-                  "decode": ("decode_kernels.cuh", "device_util.cuh")}
+                  "decode": ("decode_kernels.cuh", "device_util.cuh", "rope_kernels.cuh")}
 
 
 def kernel_source_hash(kernel: str) -> str:
@@ -286,7 +286,7 @@ def gpu_arm(args):
         off_ms, _, _ = time_steps(step_off, args.warmup, max(3, args.steps // 4), flush, world)
         off_ms_step = off_ms / max(3, args.steps // 4)
         ms_step = total_ms / args.steps
-        masked = None
+        masked = rope_res = None
         if not args.only_primary:
             # the same call under a MInference-shaped block mask (vertical + slash tiles)
             mask = inputs.vertical_slash_mask(w.B, w.Hq, w.Nq, w.Nk, seed=rank, q_pos0=w.q_pos0,
@@ -318,6 +318,41 @@ def gpu_arm(args):
                 "mask": "vertical-slash: sink + 3 random key tiles per head, 16-tile diagonal band",
             }
             del words, mask
+            # the same prefill from pre-RoPE q and k: rotation pre-pass + attention,
+            # and the rotation kernel alone (HBM-bound: read and write q and k once)
+            ws_r = torch.empty(max(1, int(wp.lib().wpattn_prefill_rope_workspace_size(
+                w.B, w.Nq, w.Nk, w.Hq, w.Hkv, w.D))), dtype=torch.uint8, device=dev)
+            qr_buf = torch.empty_like(q)
+            kr_buf = torch.empty_like(k)
+
+            def step_rope_prefill():
+                wp.prefill_rope(q, k, v, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale,
+                                out=out, lse=lse, workspace=ws_r)
+
+            def step_rope_only():
+                wp.rope(q, base=w.base, pos0=w.q_pos0, out=qr_buf)
+                wp.rope(k, base=w.base, pos0=w.k_pos0, out=kr_buf)
+
+            n_r = max(3, args.steps // 2)
+            rp_ms, _, _ = time_steps(step_rope_prefill, args.warmup, n_r, flush, world)
+            ro_ms, ro_per, _ = time_steps(step_rope_only, args.warmup, n_r, flush, world)
+            if wp.device_status() != wp.OK:
+                raise RuntimeError("rope kernels status: not ok")
+            rope_bytes = 2 * 2 * (q.numel() + k.numel())
+            ro_gbs = rope_bytes / (statistics.mean(ro_per) * 1e-3) / 1e9
+            rope_res = {
+                "prefill_from_prerope": {"ms_per_step": round(rp_ms / n_r, 4),
+                                         "value": round(weak_scaling_value(eff, world, rp_ms / n_r) / 1e12, 2),
+                                         "unit": "TFLOP/s",
+                                         "overhead_vs_prefill": round((rp_ms / n_r) / ms_step - 1.0, 4)},
+                "rotation_kernels": {"ms_per_step": round(ro_ms / n_r, 4),
+                                     "roofline": {"bound": "hbm", "achieved": round(ro_gbs, 1),
+                                                  "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                                  "frac": round(ro_gbs / peaks["hbm_gbs"], 4),
+                                                  "traffic": None},
+                                     "bytes_per_step": rope_bytes},
+            }
+            del ws_r, qr_buf, kr_buf
         value = weak_scaling_value(eff, world, ms_step) / 1e12
         kernel_ms = statistics.mean(per)
         achieved = eff / (kernel_ms * 1e-3) / 1e12
@@ -343,7 +378,8 @@ def gpu_arm(args):
         })
         if masked is not None:
             result["block_sparse"] = masked
-            result["gpu_launches"] += max(3, args.steps // 2)
+            result["rope"] = rope_res
+            result["gpu_launches"] += 6 * max(3, args.steps // 2)
         # end to end through the public API with pinned host buffers
         qh = q.cpu().pin_memory()
         kh = k.cpu().pin_memory()

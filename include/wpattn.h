@@ -306,6 +306,63 @@ WPATTN_API int wpattn_decode_paged(const wpattn_window *w,
                   void *cuda_stream);
 
 /*
+ * RoPE rotation (WavePrune, Original abstract: each 2-D channel of a query or
+ * key turns at a channel-specific frequency).  Pair p = dims (p, p + D/2)
+ * turns by pos * theta_p, theta_p = rope_base^(-2p/D):
+ *   y_p = x_p cos - x_{p+D/2} sin,   y_{p+D/2} = x_p sin + x_{p+D/2} cos.
+ *   x, out: bf16 device [B, N, H, head_dim], 16-byte aligned; out may be x.
+ *   positions: device int32 [B, N] (4-byte aligned), or NULL: token t of
+ *              every sequence at pos0 + t (0 <= pos0 <= 2^40).
+ * The angle is reduced modulo 2 pi in double precision, its cosine and sine
+ * taken in float; each rotated value is rounded to bf16 (nearest even).
+ * head_dim in {64, 128} (else WPATTN_EUNSUPPORTED); rope_base > 1.
+ */
+WPATTN_API int wpattn_rope(const void *x, void *out, int32_t B, int32_t N, int32_t H,
+                  int32_t head_dim, int64_t pos0, const int32_t *positions, double rope_base,
+                  void *cuda_stream);
+
+/*
+ * Prefill from queries and keys that arrive before their RoPE rotation
+ * (v is never rotated).  Arguments and results as for wpattn_prefill; q and
+ * k are rotated with w->rope_base at their positions q_pos0 + t and
+ * k_pos0 + j (wpattn_rope), into the workspace, then attended.  The rotation
+ * is a pre-pass rather than part of the attention kernel's producer: there
+ * each key tile would be turned again by every query block that reads it,
+ * on the special-function pipe the attention's exponentials already fill.
+ *   workspace: device, 256-byte aligned, at least
+ *              wpattn_prefill_rope_workspace_size(...) bytes (else
+ *              WPATTN_EWORKSPACE); holds the rotated q and k.
+ */
+WPATTN_API int wpattn_prefill_rope(const wpattn_window *w,
+                  const void *q, const void *k, const void *v,
+                  void *out, float *lse,
+                  int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
+                  int64_t q_pos0, int64_t k_pos0, float softmax_scale,
+                  void *workspace, size_t workspace_bytes, void *cuda_stream);
+
+/* Workspace bytes wpattn_prefill_rope needs (0 on bad arguments). */
+WPATTN_API size_t wpattn_prefill_rope_workspace_size(int32_t B, int32_t Nq, int32_t Nk,
+                  int32_t Hq, int32_t Hkv, int32_t head_dim);
+
+/*
+ * Decode with the query before its RoPE rotation: the kernel turns q by its
+ * position (q_pos, kv_len - 1 by default) with w->rope_base as it loads it,
+ * rounding to bf16 exactly as wpattn_rope does, so the result equals
+ * wpattn_rope followed by wpattn_decode (or wpattn_decode_positions) bit for
+ * bit.  The cache holds rotated keys, as serving caches do.  q_pos_host,
+ * k_pos, k_pos_stride: both NULL, or both given as for
+ * wpattn_decode_positions.  Everything else as for wpattn_decode.
+ */
+WPATTN_API int wpattn_decode_rope(const wpattn_window *w,
+                  const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *kv_len_host, int64_t Lmax,
+                  const int32_t *q_pos_host, const int32_t *k_pos, int64_t k_pos_stride,
+                  int32_t B, int32_t Hq, int32_t Hkv, float softmax_scale,
+                  void *out, float *lse,
+                  void *workspace, size_t workspace_bytes,
+                  void *cuda_stream);
+
+/*
  * Synchronises `cuda_stream`, then reads and clears the current device's
  * kernel status word.  Returns WPATTN_OK, WPATTN_ETIMEOUT (a kernel gave up a
  * bounded wait; its outputs are undefined), WPATTN_EINDEX (a kernel met an

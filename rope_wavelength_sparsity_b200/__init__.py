@@ -9,7 +9,8 @@ exception is raised.
 
 Entry points (same names as the C ABI, without the ``wpattn_`` prefix):
 ``prefill``, ``decode``, ``decode_pairmajor``, ``kcache_to_pairmajor``,
-``decode_positions``, ``decode_paged``, ``prefill_masked``, ``pack_block_mask``,
+``decode_positions``, ``decode_paged``, ``prefill_masked``, ``pack_block_mask``, ``rope``,
+``prefill_rope``, ``decode_rope``,
 ``decode_workspace_size``, ``decode_noalloc``, ``pruned_fraction``,
 ``thresholds``, ``device_status``.
 """
@@ -71,6 +72,11 @@ def lib() -> ctypes.CDLL:
         L.wpattn_prefill_masked.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64,
                                             i64, f32, vp, i32, vp]
         L.wpattn_pack_block_mask.argtypes = [vp, vp, i64, i32, i32, vp]
+        L.wpattn_rope.argtypes = [vp, vp, i32, i32, i32, i32, i64, vp, ctypes.c_double, vp]
+        L.wpattn_prefill_rope.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64, i64,
+                                          f32, vp, ctypes.c_size_t, vp]
+        L.wpattn_prefill_rope_workspace_size.restype = ctypes.c_size_t
+        L.wpattn_prefill_rope_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         L.wpattn_decode_workspace_size.restype = ctypes.c_size_t
         L.wpattn_decode_workspace_size.argtypes = [wp, i32, i32, i32, i64]
         L.wpattn_decode.argtypes = [wp, vp, vp, vp, ctypes.POINTER(ctypes.c_int32), i64, i32, i32,
@@ -80,6 +86,7 @@ def lib() -> ctypes.CDLL:
         i32p = ctypes.POINTER(ctypes.c_int32)
         L.wpattn_decode_positions.argtypes = [wp, vp, vp, vp, i32p, i64, i32p, vp, i64, i32, i32,
                                               i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
+        L.wpattn_decode_rope.argtypes = L.wpattn_decode_positions.argtypes
         L.wpattn_decode_paged.argtypes = [wp, vp, vp, vp, i32, i32, vp, i32, i32p, i32p, vp, i64,
                                           i32, i32, i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
         L.wpattn_device_status.argtypes = [vp]
@@ -215,6 +222,46 @@ def prefill_masked(q, k, v, block_mask, w: Window, *, q_pos0: int = 0, k_pos0: i
     return out, lse
 
 
+def rope(x, *, base: float, pos0: int = 0, positions=None, out=None, stream=None):
+    """RoPE of x [B, N, H, D] (bf16 CUDA): pair p = dims (p, p + D/2) turns by
+    pos * base^(-2p/D), token t of each sequence at pos0 + t or positions[b, t]
+    (int32 CUDA [B, N]).  Rounded to bf16; ``out`` may be x."""
+    import torch
+    B, N, H, D = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().wpattn_rope(_dev_tensor(x, "x"), _dev_tensor(out, "out"), B, N, H, D, pos0,
+                             _int32_dev(positions, "positions") if positions is not None else None,
+                             float(base), _stream_ptr(stream)), "wpattn_rope")
+    return out
+
+
+def prefill_rope(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0,
+                 scale: float | None = None, out=None, lse=None, want_lse: bool = True,
+                 workspace=None, stream=None):
+    """``prefill`` from q and k before their RoPE rotation (rotated with w.rope_base at
+    q_pos0 + t and k_pos0 + j into a workspace first)."""
+    import torch
+    B, Nq, Hq, D = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    if workspace is None:
+        n = int(lib().wpattn_prefill_rope_workspace_size(B, Nq, Nk, Hq, Hkv, D))
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = lib().wpattn_prefill_rope(ctypes.byref(w._c()), _dev_tensor(q, "q"), _dev_tensor(k, "k"),
+                                   _dev_tensor(v, "v"), _dev_tensor(out, "out"),
+                                   ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+                                   B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0,
+                                   float(scale) if scale else 0.0,
+                                   ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                   _stream_ptr(stream))
+    _check(rc, "wpattn_prefill_rope")
+    return out, lse
+
+
 def decode_workspace_size(w: Window, B: int, Hq: int, Hkv: int, max_kv_len: int) -> int:
     return int(lib().wpattn_decode_workspace_size(ctypes.byref(w._c()), B, Hq, Hkv, max_kv_len))
 
@@ -332,6 +379,29 @@ def decode_positions(q, k_cache, v_cache, kv_len, q_pos, k_pos, w: Window, *,
                                        ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
                                        _stream_ptr(stream))
     _check(rc, "wpattn_decode_positions")
+    return out, lse
+
+
+def decode_rope(q, k_cache, v_cache, kv_len, w: Window, *, q_pos=None, k_pos=None,
+                scale: float | None = None, out=None, lse=None, want_lse: bool = True,
+                workspace=None, stream=None):
+    """``decode`` (or ``decode_positions``) with q before its RoPE rotation; the kernel
+    turns q by its position with w.rope_base as it loads it."""
+    B, Hq, D = q.shape
+    L, Hkv = k_cache.shape[1], k_cache.shape[2]
+    kvl = (ctypes.c_int32 * B)(*[int(x) for x in kv_len])
+    qp = (ctypes.c_int32 * B)(*[int(x) for x in q_pos]) if q_pos is not None else None
+    out, lse, workspace = _decode_outputs(q, w, B, Hq, Hkv, L, out, lse, want_lse, workspace)
+    rc = lib().wpattn_decode_rope(ctypes.byref(w._c()), _dev_tensor(q, "q"),
+                                  _dev_tensor(k_cache, "k_cache"), _dev_tensor(v_cache, "v_cache"),
+                                  kvl, L, qp,
+                                  _int32_dev(k_pos, "k_pos") if k_pos is not None else None,
+                                  k_pos.stride(0) if k_pos is not None else 0, B, Hq, Hkv,
+                                  float(scale) if scale else 0.0, _dev_tensor(out, "out"),
+                                  ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+                                  ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                  _stream_ptr(stream))
+    _check(rc, "wpattn_decode_rope")
     return out, lse
 
 

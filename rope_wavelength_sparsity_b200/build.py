@@ -19,7 +19,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libwpattn.so")
 SOURCES = ["api.cu", "planner.cpp"]
-DEPS = SOURCES + ["device_util.cuh", "decode_kernels.cuh", "prefill_kernel.cuh", "planner.h"]
+DEPS = SOURCES + ["device_util.cuh", "decode_kernels.cuh", "prefill_kernel.cuh", "rope_kernels.cuh",
+                  "planner.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

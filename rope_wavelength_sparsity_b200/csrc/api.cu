@@ -15,6 +15,7 @@
 #include "device_util.cuh"
 #include "decode_kernels.cuh"
 #include "prefill_kernel.cuh"
+#include "rope_kernels.cuh"
 
 namespace wpattn {
 namespace {
@@ -101,6 +102,33 @@ int encode_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? WPATTN_OK : WPATTN_ECUDA;
+}
+
+// theta_p = base^(-2p/D), the RoPE angle per position of pair p
+void rope_thetas(double base, int D, double* theta) {
+  for (int p = 0; p < 64; ++p)
+    theta[p] = p < D / 2 ? std::pow(base, -static_cast<double>(2 * p) / static_cast<double>(D)) : 0.0;
+}
+
+int launch_rope(const void* x, void* out, int64_t B, int64_t N, int H, int D, int64_t pos0,
+                const int32_t* pos, double base, int num_sms, cudaStream_t st) {
+  RopeParams rp;
+  std::memset(&rp, 0, sizeof rp);
+  rp.x = static_cast<const uint16_t*>(x);
+  rp.out = static_cast<uint16_t*>(out);
+  rp.pos = pos;
+  rp.pos0 = pos0;
+  rp.B = B;
+  rp.N = N;
+  rp.H = H;
+  rope_thetas(base, D, rp.theta);
+  const uint64_t n = static_cast<uint64_t>(B) * N * (D / 16);  // (token, 8-pair chunk) items
+  if (n == 0) return WPATTN_OK;
+  const uint64_t want = (n + 255) / 256;
+  const unsigned grid = static_cast<unsigned>(std::min<uint64_t>(want, static_cast<uint64_t>(num_sms) * 8));
+  if (D == 64) rope_kernel<64><<<grid, 256, 0, st>>>(rp);
+  else rope_kernel<128><<<grid, 256, 0, st>>>(rp);
+  return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
 template <int D, bool G8, bool MASK>
@@ -371,6 +399,65 @@ int wpattn_pack_block_mask(const uint8_t* mask, uint32_t* words, int64_t rows, i
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
+int wpattn_rope(const void* x, void* out, int32_t B, int32_t N, int32_t H, int32_t head_dim,
+                int64_t pos0, const int32_t* positions, double rope_base, void* cuda_stream) {
+  if (B < 0 || N < 0 || H <= 0) return WPATTN_EINVAL;
+  if (!(rope_base > 1.0) || std::isinf(rope_base)) return WPATTN_EINVAL;
+  if (head_dim != 64 && head_dim != 128) return WPATTN_EUNSUPPORTED;
+  if (B == 0 || N == 0) return WPATTN_OK;
+  if (!x || !out || !aligned16(x) || !aligned16(out)) return WPATTN_EINVAL;
+  if (positions && (reinterpret_cast<uintptr_t>(positions) & 3u) != 0) return WPATTN_EINVAL;
+  if (!positions && (pos0 < 0 || pos0 > (int64_t(1) << 40))) return WPATTN_EINVAL;
+  DeviceInfo* dev = nullptr;
+  int rc;
+  if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
+  return launch_rope(x, out, B, N, H, head_dim, pos0, positions, rope_base, dev->num_sms,
+                     static_cast<cudaStream_t>(cuda_stream));
+}
+
+size_t wpattn_prefill_rope_workspace_size(int32_t B, int32_t Nq, int32_t Nk, int32_t Hq,
+                                          int32_t Hkv, int32_t head_dim) {
+  if (B < 0 || Nq < 0 || Nk < 0 || Hq <= 0 || Hkv <= 0 || head_dim <= 0) return 0;
+  const size_t qb = static_cast<size_t>(B) * Nq * Hq * head_dim * 2;
+  const size_t kb = static_cast<size_t>(B) * Nk * Hkv * head_dim * 2;
+  return ((qb + 255) / 256) * 256 + kb;
+}
+
+int wpattn_prefill_rope(const wpattn_window* w, const void* q, const void* k, const void* v,
+                        void* out, float* lse, int32_t B, int32_t Nq, int32_t Nk, int32_t Hq,
+                        int32_t Hkv, int64_t q_pos0, int64_t k_pos0, float softmax_scale,
+                        void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  WindowPlan plan;
+  int rc = make_window_plan(w, &plan);
+  if (rc != WPATTN_OK) return rc;
+  if (B < 0 || Nq < 0 || Nk < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0) return WPATTN_EINVAL;
+  if (plan.D != 64 && plan.D != 128) return WPATTN_EUNSUPPORTED;
+  if (B == 0 || Nq == 0) return WPATTN_OK;
+  const size_t need = wpattn_prefill_rope_workspace_size(B, Nq, Nk, Hq, Hkv, plan.D);
+  if (!workspace || workspace_bytes < need) return WPATTN_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return WPATTN_EINVAL;
+  if (!q || !aligned16(q) || (Nk > 0 && (!k || !aligned16(k)))) return WPATTN_EINVAL;
+  if (q_pos0 < 0 || k_pos0 < 0 || q_pos0 > (int64_t(1) << 40) || k_pos0 > (int64_t(1) << 40))
+    return WPATTN_EINVAL;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* qr = ws;
+  void* kr = ws + ((static_cast<size_t>(B) * Nq * Hq * plan.D * 2 + 255) / 256) * 256;
+  DeviceInfo* dev = nullptr;
+  if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  // the rotations are a pre-pass: each key row is turned once, not once per
+  // query block that reads it, and off the MUFU pipe the attention needs
+  if ((rc = launch_rope(q, qr, B, Nq, Hq, plan.D, q_pos0, nullptr, w->rope_base, dev->num_sms, st)) !=
+      WPATTN_OK)
+    return rc;
+  if (Nk > 0 &&
+      (rc = launch_rope(k, kr, B, Nk, Hkv, plan.D, k_pos0, nullptr, w->rope_base, dev->num_sms, st)) !=
+          WPATTN_OK)
+    return rc;
+  return prefill_impl(w, qr, kr, v, out, lse, B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0, softmax_scale,
+                      nullptr, 0, cuda_stream);
+}
+
 size_t wpattn_decode_workspace_size(const wpattn_window* w, int32_t B, int32_t Hq, int32_t Hkv,
                                     int64_t max_kv_len) {
   WindowPlan plan;
@@ -393,6 +480,7 @@ struct DecodeLayout {
   const int32_t* q_pos_host = nullptr;    // host [B]
   const int32_t* k_pos = nullptr;         // device [B, k_pos_stride]
   int64_t k_pos_stride = 0;
+  bool rope_q = false;                    // q arrives before its RoPE rotation
 };
 
 int decode_impl(const wpattn_window* w, const void* q, const void* k_cache, const void* v_cache,
@@ -453,6 +541,8 @@ int decode_impl(const wpattn_window* w, const void* q, const void* k_cache, cons
   prm.num_pages = lay.num_pages;
   prm.k_pos = lay.k_pos;
   prm.k_pos_stride = lay.k_pos_stride;
+  prm.rope_q = lay.rope_q ? 1 : 0;
+  if (lay.rope_q) rope_thetas(w->rope_base, plan.D, prm.theta);
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   if (plan.D == 64) return launch_decode<64>(prm, gc, lay.pm, st);
   return launch_decode<128>(prm, gc, lay.pm, st);
@@ -488,6 +578,21 @@ int wpattn_decode_positions(const wpattn_window* w, const void* q, const void* k
                             void* cuda_stream) {
   if (!q_pos_host || !k_pos) return WPATTN_EINVAL;
   DecodeLayout lay;
+  lay.q_pos_host = q_pos_host;
+  lay.k_pos = k_pos;
+  lay.k_pos_stride = k_pos_stride;
+  return decode_impl(w, q, k_cache, v_cache, kv_len_host, Lmax, B, Hq, Hkv, softmax_scale, out, lse,
+                     workspace, workspace_bytes, cuda_stream, lay);
+}
+
+int wpattn_decode_rope(const wpattn_window* w, const void* q, const void* k_cache,
+                       const void* v_cache, const int32_t* kv_len_host, int64_t Lmax,
+                       const int32_t* q_pos_host, const int32_t* k_pos, int64_t k_pos_stride,
+                       int32_t B, int32_t Hq, int32_t Hkv, float softmax_scale, void* out,
+                       float* lse, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  if ((q_pos_host == nullptr) != (k_pos == nullptr)) return WPATTN_EINVAL;
+  DecodeLayout lay;
+  lay.rope_q = true;
   lay.q_pos_host = q_pos_host;
   lay.k_pos = k_pos;
   lay.k_pos_stride = k_pos_stride;

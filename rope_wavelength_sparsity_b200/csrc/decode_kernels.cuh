@@ -16,6 +16,7 @@
 #pragma once
 
 #include "device_util.cuh"
+#include "rope_kernels.cuh"
 
 namespace wpattn {
 
@@ -46,6 +47,10 @@ struct DecodeParams {
   int64_t k_pos_stride;
   int kv_len[kDecodeMaxB];
   int q_pos[kDecodeMaxB];  // position of each sequence's query
+  // rope_q: q arrives before its RoPE rotation; the kernel turns it by
+  // q_pos * theta_p (rounded to bf16, as a model would store it) on load
+  int rope_q;
+  double theta[64];
 };
 
 __device__ __forceinline__ uint4 ldg_stream(const void* ptr) {
@@ -170,9 +175,24 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     fence_barrier_init();
   }
   if (threadIdx.x < 64) sT[threadIdx.x] = p.T[threadIdx.x];
-  for (int idx = threadIdx.x; idx < GC * D; idx += blockDim.x) {
-    const int hh = idx / D, e = idx % D;
-    qs[idx] = hh < nh ? bf16lo_to_f32(p.q[((size_t)b * p.Hq + h0 + hh) * D + e]) * p.scale_log2 : 0.f;
+  if (p.rope_q) {
+    for (int idx = threadIdx.x; idx < GC * P; idx += blockDim.x) {
+      const int hh = idx / P, pp = idx % P;
+      float y0 = 0.f, y1 = 0.f;
+      if (hh < nh) {
+        const uint16_t* qr = p.q + ((size_t)b * p.Hq + h0 + hh) * D;
+        float c, sn;
+        rope_cos_sin(qpos, p.theta[pp], c, sn);
+        rope_pair_bf16(bf16lo_to_f32(qr[pp]), bf16lo_to_f32(qr[pp + P]), c, sn, y0, y1);
+      }
+      qs[hh * D + pp] = y0 * p.scale_log2;
+      qs[hh * D + pp + P] = y1 * p.scale_log2;
+    }
+  } else {
+    for (int idx = threadIdx.x; idx < GC * D; idx += blockDim.x) {
+      const int hh = idx / D, e = idx % D;
+      qs[idx] = hh < nh ? bf16lo_to_f32(p.q[((size_t)b * p.Hq + h0 + hh) * D + e]) * p.scale_log2 : 0.f;
+    }
   }
   __syncthreads();
 
