@@ -65,6 +65,11 @@ def _load():
                 ctypes.c_int64, ctypes.c_int64, vp, vp, vp]
             lib.oracle_rope.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_double, vp, vp]
+            lib.oracle_attention_positions.argtypes = [
+                vp, vp, vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, vp, ctypes.c_int64, vp, ctypes.c_int64,
+                ctypes.c_double, ctypes.c_double, ctypes.c_int, ctypes.c_double, ctypes.c_int64,
+                vp, vp, vp]
             lib.oracle_decode_positions.argtypes = [
                 vp, vp, vp, vp, vp, vp, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double,
@@ -156,6 +161,32 @@ def attention_rows_masked(q, k, v, block_mask, *, Hq, Hkv, q_pos0=0, k_pos0=0, b
         out.ctypes.data, lse.ctypes.data)
     if rc != 0:
         raise ValueError(f"oracle_attention_rows_masked failed ({rc})")
+    return out, lse
+
+
+def attention_positions(q, k, v, q_pos, k_pos, *, Hq, Hkv, base, alpha, g, scale, rows):
+    """Prefill rows with explicit positions: query t of sequence b at q_pos[b, t], key j at
+    k_pos[b, j] (int arrays [B, >= Nq] and [B, >= Nk]); otherwise as ``attention_rows``.
+    ATFlash Abstract: the window depends on the relative position only.
+    """
+    lib = _load()
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    B, Nq, _, D = q.shape
+    Nk = k.shape[1]
+    qp = np.ascontiguousarray(np.asarray(q_pos, dtype=np.int64).reshape(B, -1))
+    kp = np.ascontiguousarray(np.asarray(k_pos, dtype=np.int64).reshape(B, -1))
+    if qp.shape[1] < Nq or kp.shape[1] < Nk:
+        raise ValueError("position arrays shorter than the sequences")
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    n = rows.shape[0]
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros(n, dtype=np.float64)
+    rc = lib.oracle_attention_positions(
+        q.ctypes.data, k.ctypes.data, v.ctypes.data, B, Nq, Nk, Hq, Hkv, D, qp.ctypes.data,
+        qp.shape[1], kp.ctypes.data, kp.shape[1], base, alpha, g, scale, n, rows.ctypes.data,
+        out.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_attention_positions failed ({rc})")
     return out, lse
 
 

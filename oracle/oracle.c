@@ -232,6 +232,68 @@ int oracle_attention_rows_masked(const uint16_t *q, const uint16_t *k, const uin
 }
 
 /*
+ * Prefill rows with explicit positions: query t of sequence b at
+ * q_pos[b * q_stride + t], key j at k_pos[b * k_stride + j].  The same
+ * definition as oracle_attention_rows with d = q_pos - k_pos; a key after its
+ * query is excluded; a row with no key left gets out = 0, lse = -inf.
+ * rows: nrows triples (b, h, t).
+ */
+int oracle_attention_positions(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                               int B, int64_t Nq, int64_t Nk, int Hq, int Hkv, int D,
+                               const int64_t *q_pos, int64_t q_stride,
+                               const int64_t *k_pos, int64_t k_stride,
+                               double base, double alpha, int g, double scale,
+                               int64_t nrows, const int64_t *rows, double *out, double *lse)
+{
+    if (Hkv <= 0 || Hq <= 0 || (Hq % Hkv) != 0 || B <= 0 || D <= 0) return -1;
+    const int P = D / 2;
+    int64_t T[4096];
+    if (oracle_thresholds(D, base, alpha, g, T, NULL) != 0) return -1;
+    const int group = Hq / Hkv;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+    if (!s) return -2;
+    for (int64_t r = 0; r < nrows; ++r) {
+        const int64_t b = rows[3 * r], h = rows[3 * r + 1], t = rows[3 * r + 2];
+        if (b < 0 || b >= B || h < 0 || h >= Hq || t < 0 || t >= Nq) { free(s); return -1; }
+        const int64_t kvh = h / group;
+        const int64_t qpos = q_pos[b * q_stride + t];
+        const uint16_t *qr = q + ((b * Nq + t) * Hq + h) * (int64_t)D;
+        double m = -INFINITY;
+        int64_t used = 0;
+        for (int64_t j = 0; j < Nk; ++j) {
+            const int64_t kpos = k_pos[b * k_stride + j];
+            if (kpos > qpos) { s[j] = NAN; continue; }
+            const int64_t d = qpos - kpos;
+            const uint16_t *kr = k + ((b * Nk + j) * Hkv + kvh) * (int64_t)D;
+            double acc = 0.0;
+            for (int p = 0; p < P; ++p) {
+                if (d > T[p]) continue; /* pruned term: contributes 0 */
+                acc += bf16_to_double(qr[p]) * bf16_to_double(kr[p]);
+                acc += bf16_to_double(qr[p + P]) * bf16_to_double(kr[p + P]);
+            }
+            s[j] = scale * acc;
+            if (s[j] > m) m = s[j];
+            ++used;
+        }
+        double *o = out + r * D;
+        for (int e = 0; e < D; ++e) o[e] = 0.0;
+        if (used == 0) { lse[r] = -INFINITY; continue; }
+        double l = 0.0;
+        for (int64_t j = 0; j < Nk; ++j) {
+            if (isnan(s[j])) continue;
+            const double w = exp(s[j] - m);
+            l += w;
+            const uint16_t *vr = v + ((b * Nk + j) * Hkv + kvh) * (int64_t)D;
+            for (int e = 0; e < D; ++e) o[e] += w * bf16_to_double(vr[e]);
+        }
+        for (int e = 0; e < D; ++e) o[e] /= l;
+        lse[r] = m + log(l);
+    }
+    free(s);
+    return 0;
+}
+
+/*
  * Decode with explicit positions (a serving cache whose keys are not at
  * positions 0..n-1: evicted or reordered tokens): sequence b has one query at
  * position q_pos[b] and keys j < kv_len[b] at positions

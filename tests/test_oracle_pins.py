@@ -531,3 +531,70 @@ def test_rope_rounds_to_nearest_bf16():
     err = np.abs(ye - b)
     assert (err <= np.abs(ye - up)).all() and (err <= np.abs(ye - dn)).all()
     assert (np.sign(b) == np.sign(ye))[ye != 0].all()
+
+
+# ---------------------------------------------------------------------------
+# prefill with explicit per-token positions (ATFlash Abstract: the window is a
+# function of the relative position)
+# ---------------------------------------------------------------------------
+
+def test_prefill_positions_contiguous_equal_attention_rows():
+    B, Nq, Nk, Hq, Hkv, D, q0, k0 = 2, 30, 50, 2, 1, 16, 40, 17
+    q = _rand((B, Nq, Hq, D), 301)
+    k = _rand((B, Nk, Hkv, D), 302)
+    v = _rand((B, Nk, Hkv, D), 303)
+    rows = [(b, h, t) for b in range(B) for h in range(Hq) for t in range(Nq)]
+    kw = dict(Hq=Hq, Hkv=Hkv, base=100.0, alpha=1.0, g=1, scale=0.3, rows=rows)
+    a = oracle.attention_rows(inputs.bits(q), inputs.bits(k), inputs.bits(v), q_pos0=q0, k_pos0=k0, **kw)
+    qp = np.tile(q0 + np.arange(Nq), (B, 1))
+    kp = np.tile(k0 + np.arange(Nk), (B, 1))
+    b = oracle.attention_positions(inputs.bits(q), inputs.bits(k), inputs.bits(v), qp, kp, **kw)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_prefill_positions_hand_case():
+    """Query (1, 2, 3, 4) at position 50 (D = 4, base 100, T = (6, 62)); keys at 0, 45, 50 and 51:
+    d = 50 (pair 0 pruned: s = 2 + 4 = 6 for k = (1, 1, 1, 1)), d = 5 (both kept: s = 1 for
+    k = (1, 0, 0, 0)), d = 0 (s = 0 for k = 0), d = -1 (future: left out)."""
+    q = _bf16_bits(np.array([1.0, 2.0, 3.0, 4.0]).reshape(1, 1, 1, 4))
+    kk = np.zeros((1, 4, 1, 4))
+    vv = np.eye(4).reshape(1, 4, 1, 4)
+    kk[0, 0, 0] = [1.0, 1.0, 1.0, 1.0]
+    kk[0, 1, 0] = [1.0, 0.0, 0.0, 0.0]
+    kk[0, 3, 0] = [9.0, 9.0, 9.0, 9.0]
+    out, lse = oracle.attention_positions(q, _bf16_bits(kk), _bf16_bits(vv), [[50]],
+                                          [[0, 45, 50, 51]], Hq=1, Hkv=1, base=100.0, alpha=1.0,
+                                          g=1, scale=1.0, rows=[(0, 0, 0)])
+    z = math.exp(6.0) + math.e + 1.0
+    np.testing.assert_allclose(out[0], [math.exp(6.0) / z, math.e / z, 1.0 / z, 0.0], rtol=0,
+                               atol=1e-12)
+    assert abs(lse[0] - math.log(z)) < 1e-12
+
+
+def test_prefill_positions_alpha_inf_is_masked_sdpa_and_shift_invariant():
+    B, Nq, Nk, Hq, Hkv, D = 2, 24, 40, 2, 2, 16
+    q = _rand((B, Nq, Hq, D), 304)
+    k = _rand((B, Nk, Hkv, D), 305)
+    v = _rand((B, Nk, Hkv, D), 306)
+    rng = np.random.default_rng(8)
+    kp = np.sort(rng.integers(0, 300, (B, Nk)), axis=1)
+    qp = np.sort(rng.integers(0, 300, (B, Nq)), axis=1)
+    rows = [(b, h, t) for b in range(B) for h in range(Hq) for t in range(Nq)]
+    out, lse = oracle.attention_positions(inputs.bits(q), inputs.bits(k), inputs.bits(v), qp, kp,
+                                          Hq=Hq, Hkv=Hkv, base=1e4, alpha=float("inf"), g=1,
+                                          scale=0.25, rows=rows)
+    for n, (b, h, t) in enumerate(rows):
+        allowed = torch.tensor(kp[b] <= qp[b, t])
+        if not allowed.any():
+            assert lse[n] == -math.inf and (out[n] == 0).all()
+            continue
+        z = 0.25 * (k[b, :, h].double() @ q[b, t, h].double())
+        z = torch.where(allowed, z, torch.tensor(-math.inf, dtype=torch.float64))
+        np.testing.assert_allclose(out[n], (torch.softmax(z, 0) @ v[b, :, h].double()).numpy(),
+                                   atol=1e-10)
+    kw = dict(Hq=Hq, Hkv=Hkv, base=1e4, alpha=1.0, g=8, scale=0.25, rows=rows)
+    a = oracle.attention_positions(inputs.bits(q), inputs.bits(k), inputs.bits(v), qp, kp, **kw)
+    b2 = oracle.attention_positions(inputs.bits(q), inputs.bits(k), inputs.bits(v), qp + 99991,
+                                    kp + 99991, **kw)
+    np.testing.assert_array_equal(a[0], b2[0])
