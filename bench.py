@@ -286,7 +286,7 @@ def gpu_arm(args):
         off_ms, _, _ = time_steps(step_off, args.warmup, max(3, args.steps // 4), flush, world)
         off_ms_step = off_ms / max(3, args.steps // 4)
         ms_step = total_ms / args.steps
-        masked = rope_res = None
+        masked = rope_res = positions_res = None
         if not args.only_primary:
             # the same call under a MInference-shaped block mask (vertical + slash tiles)
             mask = inputs.vertical_slash_mask(w.B, w.Hq, w.Nq, w.Nk, seed=rank, q_pos0=w.q_pos0,
@@ -353,6 +353,28 @@ def gpu_arm(args):
                                      "bytes_per_step": rope_bytes},
             }
             del ws_r, qr_buf, kr_buf
+            # the same prefill through the explicit-positions kernel, given the workload's
+            # own contiguous positions (same work; the cost of the searched column ranges)
+            qp = (w.q_pos0 + torch.arange(w.Nq, dtype=torch.int32, device=dev)).repeat(w.B, 1)
+            kp = (w.k_pos0 + torch.arange(w.Nk, dtype=torch.int32, device=dev)).repeat(w.B, 1)
+
+            def step_pos():
+                wp.prefill_positions(q, k, v, qp, kp, win, scale=w.scale, out=out, lse=lse)
+
+            pos_ms, pos_per, _ = time_steps(step_pos, args.warmup, n_r, flush, world)
+            if wp.device_status() != wp.OK:
+                raise RuntimeError("positions prefill status: not ok")
+            pos_ach = eff / (statistics.mean(pos_per) * 1e-3) / 1e12
+            positions_res = {
+                "value": round(weak_scaling_value(eff, world, pos_ms / n_r) / 1e12, 2),
+                "unit": "TFLOP/s", "ms_per_step": round(pos_ms / n_r, 4),
+                "roofline": {"bound": "tensor", "achieved": round(pos_ach, 2),
+                             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": round(pos_ach / peaks["bf16_tflops"], 4), "traffic": None},
+                "slowdown_vs_plain": round((pos_ms / n_r) / ms_step, 3),
+                "positions": "the workload's contiguous positions passed as int32 arrays",
+            }
+            del qp, kp
         value = weak_scaling_value(eff, world, ms_step) / 1e12
         kernel_ms = statistics.mean(per)
         achieved = eff / (kernel_ms * 1e-3) / 1e12
@@ -379,7 +401,8 @@ def gpu_arm(args):
         if masked is not None:
             result["block_sparse"] = masked
             result["rope"] = rope_res
-            result["gpu_launches"] += 6 * max(3, args.steps // 2)
+            result["explicit_positions"] = positions_res
+            result["gpu_launches"] += 7 * max(3, args.steps // 2)
         # end to end through the public API with pinned host buffers
         qh = q.cpu().pin_memory()
         kh = k.cpu().pin_memory()

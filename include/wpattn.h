@@ -143,6 +143,29 @@ WPATTN_API int wpattn_prefill_masked(const wpattn_window *w,
                   void *cuda_stream);
 
 /*
+ * Prefill with explicit per-token positions (ATFlash Abstract: the window is a
+ * function of the query-key distance alone): query t of sequence b sits at
+ * q_pos[b * q_pos_stride + t], key j at k_pos[b * k_pos_stride + j], for
+ * caches that dropped tokens, chunks with gaps, or packed inputs whose
+ * positions do not follow the index.  A key after its query is left out;
+ * otherwise arguments and results as for wpattn_prefill.
+ *   q_pos: device int32, 4-byte aligned, q_pos_stride >= Nq.
+ *   k_pos: device int32, 16-byte aligned, k_pos_stride a multiple of 4 and
+ *          >= Nk rounded up to a multiple of 128 (the kernel copies key
+ *          positions 128 at a time; entries past Nk are read, never used).
+ * Positions must be non-decreasing along each sequence and in
+ * [0, 2^31 - 1); otherwise the output is undefined (no access leaves the
+ * arrays).  Bad strides or alignment give WPATTN_EINVAL.
+ */
+WPATTN_API int wpattn_prefill_positions(const wpattn_window *w,
+                  const void *q, const void *k, const void *v,
+                  void *out, float *lse,
+                  int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
+                  const int32_t *q_pos, int64_t q_pos_stride,
+                  const int32_t *k_pos, int64_t k_pos_stride,
+                  float softmax_scale, void *cuda_stream);
+
+/*
  * Pack a byte block mask (device uint8 [rows, nkb], nonzero = attended) into
  * the bit rows wpattn_prefill_masked reads (device uint32 [rows, mask_words],
  * caller-allocated, 4-byte aligned; bit kb % 32 of word kb / 32, zero past

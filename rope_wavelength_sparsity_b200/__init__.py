@@ -10,7 +10,7 @@ exception is raised.
 Entry points (same names as the C ABI, without the ``wpattn_`` prefix):
 ``prefill``, ``decode``, ``decode_pairmajor``, ``kcache_to_pairmajor``,
 ``decode_positions``, ``decode_paged``, ``prefill_masked``, ``pack_block_mask``, ``rope``,
-``prefill_rope``, ``decode_rope``,
+``prefill_rope``, ``decode_rope``, ``prefill_positions``,
 ``decode_workspace_size``, ``decode_noalloc``, ``pruned_fraction``,
 ``thresholds``, ``device_status``.
 """
@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.wpattn_prefill_masked.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64,
                                             i64, f32, vp, i32, vp]
         L.wpattn_pack_block_mask.argtypes = [vp, vp, i64, i32, i32, vp]
+        L.wpattn_prefill_positions.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp,
+                                               i64, vp, i64, f32, vp]
         L.wpattn_rope.argtypes = [vp, vp, i32, i32, i32, i32, i64, vp, ctypes.c_double, vp]
         L.wpattn_prefill_rope.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64, i64,
                                           f32, vp, ctypes.c_size_t, vp]
@@ -259,6 +261,37 @@ def prefill_rope(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0,
                                    ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
                                    _stream_ptr(stream))
     _check(rc, "wpattn_prefill_rope")
+    return out, lse
+
+
+def prefill_positions(q, k, v, q_pos, k_pos, w: Window, *, scale: float | None = None, out=None,
+                      lse=None, want_lse: bool = True, stream=None):
+    """``prefill`` with explicit per-token positions: q_pos int32 CUDA [B, >= Nq], k_pos
+    int32 CUDA [B, >= Nk], non-decreasing along each sequence.  k_pos is copied into a
+    16-byte aligned array padded to a multiple of 128 keys when it is not one already."""
+    import torch
+    B, Nq, Hq, D = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    _int32_dev(q_pos, "q_pos")
+    _int32_dev(k_pos, "k_pos")
+    padded = max(128, -(-Nk // 128) * 128)
+    if (k_pos.stride(0) < padded or k_pos.stride(0) % 4 or k_pos.data_ptr() % 16
+            or k_pos.shape[1] < Nk):
+        kp = torch.zeros((B, padded), dtype=torch.int32, device=k_pos.device)
+        kp[:, :min(Nk, k_pos.shape[1])] = k_pos[:, :Nk]
+        k_pos = kp
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = lib().wpattn_prefill_positions(ctypes.byref(w._c()), _dev_tensor(q, "q"), _dev_tensor(k, "k"),
+                                        _dev_tensor(v, "v"), _dev_tensor(out, "out"),
+                                        ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+                                        B, Nq, Nk, Hq, Hkv, ctypes.c_void_p(q_pos.data_ptr()),
+                                        q_pos.stride(0), ctypes.c_void_p(k_pos.data_ptr()),
+                                        k_pos.stride(0), float(scale) if scale else 0.0,
+                                        _stream_ptr(stream))
+    _check(rc, "wpattn_prefill_positions")
     return out, lse
 
 

@@ -47,7 +47,7 @@ struct DeviceInfo {
   bool init = false;
   bool supported = false;
   int num_sms = 0;
-  bool prefill_attr[8] = {};  // (D 64, 128) x (g 1, 8) x (no mask, block mask)
+  bool prefill_attr[12] = {};  // (D 64, 128) x (g 1, 8) x (plain, block mask, positions)
   void* static_scratch = nullptr;  // device address of g_decode_static_scratch
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -131,7 +131,7 @@ int launch_rope(const void* x, void* out, int64_t B, int64_t N, int H, int D, in
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
-template <int D, bool G8, bool MASK>
+template <int D, bool G8, bool MASK, bool POS>
 int launch_prefill(const void* q, const void* k, const void* v, PrefillParams prm,
                    DeviceInfo* dev, cudaStream_t st) {
   using Shape = PrefillShape<D>;
@@ -146,25 +146,34 @@ int launch_prefill(const void* q, const void* k, const void* v, PrefillParams pr
   if ((rc = encode_bf16_4d(&tk, k, D, nk, hk, prm.B, 8, Shape::BN, false)) != WPATTN_OK) return rc;
   if ((rc = encode_bf16_4d(&tv, v, D, nk, hk, prm.B, 64, Shape::BN, true)) != WPATTN_OK) return rc;
   constexpr int smem = PrefillSmem<D>::ALLOC;
-  const int slot = (D == 64 ? 0 : 2) + (G8 ? 1 : 0) + (MASK ? 4 : 0);
+  const int slot = (D == 64 ? 0 : 6) + (G8 ? 3 : 0) + (MASK ? 1 : 0) + (POS ? 2 : 0);
   // a mask bit covers one 128-row query tile x one 128-key tile
   if (MASK && (Shape::BN != 128 || kBM != 128)) return WPATTN_EUNSUPPORTED;
   if (!dev->prefill_attr[slot]) {
-    if (cudaFuncSetAttribute(prefill_kernel<D, G8, MASK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(prefill_kernel<D, G8, MASK, POS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
       return WPATTN_ECUDA;
     dev->prefill_attr[slot] = true;
   }
   dim3 grid(prm.num_ctas_q, prm.Hq, prm.B);
-  prefill_kernel<D, G8, MASK><<<grid, Shape::THREADS, smem, st>>>(tq, tk, tv, prm);
+  prefill_kernel<D, G8, MASK, POS><<<grid, Shape::THREADS, smem, st>>>(tq, tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
-template <int D, bool MASK>
+template <int D, bool MASK, bool POS>
 int launch_prefill_g(const void* q, const void* k, const void* v, const PrefillParams& prm,
                      DeviceInfo* dev, cudaStream_t st) {
-  return prm.g8 ? launch_prefill<D, true, MASK>(q, k, v, prm, dev, st)
-                : launch_prefill<D, false, MASK>(q, k, v, prm, dev, st);
+  return prm.g8 ? launch_prefill<D, true, MASK, POS>(q, k, v, prm, dev, st)
+                : launch_prefill<D, false, MASK, POS>(q, k, v, prm, dev, st);
+}
+
+template <int D>
+int launch_prefill_mode(const void* q, const void* k, const void* v, const PrefillParams& prm,
+                        DeviceInfo* dev, cudaStream_t st) {
+  if (prm.block_mask && prm.q_pos) return WPATTN_EUNSUPPORTED;
+  if (prm.block_mask) return launch_prefill_g<D, true, false>(q, k, v, prm, dev, st);
+  if (prm.q_pos) return launch_prefill_g<D, false, true>(q, k, v, prm, dev, st);
+  return launch_prefill_g<D, false, false>(q, k, v, prm, dev, st);
 }
 
 template <int D, int GC, bool PM>
@@ -312,7 +321,9 @@ namespace {
 int prefill_impl(const wpattn_window* w, const void* q, const void* k, const void* v, void* out,
                  float* lse, int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
                  int64_t q_pos0, int64_t k_pos0, float softmax_scale, const uint32_t* block_mask,
-                 int32_t mask_words, void* cuda_stream) {
+                 int32_t mask_words, void* cuda_stream, const int32_t* q_pos = nullptr,
+                 int64_t q_pos_stride = 0, const int32_t* k_pos = nullptr,
+                 int64_t k_pos_stride = 0) {
   WindowPlan plan;
   int rc = make_window_plan(w, &plan);
   if (rc != WPATTN_OK) return rc;
@@ -345,6 +356,17 @@ int prefill_impl(const wpattn_window* w, const void* q, const void* k, const voi
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(plan.D));
   prm.scale_log2 = scale * 1.44269504088896340736f;
   prm.g8 = plan.g == 8 ? 1 : 0;
+  if (q_pos) {
+    // k_pos rows travel to shared memory 128 keys at a time by bulk copy
+    const int64_t padded = (static_cast<int64_t>(Nk) + 127) / 128 * 128;
+    if (!k_pos || q_pos_stride < Nq || k_pos_stride < padded || (k_pos_stride & 3) != 0 ||
+        (reinterpret_cast<uintptr_t>(q_pos) & 3u) != 0 || (reinterpret_cast<uintptr_t>(k_pos) & 15u) != 0)
+      return WPATTN_EINVAL;
+    prm.q_pos = q_pos;
+    prm.k_pos = k_pos;
+    prm.q_pos_stride = q_pos_stride;
+    prm.k_pos_stride = k_pos_stride;
+  }
   if (block_mask) {
     const int64_t nkt = (static_cast<int64_t>(Nk) + 127) / 128;
     if (mask_words < (nkt + 31) / 32 || (reinterpret_cast<uintptr_t>(block_mask) & 3u) != 0)
@@ -357,10 +379,8 @@ int prefill_impl(const wpattn_window* w, const void* q, const void* k, const voi
   const void* vv = Nk > 0 ? v : q;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   if (plan.D == 64)
-    return prm.block_mask ? launch_prefill_g<64, true>(q, kk, vv, prm, dev, st)
-                          : launch_prefill_g<64, false>(q, kk, vv, prm, dev, st);
-  return prm.block_mask ? launch_prefill_g<128, true>(q, kk, vv, prm, dev, st)
-                        : launch_prefill_g<128, false>(q, kk, vv, prm, dev, st);
+    return launch_prefill_mode<64>(q, kk, vv, prm, dev, st);
+  return launch_prefill_mode<128>(q, kk, vv, prm, dev, st);
 }
 
 }  // namespace
@@ -381,6 +401,16 @@ int wpattn_prefill_masked(const wpattn_window* w, const void* q, const void* k, 
   if (!block_mask) return WPATTN_EINVAL;
   return prefill_impl(w, q, k, v, out, lse, B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0, softmax_scale,
                       block_mask, mask_words, cuda_stream);
+}
+
+int wpattn_prefill_positions(const wpattn_window* w, const void* q, const void* k, const void* v,
+                             void* out, float* lse, int32_t B, int32_t Nq, int32_t Nk, int32_t Hq,
+                             int32_t Hkv, const int32_t* q_pos, int64_t q_pos_stride,
+                             const int32_t* k_pos, int64_t k_pos_stride, float softmax_scale,
+                             void* cuda_stream) {
+  if (!q_pos || !k_pos) return WPATTN_EINVAL;
+  return prefill_impl(w, q, k, v, out, lse, B, Nq, Nk, Hq, Hkv, 0, 0, softmax_scale, nullptr, 0,
+                      cuda_stream, q_pos, q_pos_stride, k_pos, k_pos_stride);
 }
 
 int wpattn_pack_block_mask(const uint8_t* mask, uint32_t* words, int64_t rows, int32_t nkb,

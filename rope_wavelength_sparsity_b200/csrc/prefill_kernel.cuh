@@ -76,6 +76,13 @@ struct PrefillParams {
   // rows of mask_words words, [B, Hq, ceil(Nq / 128), mask_words]
   const uint32_t* block_mask;
   int mask_words;
+  // explicit positions (the POS kernel): query t of sequence b at
+  // q_pos[b * q_pos_stride + t], key j at k_pos[b * k_pos_stride + j], both
+  // non-decreasing along the sequence; k_pos rows 16-byte aligned and padded
+  // to a multiple of 128 keys
+  const int32_t* q_pos;
+  const int32_t* k_pos;
+  int64_t q_pos_stride, k_pos_stride;
 };
 
 template <int D>
@@ -93,7 +100,9 @@ struct PrefillSmem {
   static constexpr int OFF_QM = OFF_V + NS * KTILE;          // masked first k-step of Q, per tile
   static constexpr int OFF_CT = OFF_QM + QT * 2 * PANEL_Q;    // per-warp transposed K pairs
   static constexpr int OFF_T = OFF_CT + 4 * QT * kCT * 32 * 4;  // thresholds (64 x int32)
-  static constexpr int OFF_BAR = OFF_T + 64 * 4;
+  static constexpr int OFF_QR = OFF_T + 64 * 4;               // first / last query position per tile
+  static constexpr int OFF_KP = OFF_QR + 16 * 4;              // key positions of each ring stage
+  static constexpr int OFF_BAR = OFF_KP + NS * BN * 4;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
   //           s_full[QT], p_full[QT], o_final[QT], qm_init[QT]
   static constexpr int NBAR = 1 + 4 * NS + 4 * QT;
@@ -114,8 +123,10 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 // G8: pairs share thresholds in groups of 8 (a compile-time switch, so the
 // two correction paths do not share a register allocation).  MASK: a block
 // mask selects the key tiles (compile-time too, so that the plain causal walk
-// keeps its registers).
-template <int D, bool G8, bool MASK>
+// keeps its registers).  POS: explicit, non-decreasing positions per token;
+// every column range that the contiguous kernel derives from a distance is
+// found by a binary search over the key tile's positions instead.
+template <int D, bool G8, bool MASK, bool POS>
 __global__ void __launch_bounds__(PrefillShape<D>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ PrefillParams p) {
@@ -163,10 +174,41 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int kvh = h / p.G;
   const int nkt = (p.Nk + BN - 1) / BN;
 
+  // Positions.  Without POS query i sits at qk_off + i and key j at j
+  // (relative to the first key); with POS they are read from the arrays.
+  const int32_t* qp_row = nullptr;
+  const int32_t* kp_row = nullptr;
+  if constexpr (POS) {
+    qp_row = p.q_pos + (size_t)b * p.q_pos_stride;
+    kp_row = p.k_pos + (size_t)b * p.k_pos_stride;
+  }
+  const int* sQR = reinterpret_cast<const int*>(smem + L::OFF_QR);  // POS: [t] first, [QT + t] last
+  auto k_first = [&](int kt) -> int {   // position of key tile kt's first key
+    if constexpr (POS) return __ldg(kp_row + BN * kt);
+    else return BN * kt;
+  };
+  auto k_last = [&](int kt) -> int {    // position of its last key (contiguous: as if full)
+    if constexpr (POS) return __ldg(kp_row + min(BN * kt + BN - 1, p.Nk - 1));
+    else return BN * kt + BN - 1;
+  };
+  auto q_first = [&](int t) -> int {    // position of query tile t's first row
+    if constexpr (POS) return sQR[t];
+    else return p.qk_off + (QT * cq + t) * kBM;
+  };
   // key tiles of query tile t: positions <= its last row, iterated from kt_top down
   auto last_key_tile = [&](int t) -> int {
     const int row0 = (QT * cq + t) * kBM;
     if (row0 >= p.Nq || p.Nk <= 0) return -1;
+    if constexpr (POS) {
+      // last key tile whose first key is not after the tile's last row
+      const int i_max = __ldg(qp_row + min(row0 + kBM - 1, p.Nq - 1));
+      int lo = 0, hi = nkt - 1, found = -1;
+      while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        if (k_first(mid) <= i_max) { found = mid; lo = mid + 1; } else { hi = mid - 1; }
+      }
+      return found;
+    }
     const int i_max = p.qk_off + min(row0 + kBM - 1, p.Nq - 1);
     if (i_max < 0) return -1;
     return min(i_max / BN, nkt - 1);
@@ -225,10 +267,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // Smallest distance of query tile t in key tile kt (negative on the diagonal).
   // Going down the key tiles it grows by 128, so the first kept pair of the
   // tile (p_min of that distance) only moves forward: advance it in place.
-  auto advance_plo = [&](int t, int kt, int& plo) {
-    const int dlo = p.qk_off + (QT * cq + t) * kBM - (BN * kt + BN - 1);
+  auto advance_plo_k = [&](int t, int klast, int& plo) {
+    const int dlo = q_first(t) - klast;
     while (plo < P && sT[plo] < dlo) ++plo;
   };
+  auto advance_plo = [&](int t, int kt, int& plo) { advance_plo_k(t, k_last(kt), plo); };
   // Split pair of the tile: pairs plo .. ps-1 (kept somewhere in the tile) are
   // left out of the contraction and added back where they are kept; pairs
   // ps .. P-1 are contracted and subtracted where they are pruned.  Splitting
@@ -238,15 +281,37 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // threshold, so for g = 8 the split falls on a group start.
   // The centre distance grows along the walk, so the first pair kept past it
   // (psr, carried by the caller) is advanced in place like plo.
-  auto split_pair = [&](int t, int kt, int plo, int& psr) -> int {
+  auto split_pair_k = [&](int t, int kfirst, int plo, int& psr) -> int {
     if (plo >= P) return plo;
-    const int dc = max(p.qk_off + (QT * cq + t) * kBM - BN * kt, 0);  // row 0 to key 0
+    const int dc = max(q_first(t) - kfirst, 0);  // row 0 to key 0
     const int target = dc > 0x7FFFFFDF ? 0x7FFFFFFF : dc + 32;
     while (psr < P && sT[psr] < target) ++psr;
     return min(max(psr, plo), P - (G8 ? 8 : 1));
   };
+  auto split_pair = [&](int t, int kt, int plo, int& psr) -> int {
+    return split_pair_k(t, k_first(kt), plo, psr);
+  };
+  // POS: number of the first nv keys of a ring stage whose position is below x
+  // (the stage's positions are sorted)
+  auto col_below = [&](const int* kps, int nv, int x) -> int {
+    int lo = 0, hi = nv;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (kps[mid] < x) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+  };
 
   if (threadIdx.x < 64) sT[threadIdx.x] = p.T[threadIdx.x];
+  if constexpr (POS) {
+    if (threadIdx.x < 2 * QT) {
+      const int t = threadIdx.x % QT;
+      const int row0 = (QT * cq + t) * kBM;
+      const int row = threadIdx.x < QT ? row0 : row0 + kBM - 1;
+      reinterpret_cast<int*>(smem + L::OFF_QR)[threadIdx.x] =
+          row0 < p.Nq ? __ldg(qp_row + min(row, p.Nq - 1)) : 0;
+    }
+  }
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < NS; ++s) {
@@ -292,9 +357,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int s = j % NS;
         const uint32_t ph = (j / NS) & 1;
         if (j >= NS && !mbar_wait(k_empty(s), ph ^ 1)) break;
-        mbar_arrive_expect_tx(k_full(s), L::KTILE);
+        mbar_arrive_expect_tx(k_full(s), L::KTILE + (POS ? BN * 4 : 0));
         for (int c = 0; c < D / 8; ++c)
           tma_load_4d(sK + s * L::KTILE + c * PANEL_K, &tmK, k_full(s), 8 * c, BN * kt, kvh, b);
+        if constexpr (POS)  // the tile's key positions travel with its keys
+          bulk_load(sbase + L::OFF_KP + s * BN * 4, kp_row + BN * kt, BN * 4, k_full(s));
         if (j >= NS && !mbar_wait(v_empty(s), ph ^ 1)) break;
         mbar_arrive_expect_tx(v_full(s), L::KTILE);
         for (int c = 0; c < D / 64; ++c)
@@ -319,8 +386,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint64_t qmdesc0 = make_sdesc(sQM, PANEL_Q, 128, 0);
       const uint64_t kdesc0 = make_sdesc(sK, (D / 16) * PANEL_K, 128, 0);
       const uint64_t vdesc0 = make_sdesc(sV, BN * 128, 1024, 2);
-      // split pair of QK_t on key tile kt: planned ahead of the wait for P_t
-      auto plan_qk = [&](int t, int kt) -> int {
+      // split pair of QK_t on key tile kt (in ring stage stage, already filled):
+      // planned ahead of the wait for P_t
+      auto plan_qk = [&](int t, int kt, int stage) -> int {
+        if constexpr (POS) {
+          const int* kps = reinterpret_cast<const int*>(smem + L::OFF_KP) + stage * BN;
+          advance_plo_k(t, kps[min(BN, p.Nk - BN * kt) - 1], plo[t]);
+          return split_pair_k(t, kps[0], plo[t], psr[t]);
+        }
         advance_plo(t, kt, plo[t]);
         return split_pair(t, kt, plo[t], psr[t]);
       };
@@ -349,7 +422,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int t = 0; t < QT; ++t)
           if (ok && (MASK ? ((mem_top >> t) & 1u) != 0 : kt_last[t] >= kt_top) &&
-              !issue_qk(t, 0, plan_qk(t, kt_top)))
+              !issue_qk(t, 0, plan_qk(t, kt_top, 0)))
             ok = false;
         umma_commit(k_empty(0));
       } else {
@@ -371,7 +444,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const bool in_n = MASK ? ((mem_n >> t) & 1u) != 0 : kt_n <= kt_last[t];
           const bool in_j = MASK ? ((mem >> t) & 1u) != 0 : kt <= kt_last[t];
           const bool do_qk = ok && next && in_n;
-          const int ps_n = do_qk ? plan_qk(t, kt_n) : 0;
+          const int ps_n = do_qk ? plan_qk(t, kt_n, (j + 1) % NS) : 0;
           if (ok && in_j) {
             if (!mbar_wait(p_full(t), cnt[t] & 1)) { ok = false; }
             if (ok) {
@@ -403,13 +476,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int wq = warp & 3;                   // TMEM lane quarter
     const int r = wq * 32 + lane;              // row within the tile = TMEM lane
     const int row = (QT * cq + t) * kBM + r;   // query index
-    const int i_pos = p.qk_off + row;          // relative position of this row
+    // position of this row (relative to the first key without POS)
+    const int i_pos = POS ? __ldg(qp_row + min(row, p.Nq - 1)) : p.qk_off + row;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t tS = lane_base + t * BN;
     const uint32_t tO = lane_base + TMEM_O + t * D;
     const uint8_t* smem_q = smem + L::OFF_Q + t * L::QTILE;
     uint8_t* smem_qm = smem + L::OFF_QM + t * 2 * PANEL_Q;
-    const int i_tile0 = p.qk_off + (QT * cq + t) * kBM;  // relative position of the first row
+    const int i_tile0 = q_first(t);           // position of the tile's first row
     const int my_kt_last = last_key_tile(t);
     int my_next = attended_below(t, my_kt_last, my_kt_last);  // this tile's next key tile, -1 when done
     float m_ref = -INFINITY;   // exponent reference of O and l (log2 units)
@@ -459,7 +533,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         continue;
       }
       const int kp0 = BN * kt;
-      const int d_row = i_pos - kp0;         // distance to the tile's first key
+      // POS: the stage's key positions (the first nv are keys), read after its fill;
+      // this row attends columns [0, c_caus)
+      const int* kps = reinterpret_cast<const int*>(smem + L::OFF_KP) + s * BN;
+      int nv = BN, k_lo = 0, k_hi = 0, c_caus = 0;
+      if constexpr (POS) {
+        if (!__all_sync(FULL, mbar_wait(k_full(s), (j / NS) & 1))) { ok = false; break; }
+        nv = min(BN, p.Nk - kp0);
+        k_lo = kps[0];
+        k_hi = kps[nv - 1];
+        c_caus = col_below(kps, nv, i_pos + 1);
+      }
+      const int d_row = i_pos - (POS ? k_lo : kp0);  // distance to the tile's first key
       const int plo = plo_next, ps = ps_next;
       const bool all_pruned = plo >= P;
       if constexpr (MASK) my_next = attended_below(t, kt - 1, my_kt_last);
@@ -478,12 +563,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // while the tensor core is still computing S, and S is added once it
       // is ready; for g = 8 they are applied to S in TMEM before it is read.
       const bool need_sub = !all_pruned && __any_sync(FULL, d_row > sT[ps]);
+      const int d_last = POS ? i_pos - k_hi : d_row - (BN - 1);  // distance to the last key
       const bool need_add = !all_pruned && ps > plo &&
-                            __any_sync(FULL, d_row >= 0 && d_row - (BN - 1) <= sT[ps - 1]);
+                            __any_sync(FULL, d_row >= 0 && d_last <= sT[ps - 1]);
       const bool corr = need_sub || need_add;
       // K stage s is released below; waiting for its fill first makes the
       // arrival count towards iteration j (the stage's previous phase is over)
-      if (!__all_sync(FULL, mbar_wait(k_full(s), (j / NS) & 1))) { ok = false; break; }
+      if constexpr (!POS) {
+        if (!__all_sync(FULL, mbar_wait(k_full(s), (j / NS) & 1))) { ok = false; break; }
+      }
       float sc[BN];
       if (corr && !G8) {
         const uint8_t* kb = smem + L::OFF_K + s * L::KTILE;
@@ -504,9 +592,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int T_lo = ps > plo ? sT[ps - 1] : 0;
 #pragma unroll 1
         for (int cc = 0; cc < BN / 32; ++cc) {
-          const int dc = d_row - 32 * cc;                  // distance at the chunk's first column
+          if (POS && 32 * cc >= nv) break;                 // no key in this chunk
+          // distance at the chunk's first column
+          const int dc = POS ? i_pos - kps[32 * cc] : d_row - 32 * cc;
           const int dmax = __shfl_sync(FULL, dc, 31);      // largest distance of the block
-          const int dmin = max(__shfl_sync(FULL, dc, 0) - 31, 0);
+          const int dmin = POS ? max(__shfl_sync(FULL, i_pos - kps[min(32 * cc + 31, nv - 1)], 0), 0)
+                               : max(__shfl_sync(FULL, dc, 0) - 31, 0);
           if (dmax < 0) continue;                          // wholly acausal
           // pairs ps .. pb-1 are pruned somewhere in the block, pa .. ps-1 kept somewhere
           int pb = ps;
@@ -537,7 +628,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               const int T = sT[pp];
               int lo, hi;  // chunk columns of this row that take the pair's term
               float sgn;
-              if (pp >= ps) {
+              if constexpr (POS) {
+                // chunk columns before cth are farther than T
+                const int cth = col_below(kps, nv, i_pos - T) - 32 * cc;
+                if (pp >= ps) {
+                  lo = 0;
+                  hi = min(cth, 32) - 1;
+                  sgn = -1.f;
+                } else {
+                  lo = max(cth, 0);
+                  hi = min(c_caus - 32 * cc, 32) - 1;
+                  sgn = 1.f;
+                }
+              } else if (pp >= ps) {
                 lo = 0;
                 hi = dc > T ? min(dc - T, 32) - 1 : -1;
                 sgn = -1.f;
@@ -593,7 +696,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const bool sub = gp >= ps;
           const int T = sT[gp];
           int c_lo, c_hi;  // columns of this row that take the group's term
-          if (sub) {
+          if constexpr (POS) {
+            const int cth = col_below(kps, nv, i_pos - T);  // columns farther than T
+            c_lo = sub ? 0 : cth;
+            c_hi = sub ? cth - 1 : c_caus - 1;
+          } else if (sub) {
             c_lo = 0;
             c_hi = d_row > T ? min(d_row - T - 1, BN - 1) : -1;
           } else {
@@ -669,11 +776,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
 
       // causal mask (d < 0) and the ragged key tail: columns c > cm
-      const bool need_mask = (i_tile0 - (kp0 + BN - 1) < 0) || (kp0 + BN > p.Nk);
+      const bool need_mask = POS ? (i_tile0 - k_hi < 0) || (nv < BN)
+                                 : (i_tile0 - (kp0 + BN - 1) < 0) || (kp0 + BN > p.Nk);
       int cm = BN - 1;
       if (need_mask) {
         // last column with d >= 0, and the last real key
-        cm = min(max(min(d_row, p.Nk - 1 - kp0), -1), BN);
+        cm = POS ? c_caus - 1 : min(max(min(d_row, p.Nk - 1 - kp0), -1), BN);
 #pragma unroll
         for (int c = 0; c < BN; ++c)
           if (c > cm) sc[c] = -INFINITY;

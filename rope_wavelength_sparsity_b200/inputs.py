@@ -270,3 +270,20 @@ def vertical_slash_mask(B: int, Hq: int, Nq: int, Nk: int, seed: int, q_pos0: in
                 if hi >= lo:
                     m[b, h, qb, lo:hi + 1] = True
     return m
+
+
+def sorted_positions(B: int, N: int, seed: int, span: float = 3.0, repeats: bool = False):
+    """int32 [B, N] non-decreasing positions: each row keeps N of the first
+    round(span * N) positions (a random sorted subset: a sequence with dropped
+    tokens).  ``repeats`` draws with replacement instead, so equal positions
+    occur (tokens sharing a position)."""
+    g = _gen(seed, "cpu")
+    total = max(N, int(round(span * N)))
+    rows = []
+    for _ in range(B):
+        if repeats:
+            r = torch.randint(0, total, (N,), generator=g).sort().values
+        else:
+            r = torch.randperm(total, generator=g)[:N].sort().values
+        rows.append(r)
+    return torch.stack(rows).to(torch.int32)
