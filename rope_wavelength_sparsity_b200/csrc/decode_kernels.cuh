@@ -85,7 +85,7 @@ struct DecodeSmem {
   static constexpr int TILE = KB * D * 2;              // K or V block
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = NS * TILE;
-  static constexpr int OFF_Q = 2 * NS * TILE;          // [8 heads][D] fp32, scaled by scale * log2(e)
+  static constexpr int OFF_Q = 2 * NS * TILE;          // [8 heads][D] bf16 query heads (zero past the CTA's)
   static constexpr int OFF_T = OFF_Q + 8 * D * 4;      // thresholds (64 x int32)
   static constexpr int OFF_P = OFF_T + 64 * 4;         // [warps][8 heads][KB] fp32 weights
   static constexpr int OFF_BAR = OFF_P + kDecodeComputeWarps * 8 * KB * 4;  // full[NS], empty[NS]
@@ -124,8 +124,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   constexpr int KB = L::KB, NS = L::NS, W = kDecodeComputeWarps;
   constexpr int P = D / 2;
   constexpr int NG = P / 8;               // groups of 8 pairs (16 dims: 8 in each half)
-  constexpr int TPK = D / 8;              // lanes per key in the PV step (one 16-byte chunk each)
-  constexpr int KPW = 32 / TPK;           // keys per PV step
+  constexpr int NMT = D / 16;             // PV: 16-dim row tiles of O^T
   constexpr uint32_t FULL = 0xffffffffu;
   static_assert(W * GC * D * 4 <= 2 * NS * L::TILE, "merge buffer must fit in the ring");
   static_assert(NS % W == 0, "each ring stage must belong to one compute warp");
@@ -137,7 +136,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   __shared__ float sm_l[W][GC];
   // the merge's partial outputs reuse the ring once every block is consumed
   float (*sm_o)[GC][D] = reinterpret_cast<float (*)[GC][D]>(smem);
-  float* qs = reinterpret_cast<float*>(smem + L::OFF_Q);
+  uint16_t* qb = reinterpret_cast<uint16_t*>(smem + L::OFF_Q);
   int* sT = reinterpret_cast<int*>(smem + L::OFF_T);
 
   const uint32_t sbase = smem_u32(smem);
@@ -176,7 +175,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   }
   if (threadIdx.x < 64) sT[threadIdx.x] = p.T[threadIdx.x];
   if (p.rope_q) {
-    for (int idx = threadIdx.x; idx < GC * P; idx += blockDim.x) {
+    for (int idx = threadIdx.x; idx < 8 * P; idx += blockDim.x) {
       const int hh = idx / P, pp = idx % P;
       float y0 = 0.f, y1 = 0.f;
       if (hh < nh) {
@@ -185,13 +184,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         rope_cos_sin(qpos, p.theta[pp], c, sn);
         rope_pair_bf16(bf16lo_to_f32(qr[pp]), bf16lo_to_f32(qr[pp + P]), c, sn, y0, y1);
       }
-      qs[hh * D + pp] = y0 * p.scale_log2;
-      qs[hh * D + pp + P] = y1 * p.scale_log2;
+      qb[hh * D + pp] = static_cast<uint16_t>(__float_as_uint(y0) >> 16);   // y0, y1 are bf16 values
+      qb[hh * D + pp + P] = static_cast<uint16_t>(__float_as_uint(y1) >> 16);
     }
   } else {
-    for (int idx = threadIdx.x; idx < GC * D; idx += blockDim.x) {
+    for (int idx = threadIdx.x; idx < 8 * D; idx += blockDim.x) {
       const int hh = idx / D, e = idx % D;
-      qs[idx] = hh < nh ? bf16lo_to_f32(p.q[((size_t)b * p.Hq + h0 + hh) * D + e]) * p.scale_log2 : 0.f;
+      qb[idx] = hh < nh ? p.q[((size_t)b * p.Hq + h0 + hh) * D + e] : static_cast<uint16_t>(0);
     }
   }
   __syncthreads();
@@ -286,17 +285,28 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   }
 
   // ---------------------------------------------------------------- compute
-  const int c = lane % TPK;               // PV: head-dim chunk [8c, 8c+8)
-  const int kk = lane / TPK;              // PV: key within a step
+  // PV on the tensor cores, per warp: O^T [D x 8 heads] += V^T [D x 16 keys] .
+  // P^T [16 keys x 8 heads], m16n8k16 steps (the heads of a CTA, at most 8,
+  // fill the n = 8 side).  Lane (gid = lane / 4, tig = lane % 4) holds, for row
+  // tile mt, dims 16 mt + gid and 16 mt + gid + 8 of heads 2 tig and 2 tig + 1.
+  const int gid = lane >> 2, tig = lane & 3;
   float* pw = reinterpret_cast<float*>(smem + L::OFF_P) + warp * 8 * KB;  // this warp's p rows
-  float m[GC], l[GC], o[GC][8];
+  float m[GC], l[GC];
+  float oacc[NMT][4];
 #pragma unroll
   for (int hh = 0; hh < GC; ++hh) {
     m[hh] = -INFINITY;
     l[hh] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) o[hh][e] = 0.f;
   }
+#pragma unroll
+  for (int mt = 0; mt < NMT; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) oacc[mt][e] = 0.f;
+  // lane's row address of matrix ldm_m = lane / 8 in the ldmatrix of (row tile
+  // mt, key step ks): key 16 ks + 8 (ldm_m >> 1) + lane % 8, dims chunk
+  // 2 mt + (ldm_m & 1)
+  const int ldm_key = 8 * ((lane >> 3) >> 1) + (lane & 7);
+  const int ldm_chunk = (lane >> 3) & 1;
 
   for (int i = warp; i < nblk; i += W) {
     const int s = i % NS;
@@ -324,52 +334,71 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       while (g0 < NG && sT[8 * g0 + 7] < dmin) ++g0;
     }
 
-    // ---- scores: one key per lane, groups g0 .. NG-1
-    float sc[GC];
+    // ---- scores on the tensor cores: S^T [32 keys x 8 heads] = K . Q^T over
+    // the kept groups g0 .. NG-1, one m16n8k16 step per (16 keys, group).  A
+    // group's k-step is its 16 dims: 8g..8g+7, then P+8g..P+8g+7.  Lane (gid,
+    // tig) holds the A elements of keys gid (+8) and pairs 8g + 2 tig (+1);
+    // where the window prunes a pair at a key's distance the element is zeroed.
+    float sacc[KB / 16][4];
 #pragma unroll
-    for (int hh = 0; hh < GC; ++hh) sc[hh] = 0.f;
+    for (int mt = 0; mt < KB / 16; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[mt][e] = 0.f;
+    {
+      int dk[KB / 8];                     // distances of keys gid, gid + 8, gid + 16, gid + 24
+#pragma unroll
+      for (int r = 0; r < KB / 8; ++r) dk[r] = __shfl_sync(FULL, dist, gid + 8 * r);
+      const uint16_t* qrow = qb + gid * D;
+      // this lane's ldmatrix row: matrix lane / 8 = (keys + 8 (lane / 8 & 1), half lane / 16)
+      const int lkey = 8 * ((lane >> 3) & 1) + (lane & 7);
+      const int lhalf = lane >> 4;
 #pragma unroll 1
-    for (int g = g0; g < NG; ++g) {
-      float kf[16];
-      {
-        float a[8], bb[8];
-        if (PM) {  // this key's 32-byte row of slab g
-          const uint4* row = reinterpret_cast<const uint4*>(kt + g * KB * 32 + lane * 32);
-          unpack8(row[0], a);
-          unpack8(row[1], bb);
-        } else {
-          unpack8(ring_chunk<D>(kt, lane, g), a);            // dims 8g .. 8g+7
-          unpack8(ring_chunk<D>(kt, lane, NG + g), bb);      // dims P+8g .. P+8g+7
+      for (int g = g0; g < NG; ++g) {
+        // B = Q^T: dims 8g + 2 tig (+1) and P + 8g + 2 tig (+1) of head gid
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(qrow + 8 * g + 2 * tig);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(qrow + P + 8 * g + 2 * tig);
+        const bool prune = __any_sync(FULL, dist > sT[8 * g]);
+        const int T0 = sT[8 * g + 2 * tig], T1 = sT[8 * g + 2 * tig + 1];
+#pragma unroll
+        for (int mt = 0; mt < KB / 16; ++mt) {
+          const int key = 16 * mt + lkey;
+          uint32_t addr;
+          if (PM) {
+            addr = smem_u32(kt) + g * KB * 32 + key * 32 + lhalf * 16;
+          } else {
+            const int ch = lhalf ? NG + g : g;
+            addr = smem_u32(kt) + (ch >> 3) * L::PANEL + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
+          }
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(addr, a0, a1, a2, a3);
+          if (prune) {
+            const int d0 = dk[2 * mt], d1 = dk[2 * mt + 1];
+            const uint32_t m0 = (d0 > T0 ? 0u : 0x0000FFFFu) | (d0 > T1 ? 0u : 0xFFFF0000u);
+            const uint32_t m1 = (d1 > T0 ? 0u : 0x0000FFFFu) | (d1 > T1 ? 0u : 0xFFFF0000u);
+            a0 &= m0; a2 &= m0; a1 &= m1; a3 &= m1;
+          }
+          mma_16816_bf16(sacc[mt], a0, a1, a2, a3, b0, b1);
         }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) { kf[e] = a[e]; kf[8 + e] = bb[e]; }
-      }
-      // pairs of the group pruned at this key's distance contribute 0
-      if (__any_sync(FULL, dist > sT[8 * g])) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (dist > sT[8 * g + e]) { kf[e] = 0.f; kf[8 + e] = 0.f; }
-        }
-      }
-#pragma unroll
-      for (int hh = 0; hh < GC; ++hh) {
-        const float4* qa = reinterpret_cast<const float4*>(qs + hh * D + 8 * g);
-        const float4* qb = reinterpret_cast<const float4*>(qs + hh * D + P + 8 * g);
-        const float4 x0 = qa[0], x1 = qa[1], y0 = qb[0], y1 = qb[1];
-        float a0 = 0.f, a1 = 0.f;
-        fma2(a0, a1, x0.x, x0.y, kf[0], kf[1], a0, a1);
-        fma2(a0, a1, x0.z, x0.w, kf[2], kf[3], a0, a1);
-        fma2(a0, a1, x1.x, x1.y, kf[4], kf[5], a0, a1);
-        fma2(a0, a1, x1.z, x1.w, kf[6], kf[7], a0, a1);
-        fma2(a0, a1, y0.x, y0.y, kf[8], kf[9], a0, a1);
-        fma2(a0, a1, y0.z, y0.w, kf[10], kf[11], a0, a1);
-        fma2(a0, a1, y1.x, y1.y, kf[12], kf[13], a0, a1);
-        fma2(a0, a1, y1.z, y1.w, kf[14], kf[15], a0, a1);
-        sc[hh] += a0 + a1;
       }
     }
+    // S^T through the warp's p rows (free until the softmax writes them): each
+    // lane then holds its own key's scores for every head, in log2 units
+    {
+      float* ssc = pw;                    // [32 keys][8 heads]
+#pragma unroll
+      for (int mt = 0; mt < KB / 16; ++mt) {
+        *reinterpret_cast<float2*>(ssc + (16 * mt + gid) * 8 + 2 * tig) = make_float2(sacc[mt][0], sacc[mt][1]);
+        *reinterpret_cast<float2*>(ssc + (16 * mt + gid + 8) * 8 + 2 * tig) = make_float2(sacc[mt][2], sacc[mt][3]);
+      }
+    }
+    __syncwarp();
+    float sc[GC];
+#pragma unroll
+    for (int hh = 0; hh < GC; ++hh) sc[hh] = pw[lane * 8 + hh] * p.scale_log2;
+    __syncwarp();                         // every lane has its scores before p overwrites them
 
     // ---- online softmax over the block (warp-wide max per head)
+    float corr_h[GC];
 #pragma unroll
     for (int hh = 0; hh < GC; ++hh) {
       const float sv = valid ? sc[hh] : -INFINITY;
@@ -378,60 +407,97 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       for (int off = 16; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(FULL, bm, off));
       const float mn = fmaxf(m[hh], bm);
       float pv = 0.f;
+      corr_h[hh] = 1.f;
       if (mn != -INFINITY) {
         const float corr = (m[hh] == -INFINITY) ? 0.f : ex2_approx(m[hh] - mn);
         pv = ex2_approx(sv - mn);
         l[hh] = l[hh] * corr + pv;        // this lane's key only; summed over lanes at the end
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) mul2(o[hh][e], o[hh][e + 1], o[hh][e], o[hh][e + 1], corr, corr);
+        corr_h[hh] = corr;
         m[hh] = mn;
       }
       pw[hh * KB + lane] = pv;
     }
     __syncwarp();
 
-    // ---- O += p V: lane (kk, c) takes chunk c of keys kk, kk + KPW, ...
-    // (keys past the sequence end are not read: a cache may hold anything there)
-    const int nvalid = min(KB, j_end - j0);
-#pragma unroll 4
-    for (int r = kk; r < nvalid; r += KPW) {
-      float vf[8];
-      unpack8(ring_chunk<D>(vt, r, c), vf);
+    // ---- O^T = O^T * corr + V^T P^T on the tensor cores
+    {
+      // this lane's heads 2 tig, 2 tig + 1 (1 where they are past the CTA's heads)
+      float ca = 1.f, cb = 1.f;
+      bool moved = false;
 #pragma unroll
       for (int hh = 0; hh < GC; ++hh) {
-        const float pr = pw[hh * KB + r];
+        moved |= corr_h[hh] != 1.f;
+        if (hh == 2 * tig) ca = corr_h[hh];
+        if (hh == 2 * tig + 1) cb = corr_h[hh];
+      }
+      if (moved) {
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) fma2(o[hh][e], o[hh][e + 1], pr, pr, vf[e], vf[e + 1], o[hh][e], o[hh][e + 1]);
+        for (int mt = 0; mt < NMT; ++mt) {
+          mul2(oacc[mt][0], oacc[mt][1], oacc[mt][0], oacc[mt][1], ca, cb);
+          mul2(oacc[mt][2], oacc[mt][3], oacc[mt][2], oacc[mt][3], ca, cb);
+        }
+      }
+    }
+    // keys past the sequence end hold anything (a cache may keep NaN there):
+    // their V elements are zeroed before the product, their p is 0
+    const int nvalid = min(KB, j_end - j0);
+#pragma unroll
+    for (int ks = 0; ks < KB / 16; ++ks) {
+      if (16 * ks >= nvalid) break;
+      // B = P^T: keys 16 ks + 2 tig (+1) and + 8, head gid (0 past the CTA's heads)
+      uint32_t b0 = 0u, b1 = 0u;
+      if (gid < GC) {
+        const float2 x0 = *reinterpret_cast<const float2*>(pw + gid * KB + 16 * ks + 2 * tig);
+        const float2 x1 = *reinterpret_cast<const float2*>(pw + gid * KB + 16 * ks + 8 + 2 * tig);
+        b0 = pack_bf16x2(x0.x, x0.y);
+        b1 = pack_bf16x2(x1.x, x1.y);
+      }
+      const int key = 16 * ks + ldm_key;
+      // element masks of the A registers: (key 2 tig, 2 tig + 1) and the same + 8
+      const int kl = 16 * ks + 2 * tig;
+      const uint32_t mlo = (kl < nvalid ? 0x0000FFFFu : 0u) | (kl + 1 < nvalid ? 0xFFFF0000u : 0u);
+      const uint32_t mhi = (kl + 8 < nvalid ? 0x0000FFFFu : 0u) | (kl + 9 < nvalid ? 0xFFFF0000u : 0u);
+#pragma unroll
+      for (int mt = 0; mt < NMT; ++mt) {
+        const int chunk = 2 * mt + ldm_chunk;
+        const uint32_t addr = smem_u32(vt) + (chunk >> 3) * L::PANEL + key * 128 +
+                              (((chunk & 7) ^ (key & 7)) << 4);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_trans(addr, a0, a1, a2, a3);
+        a0 &= mlo; a1 &= mlo; a2 &= mhi; a3 &= mhi;
+        mma_16816_bf16(oacc[mt], a0, a1, a2, a3, b0, b1);
       }
     }
     __syncwarp();  // the p rows are rewritten by the next block
     if (lane == 0) mbar_arrive(empty(s));
   }
 
-  // combine this warp's lanes: l over keys (all lanes), o over the KPW key groups
+  // combine this warp's lanes' l (one key each)
 #pragma unroll
   for (int hh = 0; hh < GC; ++hh) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) l[hh] += __shfl_xor_sync(FULL, l[hh], off);
-#pragma unroll
-    for (int off = TPK; off < 32; off <<= 1) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[hh][e] += __shfl_xor_sync(FULL, o[hh][e], off);
-    }
   }
 
   // merge the warps of this CTA (compute warps only); every block has been
   // consumed, so the ring is free
   asm volatile("bar.sync 1, %0;" ::"n"(W * 32) : "memory");
-  if (kk == 0) {
+#pragma unroll
+  for (int mt = 0; mt < NMT; ++mt) {
+    if (2 * tig < GC) {
+      sm_o[warp][2 * tig][16 * mt + gid] = oacc[mt][0];
+      sm_o[warp][2 * tig][16 * mt + gid + 8] = oacc[mt][2];
+    }
+    if (2 * tig + 1 < GC) {
+      sm_o[warp][2 * tig + 1][16 * mt + gid] = oacc[mt][1];
+      sm_o[warp][2 * tig + 1][16 * mt + gid + 8] = oacc[mt][3];
+    }
+  }
+  if (lane == 0) {
 #pragma unroll
     for (int hh = 0; hh < GC; ++hh) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) sm_o[warp][hh][8 * c + e] = o[hh][e];
-      if (c == 0) {
-        sm_m[warp][hh] = m[hh];
-        sm_l[warp][hh] = l[hh];
-      }
+      sm_m[warp][hh] = m[hh];
+      sm_l[warp][hh] = l[hh];
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(W * 32) : "memory");
