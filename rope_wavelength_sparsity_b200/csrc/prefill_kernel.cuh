@@ -271,7 +271,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int dlo = q_first(t) - klast;
     while (plo < P && sT[plo] < dlo) ++plo;
   };
-  auto advance_plo = [&](int t, int kt, int& plo) { advance_plo_k(t, k_last(kt), plo); };
+  // (the contiguous forms are written out: routed through the position lambdas
+  // the MMA lane's code came out 2% slower on the 32K Qwen-shaped prefill)
+  auto advance_plo = [&](int t, int kt, int& plo) {
+    if constexpr (!POS) {
+      const int dlo = p.qk_off + (QT * cq + t) * kBM - (BN * kt + BN - 1);
+      while (plo < P && sT[plo] < dlo) ++plo;
+    } else {
+      advance_plo_k(t, k_last(kt), plo);
+    }
+  };
   // Split pair of the tile: pairs plo .. ps-1 (kept somewhere in the tile) are
   // left out of the contraction and added back where they are kept; pairs
   // ps .. P-1 are contracted and subtracted where they are pruned.  Splitting
@@ -289,7 +298,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     return min(max(psr, plo), P - (G8 ? 8 : 1));
   };
   auto split_pair = [&](int t, int kt, int plo, int& psr) -> int {
-    return split_pair_k(t, k_first(kt), plo, psr);
+    if constexpr (!POS) {
+      if (plo >= P) return plo;
+      const int dc = max(p.qk_off + (QT * cq + t) * kBM - BN * kt, 0);  // row 0 to key 0
+      const int target = dc > 0x7FFFFFDF ? 0x7FFFFFFF : dc + 32;
+      while (psr < P && sT[psr] < target) ++psr;
+      return min(max(psr, plo), P - (G8 ? 8 : 1));
+    } else {
+      return split_pair_k(t, k_first(kt), plo, psr);
+    }
   };
   // POS: number of the first nv keys of a ring stage whose position is below x
   // (the stage's positions are sorted)
