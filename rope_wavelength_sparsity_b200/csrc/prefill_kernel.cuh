@@ -49,17 +49,23 @@ constexpr int kCT = 16;               // pairs per batch of the per-warp K trans
 // both head dims (2 x (128 + 128) = 512 columns at D = 128).  The kernel
 // also supports three query tiles on 96-key tiles (3 x (96 + 64) = 480
 // columns at D = 64); measured slower there (its 152-register softmax
-// warpgroups spill), so it is not selected.
+// warpgroups spill), so it is not selected.  One query tile per CTA with two
+// CTAs per SM (two MMA lanes per SM) is supported too; at D = 64 it measured
+// 6% slower windowed and no faster with the window off, so it is not selected.
 template <int D>
 struct PrefillShape {
-  static constexpr int QT = 2;                        // query tiles per CTA = softmax warpgroups
+  // query tiles per CTA = softmax warpgroups
+  static constexpr int QT = 2;
   static constexpr int BN = 128;                      // keys per tile
   static constexpr int THREADS = (QT + 1) * 128;      // + producer, MMA issuer, 2 idle warps
-  // Registers: launched at 65536 / THREADS per thread; the softmax warpgroups
-  // grow and the last warpgroup shrinks to 56:
-  //   QT = 2: 256 x 224 + 128 x 56 = 64512;  QT = 3: 384 x 152 + 128 x 56 = 65536.
-  static constexpr uint32_t REGS_SOFTMAX = (QT == 3) ? 152 : 224;
+  static constexpr int CTAS_PER_SM = (QT == 1) ? 2 : 1;
+  // Registers: launched at 65536 / (THREADS x CTAS_PER_SM) per thread; the
+  // softmax warpgroups grow and the last warpgroup shrinks to 56:
+  //   QT = 2: 256 x 224 + 128 x 56 = 64512;  QT = 3: 384 x 152 + 128 x 56 = 65536;
+  //   QT = 1 (two CTAs per SM): 2 x (128 x 200 + 128 x 56) = 65536.
+  static constexpr uint32_t REGS_SOFTMAX = (QT == 3) ? 152 : (QT == 1) ? 200 : 224;
   static constexpr uint32_t REGS_OTHER = 56;
+  static constexpr uint32_t TMEM_COLS = (QT == 1) ? 256 : 512;  // S tiles then O tiles
 };
 
 struct PrefillParams {
@@ -88,7 +94,7 @@ struct PrefillParams {
 template <int D>
 struct PrefillSmem {
   static constexpr int QT = PrefillShape<D>::QT, BN = PrefillShape<D>::BN;
-  static constexpr int NS = (D == 64) ? 4 : 2;       // K/V ring depth
+  static constexpr int NS = (D == 64 && QT > 1) ? 4 : 2;  // K/V ring depth
   static constexpr int NPOLY = 0;                    // of every 8 column pairs, exp2 on the FMA pipe
   static constexpr int QTILE = kBM * D * 2;          // one Q tile in bytes
   static constexpr int KTILE = BN * D * 2;           // one K or V tile in bytes
@@ -127,7 +133,7 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 // every column range that the contiguous kernel derives from a distance is
 // found by a binary search over the key tile's positions instead.
 template <int D, bool G8, bool MASK, bool POS>
-__global__ void __launch_bounds__(PrefillShape<D>::THREADS, 1)
+__global__ void __launch_bounds__(PrefillShape<D>::THREADS, PrefillShape<D>::CTAS_PER_SM)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ PrefillParams p) {
   using L = PrefillSmem<D>;
@@ -347,7 +353,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     fence_barrier_init();
   }
   if (warp == W_MMA) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_alloc(smem_u32(tmem_slot), PrefillShape<D>::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -933,7 +939,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, 512);
+  if (warp == W_MMA) tmem_dealloc(tmem, PrefillShape<D>::TMEM_COLS);
 }
 
 // Byte block mask [rows, nkb] (nonzero = attended) -> the kernel's bit rows of
