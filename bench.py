@@ -547,6 +547,30 @@ def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
     }
     res["gpu_launches"] += 2 * steps
     del kp, vp, ws_pg
+    if world > 1 and getattr(args, "kv_split", False):
+        # strong scaling: the same decode (rank 0's problem) with its cache split by
+        # length; each rank holds L / world keys of every sequence
+        from rope_wavelength_sparsity_b200 import distributed as wd
+        q0, kc0, vc0, kvl0 = inputs.decode_inputs(w, seed=0, device=dev)
+        kvl0 = [int(x) for x in kvl0]
+        shard = (w.Nk + world - 1) // world
+        ks = kc0[:, rank * shard:(rank + 1) * shard].contiguous()
+        vs = vc0[:, rank * shard:(rank + 1) * shard].contiguous()
+        del kc0, vc0
+        alg0, _ = decode_bytes(w, win, wp, kvl0)
+
+        def step_split():
+            wd.decode_kv_split(q0, ks, vs, kvl0, win, shard_len=shard, rank=rank, world=world,
+                               scale=w.scale)
+
+        sp_ms, _, _ = time_steps(step_split, args.warmup, steps, flush, world,
+                                 per_step_events=False)
+        res["kv_split"] = {
+            "value": round(alg0 / (sp_ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "ms_per_step": round(sp_ms / steps, 4), "scaling": "strong",
+            "exchange": "one all-gather of (out, lse) parts per step, then merge_lse",
+        }
+        del ks, vs
     if primary:
         res["clocks"] = clk
         qh = q.cpu().pin_memory()
@@ -665,6 +689,9 @@ def main():
     ap.add_argument("--only-primary", action="store_true",
                     help="skip the secondary decode measurement of the default workload")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--kv-split", action="store_true",
+                    help="with N > 1: also time the decode with its cache split by length over "
+                         "the ranks (strong scaling, one all-gather per step)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -386,6 +386,45 @@ WPATTN_API int wpattn_decode_rope(const wpattn_window *w,
                   void *cuda_stream);
 
 /*
+ * One shard of a decode whose KV cache is split by length across devices
+ * (each device holds a contiguous range of every sequence's keys).  The call
+ * attends the query to the shard's keys only and returns the result
+ * normalised over them, with its log-sum-exp; wpattn_merge_lse then combines
+ * the shards' results into the decode over the whole cache (exactly, up to
+ * rounding: each shard's part enters with weight exp(lse_shard - lse)).
+ *   k_shard, v_shard: bf16 device [B, Lmax, Hkv, D], the shard's keys.
+ *   kv_len_host: host int32 [B], keys of each sequence in this shard,
+ *                0 <= kv_len <= Lmax (0: the shard has none of them).
+ *   q_pos_host:  host int64 [B], position of each query in the whole cache.
+ *   k_pos0_host: host int64 [B], position of the shard's first key of each
+ *                sequence; its key j sits at k_pos0 + j.  Every key of the
+ *                shard must be at or before the query (else WPATTN_EINVAL).
+ *   lse: required.  A sequence with no key in the shard gets out = 0 and
+ *        lse = -inf.  Workspace and the remaining arguments as for
+ *        wpattn_decode (size it with the shard's Lmax).
+ */
+WPATTN_API int wpattn_decode_shard(const wpattn_window *w,
+                  const void *q, const void *k_shard, const void *v_shard,
+                  const int32_t *kv_len_host, int64_t Lmax,
+                  const int64_t *q_pos_host, const int64_t *k_pos0_host,
+                  int32_t B, int32_t Hq, int32_t Hkv, float softmax_scale,
+                  void *out, float *lse,
+                  void *workspace, size_t workspace_bytes,
+                  void *cuda_stream);
+
+/*
+ * Combine R partial attention results of the same rows:
+ *   outs: bf16 device [R, rows, head_dim], each normalised over its keys;
+ *   lses: fp32 device [R, rows], natural-log sum-exp of each part (-inf: no key);
+ *   out:  bf16 device [rows, head_dim];  lse: fp32 device [rows] or NULL.
+ * out = sum_r w_r outs_r / sum_r w_r with w_r = exp(lses_r - max_r lses_r);
+ * lse = max + ln(sum_r w_r).  A row whose parts are all empty gets 0 and
+ * -inf.  head_dim in {64, 128}.  Asynchronous on `cuda_stream`.
+ */
+WPATTN_API int wpattn_merge_lse(const void *outs, const float *lses, int32_t R, int64_t rows,
+                  int32_t head_dim, void *out, float *lse, void *cuda_stream);
+
+/*
  * Synchronises `cuda_stream`, then reads and clears the current device's
  * kernel status word.  Returns WPATTN_OK, WPATTN_ETIMEOUT (a kernel gave up a
  * bounded wait; its outputs are undefined), WPATTN_EINDEX (a kernel met an

@@ -10,7 +10,7 @@ exception is raised.
 Entry points (same names as the C ABI, without the ``wpattn_`` prefix):
 ``prefill``, ``decode``, ``decode_pairmajor``, ``kcache_to_pairmajor``,
 ``decode_positions``, ``decode_paged``, ``prefill_masked``, ``pack_block_mask``, ``rope``,
-``prefill_rope``, ``decode_rope``, ``prefill_positions``,
+``prefill_rope``, ``decode_rope``, ``prefill_positions``, ``decode_shard``, ``merge_lse``,
 ``decode_workspace_size``, ``decode_noalloc``, ``pruned_fraction``,
 ``thresholds``, ``device_status``.
 """
@@ -89,6 +89,10 @@ def lib() -> ctypes.CDLL:
         L.wpattn_decode_positions.argtypes = [wp, vp, vp, vp, i32p, i64, i32p, vp, i64, i32, i32,
                                               i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
         L.wpattn_decode_rope.argtypes = L.wpattn_decode_positions.argtypes
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        L.wpattn_decode_shard.argtypes = [wp, vp, vp, vp, i32p, i64, i64p, i64p, i32, i32, i32,
+                                          f32, vp, vp, vp, ctypes.c_size_t, vp]
+        L.wpattn_merge_lse.argtypes = [vp, vp, i32, i64, i32, vp, vp, vp]
         L.wpattn_decode_paged.argtypes = [wp, vp, vp, vp, i32, i32, vp, i32, i32p, i32p, vp, i64,
                                           i32, i32, i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
         L.wpattn_device_status.argtypes = [vp]
@@ -435,6 +439,48 @@ def decode_rope(q, k_cache, v_cache, kv_len, w: Window, *, q_pos=None, k_pos=Non
                                   ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
                                   _stream_ptr(stream))
     _check(rc, "wpattn_decode_rope")
+    return out, lse
+
+
+def decode_shard(q, k_shard, v_shard, kv_len, q_pos, k_pos0, w: Window, *,
+                 scale: float | None = None, out=None, lse=None, workspace=None, stream=None):
+    """Decode over one length-shard of a cache: the query of sequence b at q_pos[b], the
+    shard's keys at k_pos0[b] + j for j < kv_len[b] (host ints; kv_len may be 0).  Returns
+    (out normalised over the shard's keys, lse) for ``merge_lse``."""
+    import torch
+    B, Hq, D = q.shape
+    L, Hkv = k_shard.shape[1], k_shard.shape[2]
+    kvl = (ctypes.c_int32 * B)(*[int(x) for x in kv_len])
+    qp = (ctypes.c_int64 * B)(*[int(x) for x in q_pos])
+    kp = (ctypes.c_int64 * B)(*[int(x) for x in k_pos0])
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    out, lse, workspace = _decode_outputs(q, w, B, Hq, Hkv, L, out, lse, True, workspace)
+    rc = lib().wpattn_decode_shard(ctypes.byref(w._c()), _dev_tensor(q, "q"),
+                                   _dev_tensor(k_shard, "k_shard"), _dev_tensor(v_shard, "v_shard"),
+                                   kvl, L, qp, kp, B, Hq, Hkv, float(scale) if scale else 0.0,
+                                   _dev_tensor(out, "out"), ctypes.c_void_p(lse.data_ptr()),
+                                   ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                   _stream_ptr(stream))
+    _check(rc, "wpattn_decode_shard")
+    return out, lse
+
+
+def merge_lse(outs, lses, *, out=None, lse=None, stream=None):
+    """Combine parts outs [R, ..., D] (bf16 CUDA) with their lses [R, ...] (fp32 CUDA)
+    into (out [..., D], lse [...])."""
+    import torch
+    R, D = outs.shape[0], outs.shape[-1]
+    rows = outs[0].numel() // D
+    if lses.dtype != torch.float32 or not lses.is_cuda or not lses.is_contiguous():
+        raise TypeError("lses must be a contiguous fp32 CUDA tensor")
+    if out is None:
+        out = torch.empty(outs.shape[1:], dtype=outs.dtype, device=outs.device)
+    if lse is None:
+        lse = torch.empty(lses.shape[1:], dtype=torch.float32, device=outs.device)
+    _check(lib().wpattn_merge_lse(_dev_tensor(outs, "outs"), ctypes.c_void_p(lses.data_ptr()), R,
+                                  rows, D, _dev_tensor(out, "out"), ctypes.c_void_p(lse.data_ptr()),
+                                  _stream_ptr(stream)), "wpattn_merge_lse")
     return out, lse
 
 

@@ -511,6 +511,7 @@ struct DecodeLayout {
   const int32_t* k_pos = nullptr;         // device [B, k_pos_stride]
   int64_t k_pos_stride = 0;
   bool rope_q = false;                    // q arrives before its RoPE rotation
+  bool shard = false;                     // one shard of a longer cache: kv_len may be 0
 };
 
 int decode_impl(const wpattn_window* w, const void* q, const void* k_cache, const void* v_cache,
@@ -529,8 +530,8 @@ int decode_impl(const wpattn_window* w, const void* q, const void* k_cache, cons
   const int G = Hq / Hkv;
   if (G > 16 || B > kDecodeMaxB || Lmax >= (int64_t(1) << 31)) return WPATTN_EUNSUPPORTED;
   for (int b = 0; b < B; ++b)
-    if (kv_len_host[b] < 1 || kv_len_host[b] > Lmax) return WPATTN_EINVAL;
-  if (lay.q_pos_host)
+    if (kv_len_host[b] < (lay.shard ? 0 : 1) || kv_len_host[b] > Lmax) return WPATTN_EINVAL;
+  if (lay.q_pos_host && !lay.shard)
     for (int b = 0; b < B; ++b)
       if (lay.q_pos_host[b] < 0 || lay.q_pos_host[b] == INT32_MAX) return WPATTN_EINVAL;
   if (lay.k_pos) {
@@ -628,6 +629,48 @@ int wpattn_decode_rope(const wpattn_window* w, const void* q, const void* k_cach
   lay.k_pos_stride = k_pos_stride;
   return decode_impl(w, q, k_cache, v_cache, kv_len_host, Lmax, B, Hq, Hkv, softmax_scale, out, lse,
                      workspace, workspace_bytes, cuda_stream, lay);
+}
+
+int wpattn_decode_shard(const wpattn_window* w, const void* q, const void* k_shard,
+                        const void* v_shard, const int32_t* kv_len_host, int64_t Lmax,
+                        const int64_t* q_pos_host, const int64_t* k_pos0_host, int32_t B,
+                        int32_t Hq, int32_t Hkv, float softmax_scale, void* out, float* lse,
+                        void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  if (!q_pos_host || !k_pos0_host || !lse || !kv_len_host || B <= 0 || B > kDecodeMaxB)
+    return WPATTN_EINVAL;
+  // the kernel measures distances from the shard's first key: the query sits
+  // at q_pos - k_pos0, the shard's key j at j, every one of them before it
+  int32_t rel[kDecodeMaxB];
+  for (int b = 0; b < B; ++b) {
+    const int64_t r = q_pos_host[b] - k_pos0_host[b];
+    if (q_pos_host[b] < 0 || k_pos0_host[b] < 0 || r >= INT32_MAX) return WPATTN_EINVAL;
+    if (kv_len_host[b] > 0 && r < static_cast<int64_t>(kv_len_host[b]) - 1) return WPATTN_EINVAL;
+    rel[b] = kv_len_host[b] > 0 ? static_cast<int32_t>(r) : 0;
+  }
+  DecodeLayout lay;
+  lay.shard = true;
+  lay.q_pos_host = rel;
+  return decode_impl(w, q, k_shard, v_shard, kv_len_host, Lmax, B, Hq, Hkv, softmax_scale, out, lse,
+                     workspace, workspace_bytes, cuda_stream, lay);
+}
+
+int wpattn_merge_lse(const void* outs, const float* lses, int32_t R, int64_t rows, int32_t head_dim,
+                     void* out, float* lse, void* cuda_stream) {
+  if (R <= 0 || rows < 0) return WPATTN_EINVAL;
+  if (head_dim != 64 && head_dim != 128) return WPATTN_EUNSUPPORTED;
+  if (rows == 0) return WPATTN_OK;
+  if (!outs || !lses || !out || rows > 0x7FFFFFFFLL) return WPATTN_EINVAL;
+  DeviceInfo* dev = nullptr;
+  int rc;
+  if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (head_dim == 64)
+    merge_lse_kernel<64><<<static_cast<unsigned>(rows), 64, 0, st>>>(
+        static_cast<const uint16_t*>(outs), lses, R, rows, static_cast<uint16_t*>(out), lse);
+  else
+    merge_lse_kernel<128><<<static_cast<unsigned>(rows), 128, 0, st>>>(
+        static_cast<const uint16_t*>(outs), lses, R, rows, static_cast<uint16_t*>(out), lse);
+  return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
 int wpattn_decode_paged(const wpattn_window* w, const void* q, const void* k_pages,

@@ -587,4 +587,30 @@ decode_combine_kernel(const __grid_constant__ DecodeParams p) {
     p.lse[bh] = Ls > 0.f ? (M + __log2f(Ls)) * 0.69314718055994530942f : -INFINITY;
 }
 
+// Merge of R partial results of the same rows (each normalised over its own
+// keys, with its log-sum-exp): out = sum_r w_r out_r / sum_r w_r, w_r =
+// exp(lse_r - max lse), lse = max lse + ln sum_r w_r.  One block per row,
+// one thread per head dim; a row whose parts are all empty gets 0 and -inf.
+template <int D>
+__global__ void __launch_bounds__(D)
+merge_lse_kernel(const uint16_t* __restrict__ outs, const float* __restrict__ lses, int R,
+                 int64_t rows, uint16_t* __restrict__ out, float* __restrict__ lse) {
+  const int64_t row = blockIdx.x;
+  const int e = threadIdx.x;
+  float M = -INFINITY;
+  for (int r = 0; r < R; ++r) M = fmaxf(M, lses[(size_t)r * rows + row]);
+  float W = 0.f, acc = 0.f;
+  if (M != -INFINITY) {
+    for (int r = 0; r < R; ++r) {
+      const float lr = lses[(size_t)r * rows + row];
+      const float w = lr == -INFINITY ? 0.f : __expf(lr - M);
+      W += w;
+      acc += w * bf16lo_to_f32(outs[((size_t)r * rows + row) * D + e]);
+    }
+  }
+  const float val = W > 0.f ? acc / W : 0.f;
+  out[(size_t)row * D + e] = static_cast<uint16_t>(pack_bf16x2(val, 0.f) & 0xFFFFu);
+  if (lse && e == 0) lse[row] = W > 0.f ? M + __logf(W) : -INFINITY;
+}
+
 }  // namespace wpattn

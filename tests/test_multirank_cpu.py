@@ -67,3 +67,101 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
         workload, steps, warmup = "tiny", 1, 1
     rank, res = bench.reference_arm(A())
     assert rank == 1 and res is None
+
+
+# ---------------------------------------------------------------------------
+# decode with the cache split by length over ranks: the exchange and merge
+# logic of rope_wavelength_sparsity_b200.distributed on two gloo ranks, with
+# the oracle standing in for the per-shard kernel (CPU only) and a numpy merge
+# ---------------------------------------------------------------------------
+
+def _oracle_shard(q, k_, v_, kv_len, q_pos, k_pos0, win, scale):
+    import numpy as np
+    import torch
+    import oracle
+    from rope_wavelength_sparsity_b200 import inputs
+    B, Hq, D = q.shape
+    L = k_.shape[1]
+    kp = np.array([[k_pos0[b] + j for j in range(L)] for b in range(B)], dtype=np.int64)
+    o, l = oracle.decode_positions(inputs.bits(q), inputs.bits(k_), inputs.bits(v_), kv_len, q_pos,
+                                   kp, Hq=Hq, Hkv=k_.shape[2], base=win.rope_base,
+                                   alpha=win.alpha, g=win.group_pairs, scale=scale)
+    out = torch.tensor(o.reshape(B, Hq, D), dtype=torch.float32).to(torch.bfloat16)
+    return out, torch.tensor(l.reshape(B, Hq), dtype=torch.float32)
+
+
+def _numpy_merge(outs, lses):
+    import numpy as np
+    import torch
+    o = outs.float().numpy().astype(np.float64)
+    l = lses.numpy().astype(np.float64)
+    M = l.max(axis=0)
+    with np.errstate(invalid="ignore"):
+        w = np.where(np.isneginf(l), 0.0, np.exp(l - M))
+    W = w.sum(axis=0)
+    out = np.where(W[..., None] > 0, (w[..., None] * o).sum(axis=0) / np.maximum(W, 1e-300)[..., None], 0.0)
+    lse = np.where(W > 0, M + np.log(np.maximum(W, 1e-300)), -np.inf)
+    return torch.tensor(out), torch.tensor(lse)
+
+
+def _split_worker(rank, world, port, q_out):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    import datetime
+    import torch.distributed as dist
+    import rope_wavelength_sparsity_b200 as wp
+    from rope_wavelength_sparsity_b200 import inputs
+    from rope_wavelength_sparsity_b200 import distributed as wd
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        B, Hq, Hkv, D, shard = 3, 4, 2, 16, 40
+        kv_len = [80, 23, 41]                 # sequence 1 ends inside rank 0's shard
+        q = inputs.randn_bf16((B, Hq, D), 601)
+        kc = inputs.randn_bf16((B, world * shard, Hkv, D), 602)
+        vc = inputs.randn_bf16((B, world * shard, Hkv, D), 603)
+        win = wp.Window(D, 100.0, 1.0, 1)
+        ks = kc[:, rank * shard:(rank + 1) * shard].contiguous()
+        vs = vc[:, rank * shard:(rank + 1) * shard].contiguous()
+        out, lse = wd.decode_kv_split(q, ks, vs, kv_len, win, shard_len=shard, rank=rank,
+                                      world=world, scale=0.25, shard_fn=_oracle_shard,
+                                      merge_fn=_numpy_merge)
+        q_out.put((rank, out.numpy(), lse.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_decode_kv_split_exchange_gloo():
+    import numpy as np
+    import oracle
+    import rope_wavelength_sparsity_b200 as wp
+    from rope_wavelength_sparsity_b200 import inputs
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    procs = [ctx.Process(target=_split_worker, args=(r, world, port, qq)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted((qq.get(timeout=120) for _ in range(world)), key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    B, Hq, Hkv, D, shard = 3, 4, 2, 16, 40
+    kv_len = [80, 23, 41]
+    q = inputs.randn_bf16((B, Hq, D), 601)
+    kc = inputs.randn_bf16((B, world * shard, Hkv, D), 602)
+    vc = inputs.randn_bf16((B, world * shard, Hkv, D), 603)
+    o_ref, l_ref = oracle.decode_rows(inputs.bits(q), inputs.bits(kc), inputs.bits(vc), kv_len,
+                                      Hq=Hq, Hkv=Hkv, base=100.0, alpha=1.0, g=1, scale=0.25)
+    for rank, out, lse in got:                   # every rank holds the whole result
+        np.testing.assert_allclose(out.reshape(-1, D), o_ref, atol=1e-2)   # parts travel as bf16
+        np.testing.assert_allclose(lse.reshape(-1), l_ref, atol=1e-5)
+    assert np.array_equal(got[0][1], got[1][1])
+
+
+def test_shard_keys_bounds():
+    from rope_wavelength_sparsity_b200 import distributed as wd
+    assert wd.shard_keys([100, 30, 0], 0, 40) == ([0, 0, 0], [40, 30, 0])
+    assert wd.shard_keys([100, 30, 0], 1, 40) == ([40, 40, 40], [40, 0, 0])
+    assert wd.shard_keys([100, 30, 0], 2, 40) == ([80, 80, 80], [20, 0, 0])
