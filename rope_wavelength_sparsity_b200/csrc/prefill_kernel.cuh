@@ -565,7 +565,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         nv = min(BN, p.Nk - kp0);
         k_lo = kps[0];
         k_hi = kps[nv - 1];
-        c_caus = col_below(kps, nv, i_pos + 1);
+        // rows at or past the tile's last key attend all of it (no search)
+        c_caus = i_pos >= k_hi ? nv : col_below(kps, nv, i_pos + 1);
       }
       const int d_row = i_pos - (POS ? k_lo : kp0);  // distance to the tile's first key
       const int plo = plo_next, ps = ps_next;
