@@ -737,19 +737,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           const float sgn = sub ? -1.f : 1.f;
           const int grp = gp >> 3;
-          float qv[16];
-          {
-            const uint4 a = *reinterpret_cast<const uint4*>(smem_q + grp * PANEL_Q + r * 16);
-            const uint4 c = *reinterpret_cast<const uint4*>(smem_q + (P / 8 + grp) * PANEL_Q + r * 16);
-            qv[0] = bf16lo_to_f32(a.x); qv[1] = bf16hi_to_f32(a.x);
-            qv[2] = bf16lo_to_f32(a.y); qv[3] = bf16hi_to_f32(a.y);
-            qv[4] = bf16lo_to_f32(a.z); qv[5] = bf16hi_to_f32(a.z);
-            qv[6] = bf16lo_to_f32(a.w); qv[7] = bf16hi_to_f32(a.w);
-            qv[8] = bf16lo_to_f32(c.x); qv[9] = bf16hi_to_f32(c.x);
-            qv[10] = bf16lo_to_f32(c.y); qv[11] = bf16hi_to_f32(c.y);
-            qv[12] = bf16lo_to_f32(c.z); qv[13] = bf16hi_to_f32(c.z);
-            qv[14] = bf16lo_to_f32(c.w); qv[15] = bf16hi_to_f32(c.w);
+          // The group's 16-dim products for this warp's 32 rows on the tensor
+          // cores (mma.sync m16n8k16): A = Q rows (dims 8 grp.. then P + 8 grp..),
+          // B = K rows of the chunk's keys.  Lane (gid, tig) gets rows gid (+8)
+          // and keys 2 tig (+1) of each 16 x 8 block; a per-warp scratch turns
+          // them into one row per lane.  A: matrix m of the ldmatrix = rows
+          // 8 (m & 1) .., first (m < 2) or second half of the group.
+          const int qm = lane >> 3, qi = lane & 7;
+          uint32_t afr[2][4];
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            const int row_a = wq * 32 + 16 * mt + 8 * (qm & 1) + qi;
+            const int pan_a = (qm >> 1) ? P / 8 + grp : grp;
+            ldsm_x4(smem_u32(smem_q) + pan_a * PANEL_Q + row_a * 16, afr[mt][0], afr[mt][1],
+                    afr[mt][2], afr[mt][3]);
           }
+          float* scr = reinterpret_cast<float*>(smem + L::OFF_CT) + warp * (32 * 16);  // [32 rows][16 keys]
 #pragma unroll 1
           for (int cc = 0; cc < BN / 32; ++cc) {
             const int lo = c_lo - 32 * cc, hi = c_hi - 32 * cc;  // chunk-local range
@@ -758,19 +761,45 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tmem_ld32(tS + 32 * cc, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const uint4 a = *reinterpret_cast<const uint4*>(kb + grp * PANEL_K + (32 * cc + c) * 16);
-              const uint4 b2 = *reinterpret_cast<const uint4*>(kb + (P / 8 + grp) * PANEL_K + (32 * cc + c) * 16);
-              float d0 = 0.f, d1 = 0.f;
-              fma2(d0, d1, qv[0], qv[1], bf16lo_to_f32(a.x), bf16hi_to_f32(a.x), d0, d1);
-              fma2(d0, d1, qv[2], qv[3], bf16lo_to_f32(a.y), bf16hi_to_f32(a.y), d0, d1);
-              fma2(d0, d1, qv[4], qv[5], bf16lo_to_f32(a.z), bf16hi_to_f32(a.z), d0, d1);
-              fma2(d0, d1, qv[6], qv[7], bf16lo_to_f32(a.w), bf16hi_to_f32(a.w), d0, d1);
-              fma2(d0, d1, qv[8], qv[9], bf16lo_to_f32(b2.x), bf16hi_to_f32(b2.x), d0, d1);
-              fma2(d0, d1, qv[10], qv[11], bf16lo_to_f32(b2.y), bf16hi_to_f32(b2.y), d0, d1);
-              fma2(d0, d1, qv[12], qv[13], bf16lo_to_f32(b2.z), bf16hi_to_f32(b2.z), d0, d1);
-              fma2(d0, d1, qv[14], qv[15], bf16lo_to_f32(b2.w), bf16hi_to_f32(b2.w), d0, d1);
-              if (c >= lo && c <= hi) v[c] = fmaf(sgn, d0 + d1, v[c]);
+            for (int half = 0; half < 2; ++half) {
+              // B: matrix m = keys 8 (m >> 1) .., first (m even) or second half of the group
+              const int key = 32 * cc + 16 * half + 8 * (qm >> 1) + qi;
+              const int pan_b = (qm & 1) ? P / 8 + grp : grp;
+              uint32_t b00, b01, b10, b11;
+              ldsm_x4(smem_u32(kb) + pan_b * PANEL_K + key * 16, b00, b01, b10, b11);
+              float acc[2][2][4];
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt) {
+                mma_16816_bf16(acc[mt][0], afr[mt][0], afr[mt][1], afr[mt][2], afr[mt][3], b00, b01);
+                mma_16816_bf16(acc[mt][1], afr[mt][0], afr[mt][1], afr[mt][2], afr[mt][3], b10, b11);
+              }
+              __syncwarp();                 // the previous half's rows have been read
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                  const int rr = 16 * mt + (lane >> 2), cl = 8 * nt + 2 * (lane & 3);
+                  *reinterpret_cast<float2*>(scr + rr * 16 + cl) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+                  *reinterpret_cast<float2*>(scr + (rr + 8) * 16 + cl) = make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+                }
+              __syncwarp();
+              const float4* mine = reinterpret_cast<const float4*>(scr + lane * 16);
+#pragma unroll
+              for (int c4 = 0; c4 < 4; ++c4) {
+                const float4 x = mine[c4];
+                const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int c = 16 * half + 4 * c4 + e;
+                  if (c >= lo && c <= hi) v[c] = fmaf(sgn, xs[e], v[c]);
+                }
+              }
             }
             tmem_st32(tS + 32 * cc, v);
           }
