@@ -48,8 +48,8 @@ FLUSH_BYTES = 512 << 20
 # that kernel's sources at capture time: a changed kernel reports null until
 # it is captured again.
 NCU_TRAFFIC = {
-    # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.182272 MB read + 23.981824 MB written
-    ("qwen2.5-0.5b-32k", "8164e7464720ac0c"): 76182272 + 23981824,
+    # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.157440 MB read + 24.292096 MB written
+    ("qwen2.5-0.5b-32k", "978b5944f120cf2a"): 76157440 + 24292096,
     # profiles/decode_split_kernel_llama3.2-3b-decode-32k.md: 536.957696 MB read + 5.210368 MB
     # written for B=4, L=32768, scaled by the 16x keys x heads of the B=16, L=131072 call
     ("llama3.2-3b-decode-128k", "d5ef4dbd68e2bc2c"): 16 * (536957696 + 5210368),
