@@ -58,3 +58,29 @@ def test_decode_workspace_too_small(cuda_dev):
     with pytest.raises(wp.WpattnError) as e:
         wp.decode(q, kc, kc, [L], win, workspace=ws)
     assert e.value.code == wp.EWORKSPACE
+
+
+def test_decode_maximum_batch(cuda_dev):
+    """The largest batch one call takes (1024 sequences), with lengths from 1 to 64:
+    every row against the oracle; one more sequence is refused."""
+    import numpy as np
+    import oracle
+    from _parity import check_rows
+    B, Hq, Hkv, D, L = 1024, 4, 2, 64, 64
+    q = inputs.randn_bf16((B, Hq, D), 81)
+    kc = inputs.randn_bf16((B, L, Hkv, D), 82)
+    vc = inputs.randn_bf16((B, L, Hkv, D), 83)
+    kv_len = [1 + (7 * b) % L for b in range(B)]
+    win = wp.Window(D, 1e4, 1.0, 1)
+    out, lse = wp.decode(q.cuda(), kc.cuda(), vc.cuda(), kv_len, win)
+    assert wp.device_status() == wp.OK
+    o_ref, l_ref = oracle.decode_rows(inputs.bits(q), inputs.bits(kc), inputs.bits(vc), kv_len,
+                                      Hq=Hq, Hkv=Hkv, base=1e4, alpha=1.0, g=1,
+                                      scale=1.0 / D ** 0.5)
+    check_rows(out.float().cpu().reshape(B * Hq, D).numpy(), lse.cpu().reshape(-1).numpy(),
+               o_ref, l_ref, "B=1024")
+    q1 = torch.zeros((B + 1, Hq, D), dtype=torch.bfloat16, device="cuda")
+    k1 = torch.zeros((B + 1, 8, Hkv, D), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(wp.WpattnError) as e:
+        wp.decode(q1, k1, k1, [8] * (B + 1), win)
+    assert e.value.code == wp.EUNSUPPORTED
