@@ -597,115 +597,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!__all_sync(FULL, mbar_wait(k_full(s), (j / NS) & 1))) { ok = false; break; }
       }
       float sc[BN];
-      if (corr && !G8) {
-        const uint8_t* kb = smem + L::OFF_K + s * L::KTILE;
-#pragma unroll
-        for (int c = 0; c < BN; ++c) sc[c] = 0.f;
-        // the chunk loops are not unrolled (this path runs on few tiles and
-        // must stay small in the instruction cache): a chunk's terms are
-        // summed into dl and added to sc by a switch on the chunk index
-#define WPATTN_ADD_CHUNK(K)                                                  \
-  case K:                                                                    \
-    _Pragma("unroll") for (int c = 0; c < 32; ++c) sc[32 * K + c] += dl[c]; \
-    break;
-        // One pair per term.  For each 32-column chunk the warp first
-        // transposes the K values of the pairs its 32 x 32 block needs into
-        // a private buffer (lane k writes key 32 cc + k), so that the
-        // column loop reads four keys per broadcast load.
-        uint32_t* ct = reinterpret_cast<uint32_t*>(smem + L::OFF_CT) + warp * (kCT * 32);
-        const int T_lo = ps > plo ? sT[ps - 1] : 0;
-#pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          if (POS && 32 * cc >= nv) break;                 // no key in this chunk
-          // distance at the chunk's first column
-          const int dc = POS ? i_pos - kps[32 * cc] : d_row - 32 * cc;
-          const int dmax = __shfl_sync(FULL, dc, 31);      // largest distance of the block
-          const int dmin = POS ? max(__shfl_sync(FULL, i_pos - kps[min(32 * cc + 31, nv - 1)], 0), 0)
-                               : max(__shfl_sync(FULL, dc, 0) - 31, 0);
-          if (dmax < 0) continue;                          // wholly acausal
-          // pairs ps .. pb-1 are pruned somewhere in the block, pa .. ps-1 kept somewhere
-          int pb = ps;
-          if (need_sub)
-            while (pb < P && sT[pb] < dmax) ++pb;
-          int pa = ps;
-          if (need_add && T_lo >= dmin)
-            while (pa > plo && sT[pa - 1] >= dmin) --pa;
-          if (pa >= pb) continue;
-          float dl[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) dl[c] = 0.f;
-#pragma unroll 1
-          for (int p0 = pa; p0 < pb; p0 += kCT) {
-            const int p1 = min(pb, p0 + kCT);
-            __syncwarp();  // the previous batch has been read
-            const uint8_t* krow = kb + (32 * cc + lane) * 16;
-#pragma unroll 1
-            for (int pp = p0; pp < p1; ++pp) {
-              const int o = (pp >> 3) * PANEL_K + (pp & 7) * 2;
-              const uint32_t klo = *reinterpret_cast<const uint16_t*>(krow + o);
-              const uint32_t khi = *reinterpret_cast<const uint16_t*>(krow + o + (P / 8) * PANEL_K);
-              ct[(pp - p0) * 32 + lane] = klo | (khi << 16);
-            }
-            __syncwarp();
-#pragma unroll 1
-            for (int pp = p0; pp < p1; ++pp) {
-              const int T = sT[pp];
-              int lo, hi;  // chunk columns of this row that take the pair's term
-              float sgn;
-              if constexpr (POS) {
-                // chunk columns before cth are farther than T
-                const int cth = col_below(kps, nv, i_pos - T) - 32 * cc;
-                if (pp >= ps) {
-                  lo = 0;
-                  hi = min(cth, 32) - 1;
-                  sgn = -1.f;
-                } else {
-                  lo = max(cth, 0);
-                  hi = min(c_caus - 32 * cc, 32) - 1;
-                  sgn = 1.f;
-                }
-              } else if (pp >= ps) {
-                lo = 0;
-                hi = dc > T ? min(dc - T, 32) - 1 : -1;
-                sgn = -1.f;
-              } else {
-                lo = T >= dc ? 0 : dc - T;
-                hi = min(dc, 31);
-                sgn = 1.f;
-              }
-              const int o = (pp >> 3) * PANEL_Q + (pp & 7) * 2 + r * 16;
-              const float qa = sgn * __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + o)) << 16);
-              const float qb = sgn * __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(smem_q + o + (P / 8) * PANEL_Q)) << 16);
-              const uint4* w4 = reinterpret_cast<const uint4*>(ct + (pp - p0) * 32);
-#pragma unroll
-              for (int c4 = 0; c4 < 8; ++c4) {
-                const uint4 w = w4[c4];
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int c = 4 * c4 + e;
-                  const float ka = __uint_as_float(ww[e] << 16);
-                  const float kh = __uint_as_float(ww[e] & 0xFFFF0000u);
-                  if (c >= lo && c <= hi) dl[c] = fmaf(qa, ka, fmaf(qb, kh, dl[c]));
-                }
-              }
-            }
-          }
-          switch (cc) {
-            WPATTN_ADD_CHUNK(0)
-            WPATTN_ADD_CHUNK(1)
-            WPATTN_ADD_CHUNK(2)
-            default:  // chunk 3 (128-key tiles only)
-              if constexpr (BN > 96) {
-#pragma unroll
-                for (int c = 0; c < 32; ++c) sc[96 + c] += dl[c];
-              }
-              break;
-          }
-        }
-#undef WPATTN_ADD_CHUNK
-      }
-      if (!(corr && G8)) {  // K stage s is no longer read by this warp
+      if (!corr) {  // K stage s is no longer read by this warp
         __syncwarp();
         if (lane == 0) mbar_arrive(k_empty(s));
       }
@@ -809,19 +701,130 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (lane == 0) mbar_arrive(k_empty(s));
       }
       if (corr && !G8) {
-#pragma unroll
+        // One pair per term, applied to S in TMEM like the groups above, its
+        // products on the tensor cores: per 32-column chunk, the pairs whose
+        // thresholds fall inside the block's distances; a pair's product is
+        // its group's MMA with every A element but the pair's two dims zeroed.
+        const uint8_t* kb = smem + L::OFF_K + s * L::KTILE;
+        float* scr = reinterpret_cast<float*>(smem + L::OFF_CT) + warp * (32 * 16);  // [32 rows][16 keys]
+        const int qm = lane >> 3, qi = lane & 7;
+        const int T_lo = ps > plo ? sT[ps - 1] : 0;
+#pragma unroll 1
         for (int cc = 0; cc < BN / 32; ++cc) {
+          if (POS && 32 * cc >= nv) break;                 // no key in this chunk
+          // distance at the chunk's first column
+          const int dc = POS ? i_pos - kps[32 * cc] : d_row - 32 * cc;
+          const int dmax = __shfl_sync(FULL, dc, 31);      // largest distance of the block
+          const int dmin = POS ? max(__shfl_sync(FULL, i_pos - kps[min(32 * cc + 31, nv - 1)], 0), 0)
+                               : max(__shfl_sync(FULL, dc, 0) - 31, 0);
+          if (dmax < 0) continue;                          // wholly acausal
+          // pairs ps .. pb-1 are pruned somewhere in the block, pa .. ps-1 kept somewhere
+          int pb = ps;
+          if (need_sub)
+            while (pb < P && sT[pb] < dmax) ++pb;
+          int pa = ps;
+          if (need_add && T_lo >= dmin)
+            while (pa > plo && sT[pa - 1] >= dmin) --pa;
+          if (pa >= pb) continue;
           float v[32];
           tmem_ld32(tS + 32 * cc, v);
           tmem_ld_wait();
+          uint32_t afr[2][4];
+          int cur = -1;
+#pragma unroll 1
+          for (int pp = pa; pp < pb; ++pp) {
+            const int grp = pp >> 3;
+            if (grp != cur) {  // A: this warp's Q rows of the group (matrix m: rows 8 (m & 1) .., half m >> 1)
+              cur = grp;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) sc[32 * cc + c] += v[c];
+              for (int mt = 0; mt < 2; ++mt) {
+                const int row_a = wq * 32 + 16 * mt + 8 * (qm & 1) + qi;
+                const int pan_a = (qm >> 1) ? P / 8 + grp : grp;
+                ldsm_x4(smem_u32(smem_q) + pan_a * PANEL_Q + row_a * 16, afr[mt][0], afr[mt][1],
+                        afr[mt][2], afr[mt][3]);
+              }
+            }
+            const int T = sT[pp];
+            int lo, hi;  // chunk columns of this row that take the pair's term
+            float sgn;
+            if constexpr (POS) {
+              // chunk columns before cth are farther than T
+              const int cth = col_below(kps, nv, i_pos - T) - 32 * cc;
+              if (pp >= ps) {
+                lo = 0;
+                hi = min(cth, 32) - 1;
+                sgn = -1.f;
+              } else {
+                lo = max(cth, 0);
+                hi = min(c_caus - 32 * cc, 32) - 1;
+                sgn = 1.f;
+              }
+            } else if (pp >= ps) {
+              lo = 0;
+              hi = dc > T ? min(dc - T, 32) - 1 : -1;
+              sgn = -1.f;
+            } else {
+              lo = T >= dc ? 0 : dc - T;
+              hi = min(dc, 31);
+              sgn = 1.f;
+            }
+            if (!__any_sync(FULL, lo <= hi)) continue;
+            // keep only the pair's dims: A register halves hold pairs 8 grp + 2 tig (+1)
+            const int jp = pp & 7;
+            const uint32_t keep = ((lane & 3) == (jp >> 1)) ? ((jp & 1) ? 0xFFFF0000u : 0x0000FFFFu) : 0u;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              // B: matrix m = keys 8 (m >> 1) .., first (m even) or second half of the group
+              const int key = 32 * cc + 16 * half + 8 * (qm >> 1) + qi;
+              const int pan_b = (qm & 1) ? P / 8 + grp : grp;
+              uint32_t b00, b01, b10, b11;
+              ldsm_x4(smem_u32(kb) + pan_b * PANEL_K + key * 16, b00, b01, b10, b11);
+              float acc[2][2][4];
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt) {
+                const uint32_t a0 = afr[mt][0] & keep, a1 = afr[mt][1] & keep;
+                const uint32_t a2 = afr[mt][2] & keep, a3 = afr[mt][3] & keep;
+                mma_16816_bf16(acc[mt][0], a0, a1, a2, a3, b00, b01);
+                mma_16816_bf16(acc[mt][1], a0, a1, a2, a3, b10, b11);
+              }
+              __syncwarp();                 // the scratch's previous rows have been read
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                  const int rr = 16 * mt + (lane >> 2), cl = 8 * nt + 2 * (lane & 3);
+                  *reinterpret_cast<float2*>(scr + rr * 16 + cl) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+                  *reinterpret_cast<float2*>(scr + (rr + 8) * 16 + cl) = make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+                }
+              __syncwarp();
+              const float4* mine = reinterpret_cast<const float4*>(scr + lane * 16);
+#pragma unroll
+              for (int c4 = 0; c4 < 4; ++c4) {
+                const float4 x = mine[c4];
+                const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int c = 16 * half + 4 * c4 + e;
+                  if (c >= lo && c <= hi) v[c] = fmaf(sgn, xs[e], v[c]);
+                }
+              }
+            }
+          }
+          tmem_st32(tS + 32 * cc, v);
         }
-      } else {
-#pragma unroll
-        for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(tS + 32 * cc, &sc[32 * cc]);
-        tmem_ld_wait();
+        tmem_st_wait();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(k_empty(s));
       }
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(tS + 32 * cc, &sc[32 * cc]);
+      tmem_ld_wait();
 
       if (all_pruned) {
 #pragma unroll
