@@ -48,8 +48,8 @@ FLUSH_BYTES = 512 << 20
 # that kernel's sources at capture time: a changed kernel reports null until
 # it is captured again.
 NCU_TRAFFIC = {
-    # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.157440 MB read + 24.292096 MB written
-    ("qwen2.5-0.5b-32k", "978b5944f120cf2a"): 76157440 + 24292096,
+    # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.266496 MB read + 26.896128 MB written
+    ("qwen2.5-0.5b-32k", "08e5772bb4e2955c"): 76266496 + 26896128,
     # profiles/decode_split_kernel_llama3.2-3b-decode-32k.md: 536.957696 MB read + 5.210368 MB
     # written for B=4, L=32768, scaled by the 16x keys x heads of the B=16, L=131072 call
     ("llama3.2-3b-decode-128k", "d5ef4dbd68e2bc2c"): 16 * (536957696 + 5210368),
