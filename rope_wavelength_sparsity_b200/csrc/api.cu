@@ -47,6 +47,7 @@ struct DeviceInfo {
   bool init = false;
   bool supported = false;
   int num_sms = 0;
+  int decode_slots = 0;  // decode CTAs resident on the whole GPU at once
   bool prefill_attr[12] = {};  // (D 64, 128) x (g 1, 8) x (plain, block mask, positions)
   void* static_scratch = nullptr;  // device address of g_decode_static_scratch
 };
@@ -67,6 +68,23 @@ int device_info(DeviceInfo** out) {
       return WPATTN_ECUDA;
     d.supported = (major == 10 && minor == 0);
     d.num_sms = sms;
+    if (d.supported) {
+      // resident decode CTAs per SM, limited by the shared-memory ring and by
+      // the registers of the largest instantiation
+      int smem_sm = 0, smem_res = 0, regs_sm = 0;
+      cudaFuncAttributes fa;
+      if (cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&smem_res, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa, decode_split_kernel<128, 8, false>) != cudaSuccess)
+        return WPATTN_ECUDA;
+      const int cta_smem = std::max(DecodeSmem<64>::ALLOC, DecodeSmem<128>::ALLOC) + smem_res;
+      const int warps = kDecodeComputeWarps + 1;
+      const int cta_regs = warps * ((fa.numRegs * 32 + 255) / 256 * 256);
+      int per_sm = std::min(smem_sm / cta_smem, cta_regs > 0 ? regs_sm / cta_regs : 1);
+      if (per_sm < 1) per_sm = 1;
+      d.decode_slots = sms * per_sm;
+    }
     d.init = true;
   }
   *out = &d;
@@ -542,7 +560,7 @@ int decode_impl(const wpattn_window* w, const void* q, const void* k_cache, cons
   }
   DeviceInfo* dev = nullptr;
   if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
-  const int S = decode_splits(B, Hkv, Lmax, dev->num_sms);
+  const int S = decode_splits(B, Hkv, Lmax, dev->decode_slots);
   const size_t need = decode_workspace_bytes(B, Hq, plan.D, S);
   if (!workspace || workspace_bytes < need) return WPATTN_EWORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return WPATTN_EINVAL;
@@ -735,7 +753,7 @@ int wpattn_decode_noalloc(const wpattn_window* w, const void* q, const void* k_c
   DeviceInfo* dev = nullptr;
   if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
   // scratch this problem needs under the current device's split plan
-  const int S = decode_splits(B, Hkv, Lmax, dev->num_sms);
+  const int S = decode_splits(B, Hkv, Lmax, dev->decode_slots);
   if (decode_workspace_bytes(B, Hq, plan.D, S) > kDecodeStaticScratchBytes) return WPATTN_EWORKSPACE;
   {
     // once per device, with that device current: the array's device address

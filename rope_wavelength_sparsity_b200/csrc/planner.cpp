@@ -108,10 +108,10 @@ int decode_max_splits(int B, int Hkv, int64_t max_kv_len) {
   return static_cast<int>(s);
 }
 
-int decode_splits(int B, int Hkv, int64_t max_kv_len, int num_sms) {
+int decode_splits(int B, int Hkv, int64_t max_kv_len, int slots) {
   const int64_t units = static_cast<int64_t>(B) * Hkv;
-  const int64_t target = static_cast<int64_t>(num_sms > 0 ? num_sms : 148) * 4;
-  int64_t s = (target + units - 1) / units;
+  const int64_t target = slots > 0 ? slots : 148 * 3;
+  int64_t s = target / units;
   const int smax = decode_max_splits(B, Hkv, max_kv_len);
   if (s > smax) s = smax;
   if (s < 1) s = 1;

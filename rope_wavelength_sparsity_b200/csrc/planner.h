@@ -54,7 +54,11 @@ struct DecodeSplit {
 };
 
 int decode_max_splits(int B, int Hkv, int64_t max_kv_len);
-int decode_splits(int B, int Hkv, int64_t max_kv_len, int num_sms);
+// Splits per (sequence, kv head) for a GPU that holds `slots` decode CTAs at
+// once (SMs x resident CTAs per SM): at most one wave, since a partial second
+// wave of CTAs that stream the same number of bytes runs at a fraction of the
+// bandwidth and leaves the first wave's SMs idle.
+int decode_splits(int B, int Hkv, int64_t max_kv_len, int slots);
 size_t decode_workspace_bytes(int B, int Hq, int D, int max_splits);
 
 }  // namespace wpattn
