@@ -178,7 +178,9 @@ WPATTN_API int wpattn_pack_block_mask(const uint8_t *mask, uint32_t *words, int6
 /*
  * Bytes of device workspace wpattn_decode needs for up to B sequences of up
  * to max_kv_len keys (0 on bad arguments).  The split of each sequence into
- * key ranges depends only on (B, Hkv, max_kv_len) and the device's SM count.
+ * key ranges depends only on (B, Hkv, max_kv_len) and the device: its SM
+ * count and how many decode CTAs one SM holds at once (the split fills at
+ * most one such wave).  The size returned covers every device.
  */
 WPATTN_API size_t wpattn_decode_workspace_size(const wpattn_window *w, int32_t B, int32_t Hq,
                                     int32_t Hkv, int64_t max_kv_len);
