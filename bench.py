@@ -33,6 +33,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -140,7 +141,9 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        # raw samples: $WPATTN_CLOCK_DIR if set (to keep them), else the temp directory
+        out_dir = os.environ.get("WPATTN_CLOCK_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"wpattn_clocks_rank{device_index}_{os.getpid()}.csv")
 
     def start(self):
         try:
@@ -176,6 +179,11 @@ class ClockSampler:
             for n, val in zip(names, parts[5:9]):
                 if val.lower().startswith("active"):
                     reasons.add(n)
+        if not os.environ.get("WPATTN_CLOCK_DIR"):
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
