@@ -434,6 +434,19 @@ WPATTN_API int wpattn_merge_lse(const void *outs, const float *lses, int32_t R, 
  */
 WPATTN_API int wpattn_device_status(void *cuda_stream);
 
+/*
+ * Self-check of the failure path that every kernel's waits share (the pages
+ * have no counterpart).  Launches one CTA on `cuda_stream` whose only waiting
+ * thread waits on a shared-memory mbarrier that nothing ever arrives at.  The
+ * wait is bounded like every wait in the library's kernels (2 s on the
+ * device's global timer); when the bound runs out the thread records
+ * WPATTN_ETIMEOUT in the device status word and the kernel returns normally,
+ * so the CUDA context stays usable.  The next wpattn_device_status on the
+ * device returns WPATTN_ETIMEOUT (and clears it).  Returns WPATTN_OK once
+ * launched, WPATTN_EUNSUPPORTED off sm_100, WPATTN_ECUDA on a launch error.
+ */
+WPATTN_API int wpattn_selftest_wait_timeout(void *cuda_stream);
+
 /* Static English text for a status code. */
 WPATTN_API const char *wpattn_strerror(int code);
 

@@ -96,6 +96,7 @@ def lib() -> ctypes.CDLL:
         L.wpattn_decode_paged.argtypes = [wp, vp, vp, vp, i32, i32, vp, i32, i32p, i32p, vp, i64,
                                           i32, i32, i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
         L.wpattn_device_status.argtypes = [vp]
+        L.wpattn_selftest_wait_timeout.argtypes = [vp]
         L.wpattn_strerror.restype = ctypes.c_char_p
         L.wpattn_strerror.argtypes = [ctypes.c_int]
         L.wpattn_version.restype = ctypes.c_char_p
@@ -551,6 +552,13 @@ def decode_noalloc_max_bytes() -> int:
 def device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the kernels' status word."""
     return int(lib().wpattn_device_status(_stream_ptr(stream)))
+
+
+def selftest_wait_timeout(stream=None) -> None:
+    """Launch the library's bounded-wait self-check: one kernel waits on a
+    barrier nothing arrives at until its 2 s bound runs out, then records
+    WPATTN_ETIMEOUT for the next ``device_status``."""
+    _check(lib().wpattn_selftest_wait_timeout(_stream_ptr(stream)), "wpattn_selftest_wait_timeout")
 
 
 def default_scale(D: int) -> float:

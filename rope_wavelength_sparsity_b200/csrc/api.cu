@@ -278,6 +278,23 @@ int launch_decode(const DecodeParams& prm, int gc, bool pm, cudaStream_t st) {
 constexpr size_t kDecodeStaticScratchBytes = size_t(4) << 20;  // 4 MiB
 static __device__ __align__(256) unsigned char g_decode_static_scratch[kDecodeStaticScratchBytes];
 
+namespace wpattn {
+// One thread waits on an mbarrier that nothing arrives at: the bounded wait
+// runs out, records WPATTN_ETIMEOUT and the kernel returns (the failure path
+// of every wait in the library's kernels, exercised without a fault).
+__global__ void selftest_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(b, 0);
+  __syncthreads();
+}
+}  // namespace wpattn
+
 using namespace wpattn;
 
 extern "C" {
@@ -768,6 +785,14 @@ int wpattn_decode_noalloc(const wpattn_window* w, const void* q, const void* k_c
   }
   return wpattn_decode(w, q, k_cache, v_cache, kv_len_host, Lmax, B, Hq, Hkv, softmax_scale, out,
                        lse, dev->static_scratch, kDecodeStaticScratchBytes, cuda_stream);
+}
+
+int wpattn_selftest_wait_timeout(void* cuda_stream) {
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc != WPATTN_OK) return rc;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(cuda_stream)>>>();
+  return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
 int wpattn_device_status(void* cuda_stream) {
