@@ -3,6 +3,7 @@
 // maps and kernel launches.  Every step of the computation runs in the
 // kernels of decode_kernels.cuh and prefill_kernel.cuh.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -48,7 +49,9 @@ struct DeviceInfo {
   bool supported = false;
   int num_sms = 0;
   int decode_slots = 0;  // decode CTAs resident on the whole GPU at once
-  bool prefill_attr[12] = {};  // (D 64, 128) x (g 1, 8) x (plain, block mask, positions)
+  // shared-memory attribute set, per prefill instantiation: (D 64, 128) x (g 1, 8) x
+  // (plain, block mask, positions); atomic because host threads may launch concurrently
+  std::atomic<bool> prefill_attr[12] = {};
   void* static_scratch = nullptr;  // device address of g_decode_static_scratch
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -167,11 +170,11 @@ int launch_prefill(const void* q, const void* k, const void* v, PrefillParams pr
   const int slot = (D == 64 ? 0 : 6) + (G8 ? 3 : 0) + (MASK ? 1 : 0) + (POS ? 2 : 0);
   // a mask bit covers one 128-row query tile x one 128-key tile
   if (MASK && (Shape::BN != 128 || kBM != 128)) return WPATTN_EUNSUPPORTED;
-  if (!dev->prefill_attr[slot]) {
+  if (!dev->prefill_attr[slot].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(prefill_kernel<D, G8, MASK, POS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
       return WPATTN_ECUDA;
-    dev->prefill_attr[slot] = true;
+    dev->prefill_attr[slot].store(true, std::memory_order_release);
   }
   dim3 grid(prm.num_ctas_q, prm.Hq, prm.B);
   prefill_kernel<D, G8, MASK, POS><<<grid, Shape::THREADS, smem, st>>>(tq, tk, tv, prm);
@@ -198,14 +201,14 @@ template <int D, int GC, bool PM>
 int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& prm,
                         cudaStream_t st) {
   constexpr int smem = DecodeSmem<D>::ALLOC;
-  static bool attr_set[kMaxDevices] = {};
+  static std::atomic<bool> attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WPATTN_ECUDA;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(decode_split_kernel<D, GC, PM>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return WPATTN_ECUDA;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   dim3 grid(prm.S, prm.Hkv * prm.hchunks, prm.B);
   decode_split_kernel<D, GC, PM><<<grid, (kDecodeComputeWarps + 1) * 32, smem, st>>>(tk, tv, prm);
