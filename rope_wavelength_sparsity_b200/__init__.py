@@ -152,6 +152,28 @@ def _dev_tensor(t, name):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _shape(t, name, shape, dtype=None):
+    """Check a tensor's shape (and dtype) before its pointer reaches a kernel: the C
+    interface takes sizes, not buffers, so a short buffer would be read or written
+    past its end."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, not {t.dtype}")
+
+
+def _f32_out(t, name, shape, like):
+    """An fp32 output buffer: shape, dtype, contiguity and device of `like`."""
+    import torch
+    _shape(t, name, shape, torch.float32)
+    if not t.is_contiguous() or t.device != like.device:
+        raise TypeError(f"{name} must be contiguous and on {like.device}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
 def prefill(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0, scale: float | None = None,
             out=None, lse=None, want_lse: bool = True, stream=None):
     """Windowed causal prefill.  q [B,Nq,Hq,D], k/v [B,Nk,Hkv,D] bf16 CUDA tensors.
@@ -159,8 +181,18 @@ def prefill(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0, scale: floa
     Returns (out [B,Nq,Hq,D] bf16, lse [B,Hq,Nq] fp32 or None).
     """
     import torch
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be 4-D: [B, N, H, D]")
     B, Nq, Hq, D = q.shape
     Nk, Hkv = k.shape[1], k.shape[2]
+    if D != w.head_dim:
+        raise ValueError(f"q has head dim {D}, the window {w.head_dim}")
+    _shape(k, "k", (B, Nk, Hkv, D))
+    _shape(v, "v", (B, Nk, Hkv, D))
+    if out is not None:
+        _shape(out, "out", q.shape)
+    if lse is not None:
+        _f32_out(lse, "lse", (B, Hq, Nq), q)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
@@ -311,8 +343,20 @@ def decode(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | None = None
     Returns (out [B,Hq,D] bf16, lse [B,Hq] fp32 or None).
     """
     import torch
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be [B, Hq, D] and k_cache [B, L, Hkv, D]")
     B, Hq, D = q.shape
     L, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if D != w.head_dim:
+        raise ValueError(f"q has head dim {D}, the window {w.head_dim}")
+    _shape(k_cache, "k_cache", (B, L, Hkv, D))
+    _shape(v_cache, "v_cache", (B, L, Hkv, D))
+    if len(kv_len) != B:
+        raise ValueError(f"kv_len has {len(kv_len)} entries for {B} sequences")
+    if out is not None:
+        _shape(out, "out", q.shape)
+    if lse is not None:
+        _f32_out(lse, "lse", (B, Hq), q)
     kvl = (ctypes.c_int32 * B)(*[int(x) for x in kv_len])
     if workspace is None:
         n = decode_workspace_size(w, B, Hq, Hkv, L)
