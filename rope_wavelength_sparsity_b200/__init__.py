@@ -174,13 +174,9 @@ def _f32_out(t, name, shape, like):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def prefill(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0, scale: float | None = None,
-            out=None, lse=None, want_lse: bool = True, stream=None):
-    """Windowed causal prefill.  q [B,Nq,Hq,D], k/v [B,Nk,Hkv,D] bf16 CUDA tensors.
-
-    Returns (out [B,Nq,Hq,D] bf16, lse [B,Hq,Nq] fp32 or None).
-    """
-    import torch
+def _prefill_shapes(q, k, v, w, out, lse):
+    """(B, Nq, Hq, D, Nk, Hkv) of a prefill call, after checking that q, k, v and any
+    caller-supplied out / lse agree with them and with the window's head dim."""
     if q.dim() != 4 or k.dim() != 4:
         raise ValueError("q and k must be 4-D: [B, N, H, D]")
     B, Nq, Hq, D = q.shape
@@ -193,6 +189,17 @@ def prefill(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0, scale: floa
         _shape(out, "out", q.shape)
     if lse is not None:
         _f32_out(lse, "lse", (B, Hq, Nq), q)
+    return B, Nq, Hq, D, Nk, Hkv
+
+
+def prefill(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0, scale: float | None = None,
+            out=None, lse=None, want_lse: bool = True, stream=None):
+    """Windowed causal prefill.  q [B,Nq,Hq,D], k/v [B,Nk,Hkv,D] bf16 CUDA tensors.
+
+    Returns (out [B,Nq,Hq,D] bf16, lse [B,Hq,Nq] fp32 or None).
+    """
+    import torch
+    B, Nq, Hq, D, Nk, Hkv = _prefill_shapes(q, k, v, w, out, lse)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
@@ -238,8 +245,7 @@ def prefill_masked(q, k, v, block_mask, w: Window, *, q_pos0: int = 0, k_pos0: i
     packed int32 words from ``pack_block_mask``.
     """
     import torch
-    B, Nq, Hq, D = q.shape
-    Nk, Hkv = k.shape[1], k.shape[2]
+    B, Nq, Hq, D, Nk, Hkv = _prefill_shapes(q, k, v, w, out, lse)
     if block_mask.dtype != torch.int32:
         block_mask = pack_block_mask(block_mask, stream=stream)
     nqb = (Nq + MASK_BLOCK - 1) // MASK_BLOCK
@@ -281,8 +287,7 @@ def prefill_rope(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0,
     """``prefill`` from q and k before their RoPE rotation (rotated with w.rope_base at
     q_pos0 + t and k_pos0 + j into a workspace first)."""
     import torch
-    B, Nq, Hq, D = q.shape
-    Nk, Hkv = k.shape[1], k.shape[2]
+    B, Nq, Hq, D, Nk, Hkv = _prefill_shapes(q, k, v, w, out, lse)
     if workspace is None:
         n = int(lib().wpattn_prefill_rope_workspace_size(B, Nq, Nk, Hq, Hkv, D))
         workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
@@ -307,8 +312,7 @@ def prefill_positions(q, k, v, q_pos, k_pos, w: Window, *, scale: float | None =
     int32 CUDA [B, >= Nk], non-decreasing along each sequence.  k_pos is copied into a
     16-byte aligned array padded to a multiple of 128 keys when it is not one already."""
     import torch
-    B, Nq, Hq, D = q.shape
-    Nk, Hkv = k.shape[1], k.shape[2]
+    B, Nq, Hq, D, Nk, Hkv = _prefill_shapes(q, k, v, w, out, lse)
     _int32_dev(q_pos, "q_pos")
     _int32_dev(k_pos, "k_pos")
     padded = max(128, -(-Nk // 128) * 128)
@@ -336,13 +340,9 @@ def decode_workspace_size(w: Window, B: int, Hq: int, Hkv: int, max_kv_len: int)
     return int(lib().wpattn_decode_workspace_size(ctypes.byref(w._c()), B, Hq, Hkv, max_kv_len))
 
 
-def decode(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | None = None, out=None,
-           lse=None, want_lse: bool = True, workspace=None, stream=None):
-    """Windowed decode.  q [B,Hq,D]; caches [B,L,Hkv,D] bf16 CUDA; kv_len: host ints [B].
-
-    Returns (out [B,Hq,D] bf16, lse [B,Hq] fp32 or None).
-    """
-    import torch
+def _decode_shapes(q, k_cache, v_cache, kv_len, w, out, lse):
+    """(B, Hq, D, L, Hkv) of a decode over a contiguous cache, after checking that the
+    caches, kv_len and any caller-supplied out / lse agree with q and the window."""
     if q.dim() != 3 or k_cache.dim() != 4:
         raise ValueError("q must be [B, Hq, D] and k_cache [B, L, Hkv, D]")
     B, Hq, D = q.shape
@@ -357,6 +357,17 @@ def decode(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | None = None
         _shape(out, "out", q.shape)
     if lse is not None:
         _f32_out(lse, "lse", (B, Hq), q)
+    return B, Hq, D, L, Hkv
+
+
+def decode(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | None = None, out=None,
+           lse=None, want_lse: bool = True, workspace=None, stream=None):
+    """Windowed decode.  q [B,Hq,D]; caches [B,L,Hkv,D] bf16 CUDA; kv_len: host ints [B].
+
+    Returns (out [B,Hq,D] bf16, lse [B,Hq] fp32 or None).
+    """
+    import torch
+    B, Hq, D, L, Hkv = _decode_shapes(q, k_cache, v_cache, kv_len, w, out, lse)
     kvl = (ctypes.c_int32 * B)(*[int(x) for x in kv_len])
     if workspace is None:
         n = decode_workspace_size(w, B, Hq, Hkv, L)
@@ -420,6 +431,10 @@ def decode_pairmajor(q, k_slabs, v_cache, kv_len, w: Window, *, scale: float | N
 
 def _decode_outputs(q, w, B, Hq, Hkv, cap, out, lse, want_lse, workspace):
     import torch
+    if out is not None:
+        _shape(out, "out", q.shape)
+    if lse is not None:
+        _f32_out(lse, "lse", (B, Hq), q)
     if workspace is None:
         n = decode_workspace_size(w, B, Hq, Hkv, cap)
         if n == 0:
@@ -567,8 +582,7 @@ def decode_noalloc(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | Non
     (``decode_noalloc_max_bytes()``), calls on one device share it.
     """
     import torch
-    B, Hq, D = q.shape
-    L, Hkv = k_cache.shape[1], k_cache.shape[2]
+    B, Hq, D, L, Hkv = _decode_shapes(q, k_cache, v_cache, kv_len, w, out, lse)
     kvl = (ctypes.c_int32 * B)(*[int(x) for x in kv_len])
     if out is None:
         out = torch.empty_like(q)

@@ -77,3 +77,20 @@ def test_decode_rejects_inconsistent_buffers(what):
     with pytest.raises((ValueError, TypeError)) as e:
         wp.decode(q, kc, vc, kv_len, win, **kw)
     assert "CUDA" not in str(e.value)
+
+
+@pytest.mark.parametrize("fn", ["prefill_masked", "prefill_rope", "prefill_positions"])
+def test_prefill_variants_check_shapes_first(fn):
+    q, k, v = _bf16(1, 10, 4, 64), _bf16(1, 12, 2, 64), _bf16(1, 11, 2, 64)   # v too short
+    mask = torch.ones((1, 4, 1, 1), dtype=torch.bool)
+    pos = torch.zeros((1, 16), dtype=torch.int32)
+    args = {"prefill_masked": (q, k, v, mask, WIN), "prefill_rope": (q, k, v, WIN),
+            "prefill_positions": (q, k, v, pos, pos, WIN)}[fn]
+    with pytest.raises(ValueError, match="v has shape"):
+        getattr(wp, fn)(*args)
+
+
+def test_decode_variant_outputs_are_checked():
+    q, kc, vc = _bf16(2, 4, 64), _bf16(2, 50, 2, 64), _bf16(2, 50, 2, 64)
+    with pytest.raises(ValueError, match="lse has shape"):
+        wp.decode_noalloc(q, kc, vc, [50, 7], WIN, lse=torch.zeros((2, 5), dtype=torch.float32))
