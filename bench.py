@@ -2,13 +2,18 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-One step is one pass of the hot path over one batch of synthetic input:
-the host planner (thresholds, tile plan) and the windowed prefill kernel of
-the chosen workload, called through the C ABI.  The default workload is the
-Qwen2.5-0.5B-shaped single-layer prefill (B=1, Hq=14, Hkv=2, D=64, N=32768,
-base 1e6, alpha 1, g = 8 pairs).  The same run also times the Llama-3.2-3B-
-shaped decode step (B=16, Hq=24, Hkv=8, D=128, L=131072) for the decode
-KV GB/s half of the metric, and the same kernels with the window off.
+One step is one pass of the hot path over one batch of synthetic input: the
+host planner (thresholds, tile plan) and the windowed prefill kernel of the
+chosen workload, called through the C ABI.  The default workload is the
+largest single-GPU one: the Qwen2.5-7B-1M-shaped prefill of the last 16384
+queries against 1,048,576 causal keys (Hq=28, Hkv=4, D=128, base 1e7,
+alpha 1, g = 8 pairs).  The same run times the other workloads as nested
+objects under "configs", each with its roofline, window-off speedup and
+end-to-end figure: the Qwen2.5-0.5B-shaped 32K prefill (with the block-mask,
+pre-RoPE and explicit-positions variants), the Llama-3.2-3B-shaped 128K
+prefill at alpha 1 and 2, and the Llama-3.2-3B-shaped (B=16, L=128K) and
+Qwen2.5-7B-shaped (B=1, L=1M) decodes with their pair-major and paged
+layouts.
 
 Metric: effective TFLOP/s = (4 * kept QK pair-terms + 2 * D * causal
 (query, key) pairs) per (batch, query head), over the device time of the
@@ -21,38 +26,43 @@ Timing: CUDA events on the launching stream around every step, an L2 flush
 runs its own independent problem (weak scaling, no data-path collective).
 
 ``--impl reference`` times the oracle (the plain CPU definition) on a bounded
-sample of rows of the same workload, in the same metric.
+sample of rows of the same workload, in the same metric, on the host's cores.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
+import itertools
 import json
-import math
 import os
 import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "effective TFLOP/s (kept QK terms + PV) and decode KV GB/s, % of B200 roofline"
-DEFAULT_WORKLOAD = "qwen2.5-0.5b-32k"
-DECODE_WORKLOAD = "llama3.2-3b-decode-128k"
+DEFAULT_WORKLOAD = "qwen2.5-7b-1m-prefill"
+# the other workloads, timed as nested objects of the default line
+NESTED_PREFILL = ("qwen2.5-0.5b-32k", "llama3.2-3b-128k-a1", "llama3.2-3b-128k-a2")
+NESTED_DECODE = ("llama3.2-3b-decode-128k", "qwen2.5-7b-1m-decode")
+# the block-mask, pre-RoPE and explicit-positions variants run on this one
+VARIANTS_WORKLOAD = "qwen2.5-0.5b-32k"
 FLUSH_BYTES = 512 << 20
 
-# DRAM bytes (read + write) per launch of the dominant kernel from one ncu
-# capture (profiles/ holds the summaries), keyed by workload and by a hash of
-# that kernel's sources at capture time: a changed kernel reports null until
-# it is captured again.
+# DRAM bytes (read + write) per launch of a workload's dominant kernel from one
+# ncu capture, keyed by workload and by a hash of that kernel's sources at
+# capture time: a changed kernel reports null until it is captured again.
 NCU_TRAFFIC = {
-    # profiles/prefill_kernel_qwen2.5-0.5b-32k.md: 76.266496 MB read + 26.896128 MB written
+    # prefill_kernel<64, g8> on the Qwen2.5-0.5B 32K workload: 76.266496 MB read + 26.896128 MB
+    # written
     ("qwen2.5-0.5b-32k", "08e5772bb4e2955c"): 76266496 + 26896128,
-    # profiles/decode_split_kernel_llama3.2-3b-decode-32k.md: 536.940032 MB read + 3.973632 MB
-    # written for B=4, L=32768, scaled by the 16x keys x heads of the B=16, L=131072 call
+    # decode_split_kernel<128, 3, 0> on the reduced B=4, L=32768 Llama decode: 536.940032 MB read
+    # + 3.973632 MB written, scaled by the 16x keys x heads of the B=16, L=131072 call
     ("llama3.2-3b-decode-128k", "bdf11727c8e434b8"): 16 * (536940032 + 3973632),
 }
 
@@ -79,6 +89,21 @@ def load_peaks():
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                 "source": "fallback"}
+
+
+def workload_config(w, world: int) -> dict:
+    """The `config` object of a workload's line (the same for both arms)."""
+    if w.kind == "prefill":
+        return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                "Nq": w.Nq, "Nk": w.Nk, "q_pos0": w.q_pos0, "rope_base": w.base,
+                "alpha": w.alpha, "group_pairs": w.g, "global_batch": w.B * world,
+                "seq_len": w.Nk, "parallelism": f"independent problem per GPU x{world}",
+                "l2": "flushed between steps (512 MiB write)"}
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.Nk,
+            "rope_base": w.base, "alpha": w.alpha, "group_pairs": w.g,
+            "global_batch": w.B * world, "seq_len": w.Nk,
+            "parallelism": f"independent problem per GPU x{world}",
+            "l2": "flushed between steps (512 MiB write)"}
 
 
 # ----------------------------------------------------------- work accounting
@@ -126,10 +151,22 @@ def decode_bytes(w, win, wp, kv_len):
     return kbytes + vbytes + io, kfull + vbytes + io
 
 
-def row_flops(w, win, wp, t):
-    pruned, total, _ = wp.pruned_fraction(win, 1, w.Nk, w.q_pos0 + t, w.k_pos0)
+def row_flops_oracle(w, t):
+    """Effective FLOPs of prefill query row t of workload w, counted with the oracle's
+    own row-wise count (so that the oracle arm shares no code with the product)."""
+    import oracle
+    pruned, total = oracle.count_rows(w.D, w.base, w.alpha, w.g, 1, w.Nk, w.q_pos0 + t,
+                                      w.k_pos0)
     P = w.D // 2
     return 4 * (total - pruned) + 2 * w.D * (total // P)
+
+
+def decode_row_bytes_oracle(w, L):
+    """Algorithmic bytes of one decode (sequence, query head) row over L keys, counted with
+    the oracle's row-wise count: the group's K slice and V, shared by its G query heads."""
+    import oracle
+    pruned, total = oracle.count_rows(w.D, w.base, w.alpha, w.g, 1, L, L - 1, 0)
+    return ((total - pruned) * 4 + L * w.D * 2) / (w.Hq // w.Hkv)
 
 
 # ------------------------------------------------------------------ clocks
@@ -232,8 +269,9 @@ def _barrier(world):
     torch.cuda.synchronize()
 
 
-def time_steps(step, n_warm, n_steps, flush, world, clocks=None, per_step_events=True):
-    """Device time (ms) of n_steps calls of step(); L2 flushed before each."""
+def time_steps(step, n_warm, n_steps, flush, world, clocks=None):
+    """Device time (ms) of n_steps calls of step(); L2 flushed before each.
+    Returns (max over ranks of the summed step times, per-step times, clock record)."""
     import torch
     for _ in range(n_warm):
         flush()
@@ -252,219 +290,199 @@ def time_steps(step, n_warm, n_steps, flush, world, clocks=None, per_step_events
     _barrier(world)
     clk = clocks.stop() if clocks else None
     per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total = sum(per)
-    return _max_over_ranks(total, world), per, clk
+    return _max_over_ranks(sum(per), world), per, clk
 
 
-def gpu_arm(args):
+def _tensor_peak(peaks, clk):
+    """(peak TFLOP/s, label): the sustained GEMM figure for a kernel that ran under the
+    power cap (its clock samples saw sw_power_cap), else the burst one."""
+    capped = bool(clk) and "sw_power_cap" in (clk.get("reasons") or [])
+    if capped and peaks.get("bf16_tflops_sustained"):
+        return peaks["bf16_tflops_sustained"], f"{peaks['source']} bf16 dense (sustained, sw_power_cap active)"
+    return peaks["bf16_tflops"], f"{peaks['source']} bf16 dense (burst)"
+
+
+def _check_status(wp, what):
+    if wp.device_status() != wp.OK:
+        raise RuntimeError(f"{what}: kernel status not ok")
+
+
+def bench_prefill(w, args, world, rank, dev, flush, peaks, variants=False):
+    """One prefill workload: the windowed call, the same call with the window off, and
+    the end-to-end call with host buffers; with ``variants`` also the block-mask,
+    pre-RoPE and explicit-positions variants of the same problem."""
     import torch
     import rope_wavelength_sparsity_b200 as wp
     from rope_wavelength_sparsity_b200 import inputs
-
-    world, rank, local = _dist_setup(args)
-    dev = torch.device("cuda", local if world > 1 else 0)
-    peaks = load_peaks()
-    w = inputs.WORKLOADS[args.workload]
     win = wp.Window(w.D, w.base, w.alpha, w.g)
     win_off = wp.Window(w.D, w.base, float("inf"), w.g)
-    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    q, k, v, _ = inputs.prefill_inputs(w, seed=rank, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    eff, off_flops = prefill_flops(w, win, wp)
 
-    def flush():
-        flush_buf.fill_(1)
+    def step():
+        wp.prefill(q, k, v, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale, out=out, lse=lse)
 
-    result = {}
-    if w.kind == "prefill":
-        q, k, v, _ = inputs.prefill_inputs(w, seed=rank, device=dev)
-        out = torch.empty_like(q)
-        lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
-        eff, off_flops = prefill_flops(w, win, wp)
+    def step_off():
+        wp.prefill(q, k, v, win_off, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale, out=out,
+                   lse=lse)
 
-        def step():
-            wp.prefill(q, k, v, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale, out=out,
-                       lse=lse)
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    total_ms, per, clk = time_steps(step, args.warmup, args.steps, flush, world, clocks)
+    _check_status(wp, w.name)
+    n_off = max(3, args.steps // 4)
+    off_ms, _, _ = time_steps(step_off, args.warmup, n_off, flush, world)
+    _check_status(wp, w.name + " window off")
+    ms_step = total_ms / args.steps
+    off_ms_step = off_ms / n_off
+    kernel_ms = statistics.mean(per)
+    achieved = eff / (kernel_ms * 1e-3) / 1e12
+    peak_t, peak_label = _tensor_peak(peaks, clk)
+    res = {
+        "metric": METRIC, "value": round(weak_scaling_value(eff, world, ms_step) / 1e12, 2),
+        "unit": "TFLOP/s", "ms_per_step": round(ms_step, 4), "dtype": "bf16",
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_t,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak_t, 4),
+                     "traffic": NCU_TRAFFIC.get((w.name, kernel_source_hash("prefill"))),
+                     "peak_source": peak_label},
+        "window_off": {"ms_per_step": round(off_ms_step, 4),
+                       "speedup": round(off_ms_step / ms_step, 3),
+                       "ideal_speedup": round(off_flops / eff, 3),
+                       "effective_tflops_at_window_off_time": round(eff / (off_ms_step * 1e-3) / 1e12, 2)},
+        "work": {"effective_tflop_per_step": round(world * eff / 1e12, 4),
+                 "window_off_tflop_per_step": round(world * off_flops / 1e12, 4),
+                 "pruned_fraction": wp.pruned_fraction(win, w.Nq, w.Nk, w.q_pos0, w.k_pos0)[2]},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "config": workload_config(w, world),
+    }
+    if variants:
+        res.update(_prefill_variants(w, args, world, rank, dev, flush, peaks, q, k, v, out, lse,
+                                     win, eff, ms_step))
+    # end to end through the public API with pinned host buffers
+    qh = q.cpu().pin_memory()
+    kh = k.cpu().pin_memory()
+    vh = v.cpu().pin_memory()
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
 
-        def step_off():
-            wp.prefill(q, k, v, win_off, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale, out=out,
-                       lse=lse)
+    def step_e2e():
+        qd = q.copy_(qh, non_blocking=True)
+        kd = k.copy_(kh, non_blocking=True)
+        vd = v.copy_(vh, non_blocking=True)
+        o, _ = wp.prefill(qd, kd, vd, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale,
+                          out=out, lse=lse)
+        oh.copy_(o, non_blocking=True)
 
-        clocks = ClockSampler(dev.index) if rank == 0 else None
-        total_ms, per, clk = time_steps(step, args.warmup, args.steps, flush, world, clocks)
-        if wp.device_status() != wp.OK:
-            raise RuntimeError("kernel status: timeout")
-        off_ms, _, _ = time_steps(step_off, args.warmup, max(3, args.steps // 4), flush, world)
-        off_ms_step = off_ms / max(3, args.steps // 4)
-        ms_step = total_ms / args.steps
-        masked = rope_res = positions_res = None
-        if not args.only_primary:
-            # the same call under a MInference-shaped block mask (vertical + slash tiles)
-            mask = inputs.vertical_slash_mask(w.B, w.Hq, w.Nq, w.Nk, seed=rank, q_pos0=w.q_pos0,
-                                              k_pos0=w.k_pos0)
-            words = wp.pack_block_mask(mask.to(dev))
-            m_eff = masked_flops(w, win, wp, mask)
-
-            def step_masked():
-                wp.prefill_masked(q, k, v, words, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0,
-                                  scale=w.scale, out=out, lse=lse)
-
-            n_m = max(3, args.steps // 2)
-            m_ms, m_per, _ = time_steps(step_masked, args.warmup, n_m, flush, world)
-            if wp.device_status() != wp.OK:
-                raise RuntimeError("masked prefill kernel status: not ok")
-            m_kernel = statistics.mean(m_per)
-            causal_tiles = sum(1 for qb in range(mask.shape[2]) for kb in range(mask.shape[3])
-                               if kb * 128 + w.k_pos0 <= w.q_pos0 + qb * 128 + 127)
-            masked = {
-                "value": round(weak_scaling_value(m_eff, world, m_ms / n_m) / 1e12, 2),
-                "unit": "TFLOP/s", "ms_per_step": round(m_ms / n_m, 4),
-                "roofline": {"bound": "tensor", "achieved": round(m_eff / (m_kernel * 1e-3) / 1e12, 2),
-                             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                             "frac": round(m_eff / (m_kernel * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
-                             "traffic": None},
-                "speedup_vs_unmasked": round(ms_step / (m_ms / n_m), 3),
-                "ideal_speedup": round(eff / m_eff, 3),
-                "attended_tile_fraction": round(float(mask.sum()) / (w.B * w.Hq * causal_tiles), 4),
-                "mask": "vertical-slash: sink + 3 random key tiles per head, 16-tile diagonal band",
-            }
-            del words, mask
-            # the same prefill from pre-RoPE q and k: rotation pre-pass + attention,
-            # and the rotation kernel alone (HBM-bound: read and write q and k once)
-            ws_r = torch.empty(max(1, int(wp.lib().wpattn_prefill_rope_workspace_size(
-                w.B, w.Nq, w.Nk, w.Hq, w.Hkv, w.D))), dtype=torch.uint8, device=dev)
-            qr_buf = torch.empty_like(q)
-            kr_buf = torch.empty_like(k)
-
-            def step_rope_prefill():
-                wp.prefill_rope(q, k, v, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale,
-                                out=out, lse=lse, workspace=ws_r)
-
-            def step_rope_only():
-                wp.rope(q, base=w.base, pos0=w.q_pos0, out=qr_buf)
-                wp.rope(k, base=w.base, pos0=w.k_pos0, out=kr_buf)
-
-            n_r = max(3, args.steps // 2)
-            rp_ms, _, _ = time_steps(step_rope_prefill, args.warmup, n_r, flush, world)
-            ro_ms, ro_per, _ = time_steps(step_rope_only, args.warmup, n_r, flush, world)
-            if wp.device_status() != wp.OK:
-                raise RuntimeError("rope kernels status: not ok")
-            rope_bytes = 2 * 2 * (q.numel() + k.numel())
-            ro_gbs = rope_bytes / (statistics.mean(ro_per) * 1e-3) / 1e9
-            rope_res = {
-                "prefill_from_prerope": {"ms_per_step": round(rp_ms / n_r, 4),
-                                         "value": round(weak_scaling_value(eff, world, rp_ms / n_r) / 1e12, 2),
-                                         "unit": "TFLOP/s",
-                                         "overhead_vs_prefill": round((rp_ms / n_r) / ms_step - 1.0, 4)},
-                "rotation_kernels": {"ms_per_step": round(ro_ms / n_r, 4),
-                                     "roofline": {"bound": "hbm", "achieved": round(ro_gbs, 1),
-                                                  "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                                  "frac": round(ro_gbs / peaks["hbm_gbs"], 4),
-                                                  "traffic": None},
-                                     "bytes_per_step": rope_bytes},
-            }
-            del ws_r, qr_buf, kr_buf
-            # the same prefill through the explicit-positions kernel, given the workload's
-            # own contiguous positions (same work; the cost of the searched column ranges)
-            qp = (w.q_pos0 + torch.arange(w.Nq, dtype=torch.int32, device=dev)).repeat(w.B, 1)
-            kp = (w.k_pos0 + torch.arange(w.Nk, dtype=torch.int32, device=dev)).repeat(w.B, 1)
-
-            def step_pos():
-                wp.prefill_positions(q, k, v, qp, kp, win, scale=w.scale, out=out, lse=lse)
-
-            pos_ms, pos_per, _ = time_steps(step_pos, args.warmup, n_r, flush, world)
-            if wp.device_status() != wp.OK:
-                raise RuntimeError("positions prefill status: not ok")
-            pos_ach = eff / (statistics.mean(pos_per) * 1e-3) / 1e12
-            positions_res = {
-                "value": round(weak_scaling_value(eff, world, pos_ms / n_r) / 1e12, 2),
-                "unit": "TFLOP/s", "ms_per_step": round(pos_ms / n_r, 4),
-                "roofline": {"bound": "tensor", "achieved": round(pos_ach, 2),
-                             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                             "frac": round(pos_ach / peaks["bf16_tflops"], 4), "traffic": None},
-                "slowdown_vs_plain": round((pos_ms / n_r) / ms_step, 3),
-                "positions": "the workload's contiguous positions passed as int32 arrays",
-            }
-            del qp, kp
-        value = weak_scaling_value(eff, world, ms_step) / 1e12
-        kernel_ms = statistics.mean(per)
-        achieved = eff / (kernel_ms * 1e-3) / 1e12
-        traffic = NCU_TRAFFIC.get((args.workload, kernel_source_hash("prefill")))
-        # a kernel that runs under the power cap (long steps: the clocks saw
-        # sw_power_cap) is held against the sustained GEMM figure, else the burst one
-        capped = bool(clk) and "sw_power_cap" in (clk.get("reasons") or [])
-        sustained = capped and peaks.get("bf16_tflops_sustained")
-        peak_t = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-        peak_kind = "sustained, sw_power_cap active" if sustained else "burst"
-        result.update({
-            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s",
-            "ms_per_step": round(ms_step, 4),
-            "dtype": "bf16",
-            "roofline": {"bound": "tensor", "achieved": round(achieved, 2),
-                         "peak": peak_t, "unit": "TFLOP/s",
-                         "frac": round(achieved / peak_t, 4),
-                         "traffic": traffic,
-                         "peak_source": f"{peaks['source']} bf16 dense ({peak_kind})"},
-            "window_off": {"ms_per_step": round(off_ms_step, 4),
-                           "speedup": round(off_ms_step / ms_step, 3),
-                           "ideal_speedup": round(off_flops / eff, 3),
-                           "effective_tflops_at_window_off_time": round(eff / (off_ms_step * 1e-3) / 1e12, 2)},
-            "work": {"effective_tflop_per_step": round(world * eff / 1e12, 4),
-                     "window_off_tflop_per_step": round(world * off_flops / 1e12, 4),
-                     "pruned_fraction": wp.pruned_fraction(win, w.Nq, w.Nk, w.q_pos0, w.k_pos0)[2]},
-            "gpu_launches": args.steps,
-            "clocks": clk,
-        })
-        if masked is not None:
-            result["block_sparse"] = masked
-            result["rope"] = rope_res
-            result["explicit_positions"] = positions_res
-            result["gpu_launches"] += 7 * max(3, args.steps // 2)
-        # end to end through the public API with pinned host buffers
-        qh = q.cpu().pin_memory()
-        kh = k.cpu().pin_memory()
-        vh = v.cpu().pin_memory()
-        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-
-        def step_e2e():
-            qd = q.copy_(qh, non_blocking=True)
-            kd = k.copy_(kh, non_blocking=True)
-            vd = v.copy_(vh, non_blocking=True)
-            o, _ = wp.prefill(qd, kd, vd, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale,
-                              out=out, lse=lse)
-            oh.copy_(o, non_blocking=True)
-
-        n_e2e = max(5, args.steps // 4)
-        e2e_ms, _, _ = time_steps(step_e2e, 2, n_e2e, flush, world)
-        h2d = (q.numel() + k.numel() + v.numel()) * 2
-        result["e2e"] = {"value": round(world * eff / (e2e_ms / n_e2e * 1e-3) / 1e12, 2),
-                         "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                         "d2h_bytes_per_step": out.numel() * 2}
-        result["config"] = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                            "Nq": w.Nq, "Nk": w.Nk, "q_pos0": w.q_pos0, "rope_base": w.base,
-                            "alpha": w.alpha, "group_pairs": w.g, "global_batch": w.B * world,
-                            "seq_len": w.Nk, "parallelism": f"independent problem per GPU x{world}",
-                            "l2": "flushed between steps (512 MiB write)"}
-        del q, k, v, out, lse, qh, kh, vh, oh
-        torch.cuda.empty_cache()
-    if w.kind == "decode" or (args.workload == DEFAULT_WORKLOAD and not args.only_primary):
-        wd = w if w.kind == "decode" else inputs.WORKLOADS[DECODE_WORKLOAD]
-        dres = bench_decode(wd, args, world, rank, dev, flush, peaks,
-                            primary=(w.kind == "decode"))
-        if w.kind == "decode":
-            result.update(dres)
-        else:
-            result["decode"] = dres
-    result.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                   "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                   "data": "synthetic (seeded N(0,1) bf16; pair magnitudes / planted key per workload)"})
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, time_budget_s=args.cpu_seconds)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
-    return rank, result
+    n_e2e = max(5, args.steps // 4)
+    e2e_ms, _, _ = time_steps(step_e2e, 2, n_e2e, flush, world)
+    _check_status(wp, w.name + " end to end")
+    res["e2e"] = {"value": round(world * eff / (e2e_ms / n_e2e * 1e-3) / 1e12, 2),
+                  "unit": "TFLOP/s", "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * 2,
+                  "d2h_bytes_per_step": out.numel() * 2}
+    del q, k, v, out, lse, qh, kh, vh, oh
+    torch.cuda.empty_cache()
+    return res
 
 
-def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
+def _prefill_variants(w, args, world, rank, dev, flush, peaks, q, k, v, out, lse, win, eff,
+                      ms_step):
+    """Block-mask, pre-RoPE and explicit-positions calls of the same prefill problem."""
+    import torch
+    import rope_wavelength_sparsity_b200 as wp
+    from rope_wavelength_sparsity_b200 import inputs
+    res = {}
+    n_v = max(3, args.steps // 2)
+    # the same call under a MInference-shaped block mask (vertical + slash tiles)
+    mask = inputs.vertical_slash_mask(w.B, w.Hq, w.Nq, w.Nk, seed=rank, q_pos0=w.q_pos0,
+                                      k_pos0=w.k_pos0)
+    words = wp.pack_block_mask(mask.to(dev))
+    m_eff = masked_flops(w, win, wp, mask)
+
+    def step_masked():
+        wp.prefill_masked(q, k, v, words, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale,
+                          out=out, lse=lse)
+
+    m_ms, m_per, _ = time_steps(step_masked, args.warmup, n_v, flush, world)
+    _check_status(wp, "masked prefill")
+    m_ach = m_eff / (statistics.mean(m_per) * 1e-3) / 1e12
+    causal_tiles = sum(1 for qb in range(mask.shape[2]) for kb in range(mask.shape[3])
+                       if kb * 128 + w.k_pos0 <= w.q_pos0 + qb * 128 + 127)
+    res["block_sparse"] = {
+        "value": round(weak_scaling_value(m_eff, world, m_ms / n_v) / 1e12, 2),
+        "unit": "TFLOP/s", "ms_per_step": round(m_ms / n_v, 4),
+        "roofline": {"bound": "tensor", "achieved": round(m_ach, 2), "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(m_ach / peaks["bf16_tflops"], 4),
+                     "traffic": None},
+        "speedup_vs_unmasked": round(ms_step / (m_ms / n_v), 3),
+        "ideal_speedup": round(eff / m_eff, 3),
+        "attended_tile_fraction": round(float(mask.sum()) / (w.B * w.Hq * causal_tiles), 4),
+        "mask": "vertical-slash: sink + 3 random key tiles per head, 16-tile diagonal band",
+        "gpu_launches": n_v,
+    }
+    del words, mask
+    # the same prefill from pre-RoPE q and k: rotation pre-pass + attention, and the
+    # rotation kernel alone (HBM-bound: read and write q and k once)
+    ws_r = torch.empty(max(1, int(wp.lib().wpattn_prefill_rope_workspace_size(
+        w.B, w.Nq, w.Nk, w.Hq, w.Hkv, w.D))), dtype=torch.uint8, device=dev)
+    qr_buf = torch.empty_like(q)
+    kr_buf = torch.empty_like(k)
+
+    def step_rope_prefill():
+        wp.prefill_rope(q, k, v, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale, out=out,
+                        lse=lse, workspace=ws_r)
+
+    def step_rope_only():
+        wp.rope(q, base=w.base, pos0=w.q_pos0, out=qr_buf)
+        wp.rope(k, base=w.base, pos0=w.k_pos0, out=kr_buf)
+
+    rp_ms, _, _ = time_steps(step_rope_prefill, args.warmup, n_v, flush, world)
+    ro_ms, ro_per, _ = time_steps(step_rope_only, args.warmup, n_v, flush, world)
+    _check_status(wp, "rope kernels")
+    rope_bytes = 2 * 2 * (q.numel() + k.numel())
+    ro_gbs = rope_bytes / (statistics.mean(ro_per) * 1e-3) / 1e9
+    res["rope"] = {
+        "prefill_from_prerope": {"ms_per_step": round(rp_ms / n_v, 4),
+                                 "value": round(weak_scaling_value(eff, world, rp_ms / n_v) / 1e12, 2),
+                                 "unit": "TFLOP/s",
+                                 "overhead_vs_prefill": round((rp_ms / n_v) / ms_step - 1.0, 4),
+                                 "gpu_launches": 3 * n_v},
+        "rotation_kernels": {"ms_per_step": round(ro_ms / n_v, 4),
+                             "roofline": {"bound": "hbm", "achieved": round(ro_gbs, 1),
+                                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                          "frac": round(ro_gbs / peaks["hbm_gbs"], 4),
+                                          "traffic": None},
+                             "bytes_per_step": rope_bytes, "gpu_launches": 2 * n_v},
+    }
+    del ws_r, qr_buf, kr_buf
+    # the same prefill through the explicit-positions kernel, given the workload's own
+    # contiguous positions (same work; the cost of the searched column ranges)
+    qp = (w.q_pos0 + torch.arange(w.Nq, dtype=torch.int32, device=dev)).repeat(w.B, 1)
+    kp = (w.k_pos0 + torch.arange(w.Nk, dtype=torch.int32, device=dev)).repeat(w.B, 1)
+
+    def step_pos():
+        wp.prefill_positions(q, k, v, qp, kp, win, scale=w.scale, out=out, lse=lse)
+
+    pos_ms, pos_per, _ = time_steps(step_pos, args.warmup, n_v, flush, world)
+    _check_status(wp, "positions prefill")
+    pos_ach = eff / (statistics.mean(pos_per) * 1e-3) / 1e12
+    res["explicit_positions"] = {
+        "value": round(weak_scaling_value(eff, world, pos_ms / n_v) / 1e12, 2),
+        "unit": "TFLOP/s", "ms_per_step": round(pos_ms / n_v, 4),
+        "roofline": {"bound": "tensor", "achieved": round(pos_ach, 2), "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(pos_ach / peaks["bf16_tflops"], 4),
+                     "traffic": None},
+        "slowdown_vs_plain": round((pos_ms / n_v) / ms_step, 3),
+        "positions": "the workload's contiguous positions passed as int32 arrays",
+        "gpu_launches": n_v,
+    }
+    del qp, kp
+    return res
+
+
+def bench_decode(w, args, world, rank, dev, flush, peaks):
+    """One decode workload: the contiguous-cache call, window off, pair-major and paged
+    layouts of the same cache, and the end-to-end call with the query from the host."""
     import torch
     import rope_wavelength_sparsity_b200 as wp
     from rope_wavelength_sparsity_b200 import inputs
@@ -485,13 +503,14 @@ def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
         wp.decode(q, kc, vc, kv_len, win_off, scale=w.scale, out=out, lse=lse, workspace=ws)
 
     steps = args.steps
-    clocks = ClockSampler(dev.index) if (rank == 0 and primary) else None
+    clocks = ClockSampler(dev.index) if rank == 0 else None
     total_ms, per, clk = time_steps(step, args.warmup, steps, flush, world, clocks)
-    if wp.device_status() != wp.OK:
-        raise RuntimeError("decode kernel status: timeout")
-    off_ms, _, _ = time_steps(step_off, args.warmup, max(3, steps // 4), flush, world)
+    _check_status(wp, w.name)
+    n_off = max(3, steps // 4)
+    off_ms, _, _ = time_steps(step_off, args.warmup, n_off, flush, world)
+    _check_status(wp, w.name + " window off")
     ms = total_ms / steps
-    off_step = off_ms / max(3, steps // 4)
+    off_step = off_ms / n_off
     achieved = alg / (statistics.mean(per) * 1e-3) / 1e9
     res = {
         "metric": METRIC, "value": round(weak_scaling_value(alg, world, ms) / 1e9, 1), "unit": "GB/s",
@@ -505,11 +524,8 @@ def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
                        "ideal_speedup": round(off_bytes / alg, 3)},
         "work": {"algorithmic_bytes_per_step": alg * world, "window_off_bytes_per_step": off_bytes * world},
         "gpu_launches": 2 * steps,
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.Nk,
-                   "rope_base": w.base, "alpha": w.alpha, "group_pairs": w.g,
-                   "global_batch": w.B * world, "seq_len": w.Nk,
-                   "parallelism": f"independent problem per GPU x{world}",
-                   "l2": "flushed between steps (512 MiB write)"},
+        "clocks": clk,
+        "config": workload_config(w, world),
     }
     # the same call with K in the pair-major layout (converted once, outside the timed region):
     # the window then also cuts the bytes K moves from HBM
@@ -519,8 +535,7 @@ def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
         wp.decode_pairmajor(q, slabs, vc, kv_len, win, scale=w.scale, out=out, lse=lse, workspace=ws)
 
     pm_ms, pm_per, _ = time_steps(step_pm, args.warmup, steps, flush, world)
-    if wp.device_status() != wp.OK:
-        raise RuntimeError("pair-major decode kernel status: timeout")
+    _check_status(wp, "pair-major decode")
     pm_achieved = alg / (statistics.mean(pm_per) * 1e-3) / 1e9
     res["pairmajor"] = {
         "value": round(weak_scaling_value(alg, world, pm_ms / steps) / 1e9, 1), "unit": "GB/s",
@@ -530,11 +545,11 @@ def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
                      "traffic": None, "peak_source": f"{peaks['source']} HBM copy"},
         "speedup_vs_window_off": round(off_step / (pm_ms / steps), 3),
         "layout": "K [B, Hkv, D/16, L, 16] pair-major slabs, V [B, L, Hkv, D]",
+        "gpu_launches": 2 * steps,
     }
-    res["gpu_launches"] += 2 * steps
     del slabs
-    # the same call from a paged cache (16-row pages in shuffled pool order, the
-    # page size serving engines default to), scattered once outside the timed region
+    # the same call from a paged cache (16-row pages in shuffled pool order, the page size
+    # serving engines default to), scattered once outside the timed region
     page = 16
     table, num_pages = inputs.page_layout(kv_len, page, seed=rank + 100)
     kp = inputs.scatter_to_pages(kc, kv_len, table, page, num_pages)
@@ -548,8 +563,7 @@ def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
                         workspace=ws_pg)
 
     pg_ms, pg_per, _ = time_steps(step_pg, args.warmup, steps, flush, world)
-    if wp.device_status() != wp.OK:
-        raise RuntimeError("paged decode kernel status: not ok")
+    _check_status(wp, "paged decode")
     pg_achieved = alg / (statistics.mean(pg_per) * 1e-3) / 1e9
     res["paged"] = {
         "value": round(weak_scaling_value(alg, world, pg_ms / steps) / 1e9, 1), "unit": "GB/s",
@@ -558,8 +572,8 @@ def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
                      "unit": "GB/s", "frac": round(pg_achieved / peaks["hbm_gbs"], 4),
                      "traffic": None, "peak_source": f"{peaks['source']} HBM copy"},
         "layout": f"K, V page pools [{num_pages}, {page}, Hkv, D], shuffled block table",
+        "gpu_launches": 2 * steps,
     }
-    res["gpu_launches"] += 2 * steps
     del kp, vp, ws_pg
     if world > 1 and getattr(args, "kv_split", False):
         # strong scaling: the same decode (rank 0's problem) with its cache split by
@@ -577,93 +591,172 @@ def bench_decode(w, args, world, rank, dev, flush, peaks, primary):
             wd.decode_kv_split(q0, ks, vs, kvl0, win, shard_len=shard, rank=rank, world=world,
                                scale=w.scale)
 
-        sp_ms, _, _ = time_steps(step_split, args.warmup, steps, flush, world,
-                                 per_step_events=False)
+        sp_ms, _, _ = time_steps(step_split, args.warmup, steps, flush, world)
         res["kv_split"] = {
             "value": round(alg0 / (sp_ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
             "ms_per_step": round(sp_ms / steps, 4), "scaling": "strong",
             "exchange": "one all-gather of (out, lse) parts per step, then merge_lse",
         }
         del ks, vs
-    if primary:
-        res["clocks"] = clk
-        qh = q.cpu().pin_memory()
-        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    qh = q.cpu().pin_memory()
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
 
-        def step_e2e():
-            qd = q.copy_(qh, non_blocking=True)
-            o, _ = wp.decode(qd, kc, vc, kv_len, win, scale=w.scale, out=out, lse=lse, workspace=ws)
-            oh.copy_(o, non_blocking=True)
+    def step_e2e():
+        qd = q.copy_(qh, non_blocking=True)
+        o, _ = wp.decode(qd, kc, vc, kv_len, win, scale=w.scale, out=out, lse=lse, workspace=ws)
+        oh.copy_(o, non_blocking=True)
 
-        n_e2e = max(5, steps // 4)
-        e2e_ms, _, _ = time_steps(step_e2e, 2, n_e2e, flush, world)
-        res["e2e"] = {"value": round(world * alg / (e2e_ms / n_e2e * 1e-3) / 1e9, 1), "unit": "GB/s",
-                      "h2d_bytes_per_step": q.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
-                      "note": "the KV cache is resident on the device, as in serving"}
+    n_e2e = max(5, steps // 4)
+    e2e_ms, _, _ = time_steps(step_e2e, 2, n_e2e, flush, world)
+    _check_status(wp, w.name + " end to end")
+    res["e2e"] = {"value": round(world * alg / (e2e_ms / n_e2e * 1e-3) / 1e9, 1), "unit": "GB/s",
+                  "h2d_bytes_per_step": q.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
+                  "note": "the KV cache is resident on the device, as in serving"}
     del q, kc, vc, out, lse, ws
     torch.cuda.empty_cache()
     return res
 
 
-# --------------------------------------------------------- oracle (CPU) arm
-def oracle_sample(w, n_rows, seed=0):
-    """Query rows spread over heads and positions, and the inputs to run them."""
-    import numpy as np
+def _run_workload(name, args, world, rank, dev, flush, peaks):
     from rope_wavelength_sparsity_b200 import inputs
+    w = inputs.WORKLOADS[name]
+    if w.kind == "prefill":
+        return bench_prefill(w, args, world, rank, dev, flush, peaks,
+                             variants=(name == VARIANTS_WORKLOAD and not args.only_primary))
+    return bench_decode(w, args, world, rank, dev, flush, peaks)
+
+
+def gpu_arm(args):
+    import torch
+    from rope_wavelength_sparsity_b200 import inputs
+
+    world, rank, local = _dist_setup(args)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    peaks = load_peaks()
+    w = inputs.WORKLOADS[args.workload]
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    result = _run_workload(args.workload, args, world, rank, dev, flush, peaks)
+    if args.workload == DEFAULT_WORKLOAD and not args.only_primary:
+        result["configs"] = {name: _run_workload(name, args, world, rank, dev, flush, peaks)
+                             for name in NESTED_PREFILL + NESTED_DECODE}
+    result.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                   "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                   "data": "synthetic (seeded N(0,1) bf16; pair magnitudes / planted key per workload)"})
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, time_budget_s=args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return rank, result
+
+
+# --------------------------------------------------------- oracle (CPU) arm
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover - non-Linux hosts
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, n_rows, seed=0):
+    """Rows of a workload spread over heads and positions: (b, h, t) for a prefill,
+    (b, h) for a decode."""
+    import numpy as np
     rng = np.random.default_rng(seed)
     rows = []
     if w.kind == "prefill":
         for i in range(n_rows):
-            h = i % w.Hq
-            t = int(rng.integers(0, w.Nq))
-            rows.append((0, h, t))
+            rows.append((0, i % w.Hq, int(rng.integers(0, w.Nq))))
     else:
         for i in range(n_rows):
             rows.append((i % w.B, (i * 7) % w.Hq))
     return rows
 
 
-def cpu_baseline(w, time_budget_s=15.0):
-    """Time the oracle on a bounded sample of the workload (one host thread)."""
-    import torch
-    import oracle
-    import rope_wavelength_sparsity_b200 as wp
-    from rope_wavelength_sparsity_b200 import inputs
-    win = wp.Window(w.D, w.base, w.alpha, w.g)
-    if w.kind == "prefill":
-        q, k, v, _ = inputs.prefill_inputs(w, seed=0, device="cuda" if torch.cuda.is_available() else "cpu")
-        qb, kb, vb = inputs.bits(q), inputs.bits(k), inputs.bits(v)
-        rows = oracle_sample(w, 4096)
-        done, flops, t0 = 0, 0, time.perf_counter()
-        while done < len(rows) and time.perf_counter() - t0 < time_budget_s:
-            b, h, t = rows[done]
-            oracle.attention_rows(qb, kb, vb, Hq=w.Hq, Hkv=w.Hkv, q_pos0=w.q_pos0, k_pos0=w.k_pos0,
-                                  base=w.base, alpha=w.alpha, g=w.g, scale=w.scale, rows=[(b, h, t)])
-            flops += row_flops(w, win, wp, t)
-            done += 1
+class _OracleJob:
+    """The oracle on one sampled row at a time, with each row's work counted by the
+    oracle's own pair-term count before any timing starts."""
+
+    def __init__(self, w, n_rows):
+        import torch
+        import oracle
+        from rope_wavelength_sparsity_b200 import inputs
+        self.w = w
+        self.oracle = oracle
+        # inputs are drawn on the GPU when there is one (only to generate them quickly)
+        gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+        self.rows = oracle_sample(w, n_rows)
+        if w.kind == "prefill":
+            q, k, v, _ = inputs.prefill_inputs(w, seed=0, device=gen_dev)
+            self.work = [row_flops_oracle(w, t) for (_, _, t) in self.rows]
+            self.unit, self.scale = "TFLOP/s", 1e12
+        else:
+            q, k, v, kv_len = inputs.decode_inputs(w, seed=0, device=gen_dev)
+            self.kv_len = [int(x) for x in kv_len]
+            self.work = [decode_row_bytes_oracle(w, self.kv_len[b]) for (b, _) in self.rows]
+            self.unit, self.scale = "GB/s", 1e9
+        self.qb, self.kb, self.vb = inputs.bits(q), inputs.bits(k), inputs.bits(v)
+        del q, k, v
+
+    def run(self, i):
+        w, r = self.w, self.rows[i]
+        if w.kind == "prefill":
+            self.oracle.attention_rows(self.qb, self.kb, self.vb, Hq=w.Hq, Hkv=w.Hkv,
+                                       q_pos0=w.q_pos0, k_pos0=w.k_pos0, base=w.base,
+                                       alpha=w.alpha, g=w.g, scale=w.scale, rows=[r])
+        else:
+            self.oracle.decode_rows(self.qb, self.kb, self.vb, self.kv_len, Hq=w.Hq, Hkv=w.Hkv,
+                                    base=w.base, alpha=w.alpha, g=w.g, scale=w.scale, rows=[r])
+
+    def timed(self, budget_s, threads):
+        """(value, rows done, seconds): rows taken in order by ``threads`` host threads
+        until the budget is spent (the oracle's C code runs outside the GIL)."""
+        counter = itertools.count()
+        lock = threading.Lock()
+        done = []
+
+        def worker(t_end):
+            while time.perf_counter() < t_end:
+                with lock:
+                    i = next(counter)
+                if i >= len(self.rows):
+                    return
+                self.run(i)
+                with lock:
+                    done.append(i)
+
+        t0 = time.perf_counter()
+        ths = [threading.Thread(target=worker, args=(t0 + budget_s,)) for _ in range(threads)]
+        for th in ths:
+            th.start()
+        for th in ths:
+            th.join()
         dt = time.perf_counter() - t0
-        return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
-                "kind": "oracle",
-                "sample": f"{done} query rows (random heads/positions) of {w.name}, {dt:.1f} s, "
-                          "effective FLOPs of those rows / wall time"}
-    q, kc, vc, kv_len = inputs.decode_inputs(w, seed=0, device="cuda" if torch.cuda.is_available() else "cpu")
-    qb, kb, vb = inputs.bits(q), inputs.bits(kc), inputs.bits(vc)
-    kv_len = [int(x) for x in kv_len]
-    rows = oracle_sample(w, 1024)
-    done, nbytes, t0 = 0, 0, time.perf_counter()
-    P = w.D // 2
-    while done < len(rows) and time.perf_counter() - t0 < time_budget_s:
-        b, h = rows[done]
-        oracle.decode_rows(qb, kb, vb, kv_len, Hq=w.Hq, Hkv=w.Hkv, base=w.base, alpha=w.alpha,
-                           g=w.g, scale=w.scale, rows=[(b, h)])
-        pruned, total, _ = wp.pruned_fraction(win, 1, kv_len[b], kv_len[b] - 1, 0)
-        # one (sequence, kv head) worth of bytes is shared by the G heads of the group
-        nbytes += ((total - pruned) * 4 + kv_len[b] * w.D * 2) / (w.Hq // w.Hkv)
-        done += 1
-    dt = time.perf_counter() - t0
-    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{done} (sequence, head) rows of {w.name}, {dt:.1f} s, algorithmic bytes "
-                      "of those rows (per-head share of the group's K/V) / wall time"}
+        work = sum(self.work[i] for i in done)
+        return work / dt / self.scale, len(done), dt
+
+
+def cpu_baseline(w, time_budget_s=15.0):
+    """The oracle timed on the host on a bounded sample of the workload: on all the
+    host's cores (independent rows, one per thread) and on one core."""
+    cores = host_cores()
+    job = _OracleJob(w, n_rows=max(4096, 64 * cores))
+    what = "query rows (random heads/positions)" if w.kind == "prefill" else "(sequence, head) rows"
+    measure = ("effective FLOPs of those rows / wall time" if w.kind == "prefill" else
+               "algorithmic bytes of those rows (per-head share of the group's K/V) / wall time")
+    one, n1, t1 = job.timed(time_budget_s, 1)
+    allc, na, ta = job.timed(time_budget_s, cores)
+    return {"value": round(allc, 6), "unit": job.unit, "cores": cores, "kind": "oracle",
+            "sample": f"{na} {what} of {w.name} on {cores} threads, {ta:.1f} s; {measure}; "
+                      "work counted with the oracle's own pair-term count",
+            "one_core": {"value": round(one, 6), "unit": job.unit, "cores": 1,
+                         "sample": f"{n1} rows of the same sample, {t1:.1f} s"}}
 
 
 def reference_arm(args):
@@ -673,38 +766,48 @@ def reference_arm(args):
         return rank, None
     from rope_wavelength_sparsity_b200 import inputs
     w = inputs.WORKLOADS[args.workload]
-    per_step = max(0.2, 90.0 / max(1, args.steps + args.warmup))
+    cores = host_cores()
+    # about 90 s of oracle work in all (--ref-seconds), spread over the steps
+    per_step = max(0.2, getattr(args, "ref_seconds", 90.0) / max(1, args.steps + args.warmup))
+    job = _OracleJob(w, n_rows=max(4096, 64 * cores))
     vals = []
-    cb = None
+    rows_done = 0
     for i in range(args.warmup + args.steps):
-        cb = cpu_baseline(w, time_budget_s=per_step)
+        val, n, _ = job.timed(per_step, cores)
         if i >= args.warmup:
-            vals.append(cb["value"])
-    value = statistics.mean(vals) if vals else cb["value"]
-    unit = cb["unit"]
-    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": w.name},
-           "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
-                            "sample": f"each step: {cb['sample']}"},
-           "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            vals.append(val)
+            rows_done += n
+    value = statistics.mean(vals) if vals else 0.0
+    sample = (f"each step: rows of {w.name} on {cores} threads for {per_step:.1f} s "
+              f"({rows_done} rows over the timed steps); work counted with the oracle's own "
+              "pair-term count")
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": job.unit,
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": workload_config(w, world),
+           "cpu_baseline": {"value": value, "unit": job.unit, "cores": cores, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": job.unit, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
     return rank, out
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only-primary", action="store_true",
-                    help="skip the secondary decode measurement of the default workload")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+                    help="time only the chosen workload (no nested configs or variants)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="oracle time budget of each cpu_baseline figure (1 core, all cores)")
+    ap.add_argument("--ref-seconds", type=float, default=90.0,
+                    help="--impl reference: oracle time over all its steps")
     ap.add_argument("--kv-split", action="store_true",
-                    help="with N > 1: also time the decode with its cache split by length over "
+                    help="with N > 1: also time each decode with its cache split by length over "
                          "the ranks (strong scaling, one all-gather per step)")
     args = ap.parse_args()
     if args.warmup < 3:

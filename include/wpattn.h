@@ -197,7 +197,7 @@ WPATTN_API size_t wpattn_decode_workspace_size(const wpattn_window *w, int32_t B
  *   workspace  : device, >= wpattn_decode_workspace_size(w, B, Hq, Hkv, Lmax)
  *                bytes, 256-byte aligned; its contents are scratch (fp32 partial
  *                results of each key range) and are overwritten.
- * Requires D in {64, 128}, Hq % Hkv == 0, Hq / Hkv <= 16, B <= 4096.
+ * Requires D in {64, 128}, Hq % Hkv == 0, Hq / Hkv <= 16, B <= 1024.
  */
 WPATTN_API int wpattn_decode(const wpattn_window *w,
                   const void *q, const void *k_cache, const void *v_cache,

@@ -13,6 +13,14 @@ Entry points (same names as the C ABI, without the ``wpattn_`` prefix):
 ``prefill_rope``, ``decode_rope``, ``prefill_positions``, ``decode_shard``, ``merge_lse``,
 ``decode_workspace_size``, ``decode_noalloc``, ``pruned_fraction``,
 ``thresholds``, ``device_status``.
+
+Calls are asynchronous on the given stream (torch's current stream by
+default).  Every wait inside a kernel is bounded; when one runs out, the
+kernel returns early, its outputs are not valid, and the only report is the
+library's status word, read (and cleared) by ``device_status()``.  Callers
+that need to know must poll it after their calls, or pass ``check=True`` to
+``prefill``, ``decode`` or ``decode_noalloc``, which synchronises the stream
+and raises ``WpattnError`` (code ``ETIMEOUT``) on a nonzero status.
 """
 from __future__ import annotations
 
@@ -193,10 +201,12 @@ def _prefill_shapes(q, k, v, w, out, lse):
 
 
 def prefill(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0, scale: float | None = None,
-            out=None, lse=None, want_lse: bool = True, stream=None):
+            out=None, lse=None, want_lse: bool = True, stream=None, check: bool = False):
     """Windowed causal prefill.  q [B,Nq,Hq,D], k/v [B,Nk,Hkv,D] bf16 CUDA tensors.
 
-    Returns (out [B,Nq,Hq,D] bf16, lse [B,Hq,Nq] fp32 or None).
+    Returns (out [B,Nq,Hq,D] bf16, lse [B,Hq,Nq] fp32 or None).  The call is
+    asynchronous; a kernel that gave up a bounded wait is reported only by
+    ``device_status()``, unless ``check`` (synchronise and raise).
     """
     import torch
     B, Nq, Hq, D, Nk, Hkv = _prefill_shapes(q, k, v, w, out, lse)
@@ -210,6 +220,8 @@ def prefill(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0, scale: floa
                               B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0,
                               float(scale) if scale else 0.0, _stream_ptr(stream))
     _check(rc, "wpattn_prefill")
+    if check:
+        _check(device_status(stream), "wpattn_prefill (device status)")
     return out, lse
 
 
@@ -361,10 +373,12 @@ def _decode_shapes(q, k_cache, v_cache, kv_len, w, out, lse):
 
 
 def decode(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | None = None, out=None,
-           lse=None, want_lse: bool = True, workspace=None, stream=None):
+           lse=None, want_lse: bool = True, workspace=None, stream=None, check: bool = False):
     """Windowed decode.  q [B,Hq,D]; caches [B,L,Hkv,D] bf16 CUDA; kv_len: host ints [B].
 
-    Returns (out [B,Hq,D] bf16, lse [B,Hq] fp32 or None).
+    Returns (out [B,Hq,D] bf16, lse [B,Hq] fp32 or None).  The call is
+    asynchronous; a kernel that gave up a bounded wait is reported only by
+    ``device_status()``, unless ``check`` (synchronise and raise).
     """
     import torch
     B, Hq, D, L, Hkv = _decode_shapes(q, k_cache, v_cache, kv_len, w, out, lse)
@@ -386,6 +400,8 @@ def decode(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | None = None
                              ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
                              _stream_ptr(stream))
     _check(rc, "wpattn_decode")
+    if check:
+        _check(device_status(stream), "wpattn_decode (device status)")
     return out, lse
 
 
@@ -574,12 +590,13 @@ def decode_paged(q, k_pages, v_pages, block_table, kv_len, w: Window, *, q_pos=N
 
 
 def decode_noalloc(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | None = None,
-                   out=None, lse=None, want_lse: bool = True, stream=None):
+                   out=None, lse=None, want_lse: bool = True, stream=None, check: bool = False):
     """Decode with the library's built-in scratch instead of a workspace.
 
     For callers that cannot allocate device memory at the call site; the
     problem's partial results must fit the built-in array
-    (``decode_noalloc_max_bytes()``), calls on one device share it.
+    (``decode_noalloc_max_bytes()``), calls on one device share it.  With
+    ``check`` the stream is synchronised and a nonzero device status raises.
     """
     import torch
     B, Hq, D, L, Hkv = _decode_shapes(q, k_cache, v_cache, kv_len, w, out, lse)
@@ -598,6 +615,8 @@ def decode_noalloc(q, k_cache, v_cache, kv_len, w: Window, *, scale: float | Non
             _dev_tensor(out, "out"), ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
             _stream_ptr(stream))
     _check(rc, "wpattn_decode_noalloc")
+    if check:
+        _check(device_status(stream), "wpattn_decode_noalloc (device status)")
     return out, lse
 
 

@@ -2,16 +2,17 @@
 //
 // "ATFlash: Per-RoPE-Wavelength Attention Windows", Abstract: the window is
 // a slice of the query-key contraction axis ported into a FlashInfer-style
-// decode kernel.  Each CTA covers one (sequence, kv head, key range) and all
+// decode kernel, which then reads K only over the active head-dim slice of
+// each key block.  Each CTA covers one (sequence, kv head, key range) and all
 // the query heads of the GQA group (up to GC at a time), so a K/V byte is
 // read once for the group.  A producer warp streams blocks of 32 keys of K
-// and V through a shared-memory ring with TMA (128-byte swizzle); each block
-// is consumed by one of four compute warps.  For the scores a lane owns a
-// key and walks only the groups of 8 pairs still kept in the block; for
-// O += p V a lane owns a 16-byte chunk of the head dim.  In the
-// [B, L, Hkv, D] cache layout each half of a K row is one 128-byte line and
-// the kept slice touches both, so whole rows move from DRAM either way; the
-// window saves arithmetic here, not bytes.  A second kernel merges the key
+// and V through a shared-memory ring with TMA; each block is consumed by one
+// of four compute warps, which run both contractions on warp-level tensor-
+// core MMAs (mma.sync m16n8k16): S^T = K Q^T over the groups of 8 pairs still
+// kept in the block, then O^T += V^T P^T.  K is loaded only from the block's
+// first kept group on: in 32-byte sector columns of each half of the head
+// dim for the [B, L, Hkv, D] cache, or in 1 KB slabs for the pair-major
+// cache; a paged cache moves whole rows.  A second kernel merges the key
 // ranges by their log-sum-exp.
 #pragma once
 
@@ -53,24 +54,13 @@ struct DecodeParams {
   double theta[64];
 };
 
-__device__ __forceinline__ uint4 ldg_stream(const void* ptr) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(ptr));
-  return r;
-}
-
-__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
-  f[0] = bf16lo_to_f32(u.x); f[1] = bf16hi_to_f32(u.x);
-  f[2] = bf16lo_to_f32(u.y); f[3] = bf16hi_to_f32(u.y);
-  f[4] = bf16lo_to_f32(u.z); f[5] = bf16hi_to_f32(u.z);
-  f[6] = bf16lo_to_f32(u.w); f[7] = bf16hi_to_f32(u.w);
-}
-
-// Shared-memory ring of the split kernel: blocks of KB keys of K and V in
-// the 128-byte-swizzled layout TMA writes (64-dim panels, row = key), plus
-// the pre-scaled query heads, the thresholds and each warp's p row.
+// Shared-memory ring of the split kernel: blocks of KB keys of K and V, plus
+// the query heads, the thresholds and each warp's p row.  V (and K of a
+// paged cache) is in the 128-byte-swizzled layout TMA writes (64-dim panels,
+// row = key).  K of a [B, L, Hkv, D] cache is in sector columns: column c of
+// half h (dims h * D/2 + 16c .. + 16, one 32-byte DRAM sector of each row)
+// of the block's keys at (2c + h) * KB * 32, key r at 32 r; a group g of 8
+// pairs is the 16 bytes at (g & 1) * 16 of column g / 2 in both halves.
 constexpr int kDecodeComputeWarps = 4;
 
 template <int D>
@@ -104,12 +94,10 @@ __device__ __forceinline__ uint4 ring_chunk(const uint8_t* tile, int r, int c) {
 }
 
 // Work split inside a CTA: the producer warp streams blocks of 32 keys; block
-// i goes to compute warp i mod 4.  For the scores a lane owns one key (its
-// whole row): it walks only the groups of 8 pairs that are still kept
-// somewhere in the warp's 32 keys, with the query head dims read from shared
-// memory (broadcast), so the window removes work and no cross-lane reduction
-// is needed.  For O += p V a lane owns one 16-byte chunk of the head dim for
-// 32 / (D / 8) keys at a time.
+// i goes to compute warp i mod 4, which computes its scores for every query
+// head of the CTA over the block's kept groups, runs the online softmax and
+// accumulates O^T, all in registers (the query heads fill the n = 8 side of
+// the MMAs).  The warps merge through shared memory at the end.
 //
 // PM (pair-major K cache): K is stored as [B, Hkv, D/16, Lmax, 16], slab g
 // holding dims 8g..8g+7 and P+8g..P+8g+7 of every key (the 8 pairs of one
@@ -156,6 +144,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   const int nblk = j_end > j_begin ? (j_end - j_begin + KB - 1) / KB : 0;
   const int qpos = p.q_pos[b];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool paged = !PM && p.block_table != nullptr;  // K in swizzled rows, not sector columns
   // first group of 8 pairs kept for some key of the block starting at j0:
   // groups whose largest threshold is below the block's smallest distance
   // (that of its last real key) are pruned for every key of the block
@@ -220,7 +209,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       return pg;
     };
     int my_page = 0, next_page = 0;
-    const bool paged = !PM && p.block_table != nullptr;
     if (paged) {
       my_page = fetch_page(lane);
       next_page = fetch_page(32 + lane);
@@ -240,11 +228,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       nsub = (min(j0 + KB, j_end) - j0 + R - 1) / R;
     };
     if (paged && nblk > 0) plan_block(0);
-    // pair-major: first slab of the next block, found while its stage drains
-    int g0_next = (PM && nblk > 0) ? first_kept_group(j_begin) : 0;
+    // first kept group of the next block, found while its stage drains (with
+    // explicit key positions it is only known once the keys are: load them all)
+    auto first_loaded_group = [&](int j0) -> int { return p.k_pos ? 0 : first_kept_group(j0); };
+    int g0_next = nblk > 0 ? first_loaded_group(j_begin) : 0;
+    int issued = 0;           // blocks whose copies were issued
+    bool ok_prod = true;
     for (int i = 0; i < nblk; ++i) {
       const int s = i % NS;
-      if (i >= NS && !__all_sync(FULL, mbar_wait(empty(s), ((i / NS) & 1) ^ 1))) break;
+      if (i >= NS && !__all_sync(FULL, mbar_wait(empty(s), ((i / NS) & 1) ^ 1))) {
+        ok_prod = false;
+        break;
+      }
       const int j0 = j_begin + i * KB;
       if (paged) {
         if (lane == 0) {
@@ -260,26 +255,38 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             }
           }
         }
+        issued = i + 1;
         if (i + 1 < nblk) plan_block(i + 1);
         continue;
       }
       if (lane == 0) {
+        const int g0 = g0_next;
         if (PM) {
-          const int g0 = g0_next;
           mbar_arrive_expect_tx(full(s), (NG - g0) * KB * 32 + L::TILE);
           for (int g = g0; g < NG; ++g)
             tma_load_4d(sbase + L::OFF_K + s * L::TILE + g * KB * 32, &tmK, full(s), 0, j0, kvh * NG + g, b);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_4d(sbase + L::OFF_V + s * L::TILE + c * L::PANEL, &tmV, full(s), 64 * c, j0, kvh, b);
-          if (i + 1 < nblk) g0_next = first_kept_group(j0 + KB);
         } else {
-          mbar_arrive_expect_tx(full(s), 2 * L::TILE);
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_4d(sbase + L::OFF_K + s * L::TILE + c * L::PANEL, &tmK, full(s), 64 * c, j0, kvh, b);
-            tma_load_4d(sbase + L::OFF_V + s * L::TILE + c * L::PANEL, &tmV, full(s), 64 * c, j0, kvh, b);
-          }
+          // the 32-byte sector columns of both halves from the one holding group g0
+          constexpr int NC = P / 16;
+          const int c0 = g0 >> 1;
+          mbar_arrive_expect_tx(full(s), 2 * (NC - c0) * KB * 32 + L::TILE);
+          for (int c = c0; c < NC; ++c)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_4d(sbase + L::OFF_K + s * L::TILE + (2 * c + hf) * KB * 32, &tmK, full(s),
+                          hf * P + 16 * c, j0, kvh, b);
         }
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sbase + L::OFF_V + s * L::TILE + c * L::PANEL, &tmV, full(s), 64 * c, j0, kvh, b);
       }
+      issued = i + 1;
+      if (i + 1 < nblk) g0_next = first_loaded_group(j0 + KB);
+    }
+    if (!ok_prod) {
+      // A wait ran out: copies issued into the ring may still be landing.
+      // Wait (bounded) for the fill of every stage's last issued block before
+      // the CTA can leave; older blocks completed before their stage was reused.
+      for (int i = max(0, issued - NS); i < issued; ++i) (void)mbar_wait(full(i % NS), (i / NS) & 1);
     }
     return;  // the producer takes no part in the merge below
   }
@@ -365,9 +372,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           uint32_t addr;
           if (PM) {
             addr = smem_u32(kt) + g * KB * 32 + key * 32 + lhalf * 16;
-          } else {
+          } else if (paged) {
             const int ch = lhalf ? NG + g : g;
             addr = smem_u32(kt) + (ch >> 3) * L::PANEL + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
+          } else {  // sector column g / 2 of half lhalf, group g's 16 bytes in it
+            addr = smem_u32(kt) + (2 * (g >> 1) + lhalf) * KB * 32 + key * 32 + (g & 1) * 16;
           }
           uint32_t a0, a1, a2, a3;
           ldsm_x4(addr, a0, a1, a2, a3);

@@ -22,8 +22,10 @@ struct WindowPlan {
   int64_t T[kMaxPairs];  // per-pair threshold (group value when g = 8), nondecreasing
 };
 
-// Validates the window and fills `plan` (pairs beyond kMaxPairs need
-// `allow_wide`, used only by the host-side count).  Returns a WPATTN_* code.
+// Validates the window and fills `plan`.  Returns a WPATTN_* code; a head
+// dim above 2 * kMaxPairs (D > 128) gives WPATTN_EUNSUPPORTED, and such
+// windows are only evaluated on the host, pair by pair, through
+// pair_threshold / effective_threshold (the thresholds and the pruned count).
 int make_window_plan(const wpattn_window* w, WindowPlan* plan);
 
 // Threshold of pair p for arbitrary even D (host count path for D > 128).

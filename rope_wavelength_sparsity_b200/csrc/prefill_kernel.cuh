@@ -376,19 +376,34 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int t = 0; t < nq_tiles; ++t)
         for (int c = 0; c < D / 8; ++c)
           tma_load_4d(sQ + t * L::QTILE + c * PANEL_Q, &tmQ, q_full, 8 * c, (QT * cq + t) * kBM, h, b);
+      int nk_issued = 0, nv_issued = 0;  // K / V tiles whose copies were issued
+      bool ok_prod = true;
       for (int j = 0, kt = kt_top; kt >= 0; ++j, kt = stream_next(kt)) {
         const int s = j % NS;
         const uint32_t ph = (j / NS) & 1;
-        if (j >= NS && !mbar_wait(k_empty(s), ph ^ 1)) break;
+        if (j >= NS && !mbar_wait(k_empty(s), ph ^ 1)) { ok_prod = false; break; }
         mbar_arrive_expect_tx(k_full(s), L::KTILE + (POS ? BN * 4 : 0));
         for (int c = 0; c < D / 8; ++c)
           tma_load_4d(sK + s * L::KTILE + c * PANEL_K, &tmK, k_full(s), 8 * c, BN * kt, kvh, b);
         if constexpr (POS)  // the tile's key positions travel with its keys
           bulk_load(sbase + L::OFF_KP + s * BN * 4, kp_row + BN * kt, BN * 4, k_full(s));
-        if (j >= NS && !mbar_wait(v_empty(s), ph ^ 1)) break;
+        nk_issued = j + 1;
+        if (j >= NS && !mbar_wait(v_empty(s), ph ^ 1)) { ok_prod = false; break; }
         mbar_arrive_expect_tx(v_full(s), L::KTILE);
         for (int c = 0; c < D / 64; ++c)
           tma_load_4d(sV + s * L::KTILE + c * (BN * 128), &tmV, v_full(s), 64 * c, BN * kt, kvh, b);
+        nv_issued = j + 1;
+      }
+      if (!ok_prod) {
+        // A wait ran out: copies issued into the ring may still be landing in
+        // shared memory.  Wait (bounded) for the fill of every stage's last
+        // issued tile, and for Q, before this CTA can leave; a tile older than
+        // a stage's last one completed before its stage was reused.
+        (void)mbar_wait(q_full, 0);
+        for (int j = max(0, nk_issued - NS); j < nk_issued; ++j)
+          (void)mbar_wait(k_full(j % NS), (j / NS) & 1);
+        for (int j = max(0, nv_issued - NS); j < nv_issued; ++j)
+          (void)mbar_wait(v_full(j % NS), (j / NS) & 1);
       }
     }
   } else if (warp == W_MMA) {

@@ -23,14 +23,21 @@ def shard_keys(kv_len_total: Sequence[int], rank: int, shard_len: int):
 
 
 def _all_gather(t, world: int, group=None):
-    """[world, *t.shape] stack of every rank's t, in rank order.  Moved as raw
-    bytes so that any backend carries bf16 bit for bit."""
+    """[world, *t.shape] stack of every rank's t, in rank order, on t's device.
+    Moved as raw bytes so that any backend carries bf16 bit for bit; the gloo
+    backend, which gathers host tensors only, goes through a host copy."""
     import torch
     import torch.distributed as dist
     src = t.contiguous().view(torch.uint8)
+    staged = src.is_cuda and dist.get_backend(group) == "gloo"
+    if staged:
+        src = src.cpu()
     parts = [torch.empty_like(src) for _ in range(world)]
     dist.all_gather(parts, src, group=group)
-    return torch.stack(parts).view(t.dtype)
+    out = torch.stack(parts)
+    if staged:
+        out = out.to(t.device)
+    return out.view(t.dtype)
 
 
 def decode_kv_split(q, k_shard, v_shard, kv_len_total: Sequence[int], w, *, shard_len: int,

@@ -1,6 +1,8 @@
 """Shared helpers for the GPU parity tests: run the CUDA path through the
 C ABI, run the oracle on the same bf16 bytes, compare element by element."""
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import torch
@@ -12,6 +14,18 @@ from rope_wavelength_sparsity_b200 import inputs
 # tolerances of the parity bar (out in bf16 units of the output, LSE in nats)
 ATOL_OUT = 1e-2
 ATOL_LSE = 2e-3
+
+
+def oracle_rows_threaded(q_bits, k_bits, v_bits, rows, **kw):
+    """oracle.attention_rows over many rows, split across host threads (the oracle's
+    C code runs outside the GIL; each call computes its rows independently)."""
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
+    n_thr = max(1, min(len(rows), len(os.sched_getaffinity(0))))
+    chunks = [c for c in np.array_split(rows, n_thr) if len(c)]
+    with ThreadPoolExecutor(max_workers=len(chunks)) as ex:
+        parts = list(ex.map(lambda c: oracle.attention_rows(q_bits, k_bits, v_bits, rows=c, **kw),
+                            chunks))
+    return np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts])
 
 
 def check_rows(o_gpu, l_gpu, o_ref, l_ref, what):

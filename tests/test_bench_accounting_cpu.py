@@ -60,15 +60,30 @@ def test_prefill_flops_equal_enumeration(w):
 
 
 @pytest.mark.parametrize("w", CASES, ids=[c.name for c in CASES])
-def test_row_flops_sum_to_the_prefill(w):
+def test_oracle_row_flops_sum_to_the_prefill(w):
+    """The oracle arm's per-row count (the oracle's own pair-term count) against the
+    enumeration, and summed over every row against the product's closed form."""
     win = wp.Window(w.D, w.base, w.alpha, w.g)
     T, _ = oracle.thresholds(w.D, w.base, w.alpha, w.g)
     rows = [0, w.Nq // 2, w.Nq - 1]
     for t in rows:
         kept, causal = _row_terms(T, w.q_pos0 + t, w.k_pos0, w.Nk)
-        assert bench.row_flops(w, win, wp, t) == 4 * kept + 2 * w.D * causal
-    total = sum(bench.row_flops(w, win, wp, t) for t in range(w.Nq))
+        assert bench.row_flops_oracle(w, t) == 4 * kept + 2 * w.D * causal
+    total = sum(bench.row_flops_oracle(w, t) for t in range(w.Nq))
     assert w.B * w.Hq * total == bench.prefill_flops(w, win, wp)[0]
+
+
+@pytest.mark.parametrize("g,alpha", [(1, 1.0), (8, 1.0), (1, math.inf)])
+def test_oracle_decode_row_bytes(g, alpha):
+    """A decode row's share of its group's K slice and V, by the oracle's count, against
+    the enumeration; G rows of one (sequence, kv head) add up to the group's bytes."""
+    w = Workload("acc-dec-row", "decode", 2, 6, 2, 128, 1, 700, 5e5, alpha, g)
+    T, _ = oracle.thresholds(w.D, w.base, w.alpha, w.g)
+    G = w.Hq // w.Hkv
+    for L in (1, 257, 700):
+        d = (L - 1) - np.arange(L, dtype=np.int64)
+        kept = int(_kept_pairs(T, d).sum())
+        assert bench.decode_row_bytes_oracle(w, L) * G == pytest.approx(4 * kept + 2 * w.D * L)
 
 
 @pytest.mark.parametrize("g,alpha", [(1, 1.0), (8, 1.0), (1, math.inf), (8, 0.05)])

@@ -50,3 +50,20 @@ def test_context_usable_after_a_timeout(cuda_dev):
     lc = lse.cpu().reshape(-1).numpy()
     assert np.abs(oc - o_ref).max() <= 1e-2
     assert np.abs(lc - l_ref).max() <= 2e-3
+
+
+def test_check_option_raises_on_a_timeout(cuda_dev):
+    """``check=True`` synchronises and turns a nonzero status word into an error; a
+    clean call with it returns normally."""
+    B, Hq, Hkv, D, L = 1, 4, 2, 64, 300
+    q = inputs.randn_bf16((B, Hq, D), 21).cuda()
+    kc = inputs.randn_bf16((B, L, Hkv, D), 22).cuda()
+    vc = inputs.randn_bf16((B, L, Hkv, D), 23).cuda()
+    win = wp.Window(D, 1e4, 1.0, 1)
+    wp.device_status()
+    wp.decode(q, kc, vc, [L], win, check=True)       # clean: no error
+    wp.selftest_wait_timeout()                        # the status word now holds ETIMEOUT
+    with pytest.raises(wp.WpattnError) as err:
+        wp.decode(q, kc, vc, [L], win, check=True)
+    assert err.value.code == wp.ETIMEOUT
+    assert wp.device_status() == wp.OK                # the check's read cleared it

@@ -17,7 +17,7 @@ import oracle
 import rope_wavelength_sparsity_b200 as wp
 from rope_wavelength_sparsity_b200 import inputs
 
-from _parity import check_rows
+from _parity import check_rows, oracle_rows_threaded
 
 pytestmark = pytest.mark.gpu
 
@@ -41,9 +41,9 @@ def _run_prefill(name, per_head):
     assert wp.device_status() == wp.OK
     rows = np.asarray(_prefill_rows(w, planted, per_head), dtype=np.int64)
     qb, kb, vb = inputs.bits(q), inputs.bits(k), inputs.bits(v)
-    o_ref, l_ref = oracle.attention_rows(qb, kb, vb, Hq=w.Hq, Hkv=w.Hkv, q_pos0=w.q_pos0,
-                                         k_pos0=w.k_pos0, base=w.base, alpha=w.alpha, g=w.g,
-                                         scale=w.scale, rows=rows)
+    o_ref, l_ref = oracle_rows_threaded(qb, kb, vb, rows, Hq=w.Hq, Hkv=w.Hkv, q_pos0=w.q_pos0,
+                                        k_pos0=w.k_pos0, base=w.base, alpha=w.alpha, g=w.g,
+                                        scale=w.scale)
     oc = out.float().cpu()
     lc = lse.cpu()
     o_gpu = np.stack([oc[b, t, h].numpy() for (b, h, t) in rows])
@@ -72,7 +72,8 @@ def test_llama_3b_128k_prefill(cuda_dev, name):
 
 
 def test_qwen_7b_1m_last_chunk_prefill(cuda_dev):
-    _run_prefill("qwen2.5-7b-1m-prefill", [0, 16383])
+    # both ends of the chunk, both sides of 128- and 256-row tile boundaries, the middle
+    _run_prefill("qwen2.5-7b-1m-prefill", [0, 1, 127, 128, 255, 256, 8191, 8192, 16256, 16383])
 
 
 @pytest.mark.parametrize("name,n_rows", [("llama3.2-3b-decode-128k", 32),

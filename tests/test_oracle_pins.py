@@ -208,6 +208,21 @@ def test_count_rows_equals_bruteforce(D, alpha):
             assert bf == rw, (D, alpha, g, Nq, Nk, q0, k0)
 
 
+def test_count_rows_equals_workload_counts():
+    """The oracle's row-by-row count at the benchmark workloads' full sizes against
+    tests/golden/workload_counts.json, exact integers from per-pair arithmetic series
+    (ATFlash Abstract: the pruned share has a closed form), computed without the
+    oracle: a dropped row, an off-by-one distance range or a wrong group threshold
+    in the oracle changes these counts."""
+    with open(os.path.join(GOLD, "workload_counts.json")) as fh:
+        gold = json.load(fh)
+    assert len(gold["workloads"]) == 7
+    for w in gold["workloads"]:
+        got = oracle.count_rows(w["D"], w["base"], w["alpha"], w["g"], w["Nq"], w["Nk"],
+                                w["q_pos0"], w["k_pos0"])
+        assert got == (w["pruned"], w["total"]), w["name"]
+
+
 def test_pruned_fraction_grows_logarithmically():
     """Continuum form of the count for a causal N x N square (our derivation of
     the ATFlash Abstract's 'closed form logarithmic in N'):
