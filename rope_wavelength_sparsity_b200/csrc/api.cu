@@ -110,11 +110,10 @@ int encode_bf16_4d_strided(CUtensorMap* map, const void* base, const cuuint64_t 
   return r == CUDA_SUCCESS ? WPATTN_OK : WPATTN_ECUDA;
 }
 
-// bf16 tensor map of a [d3, d1, d2, d0] tensor (d0 contiguous); `promote`
-// widens each L2 miss to 256 bytes (whole rows of a head), which suits copies
-// of whole rows but not copies that want only some columns of each row
+// bf16 tensor map of a [d3, d1, d2, d0] tensor (d0 contiguous), L2 misses
+// widened to 256 bytes (whole rows of a head)
 int encode_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                   uint64_t d3, uint32_t box0, uint32_t box1, bool swizzle128, bool promote = true) {
+                   uint64_t d3, uint32_t box0, uint32_t box1, bool swizzle128) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return WPATTN_ECUDA;
   const cuuint64_t dims[4] = {d0, d1, d2, d3};
@@ -124,8 +123,7 @@ int encode_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                         promote ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? WPATTN_OK : WPATTN_ECUDA;
 }
 
@@ -257,11 +255,8 @@ int launch_decode(const DecodeParams& prm, int gc, bool pm, cudaStream_t st) {
     if ((rc = encode_bf16_4d(&tv, prm.v, D, prm.page_size, prm.Hkv, prm.num_pages, 64, R, true)) != WPATTN_OK)
       return rc;
   } else {
-    // caches are [B, Lmax, Hkv, D]: dims (fastest first) D, Lmax, Hkv, B.  K in 16-dim x
-    // 32-key boxes (one 32-byte sector column), only the columns of kept groups, with no
-    // L2 promotion so that a miss fetches only the sectors asked for
-    if ((rc = encode_bf16_4d(&tk, prm.k, D, prm.Lmax, prm.Hkv, prm.B, 16, KB, false, false)) !=
-        WPATTN_OK)
+    // caches are [B, Lmax, Hkv, D]: dims (fastest first) D, Lmax, Hkv, B; 64-dim x 32-key boxes
+    if ((rc = encode_bf16_4d(&tk, prm.k, D, prm.Lmax, prm.Hkv, prm.B, 64, KB, true)) != WPATTN_OK)
       return rc;
   }
   if (!prm.block_table &&

@@ -9,11 +9,14 @@
 // and V through a shared-memory ring with TMA; each block is consumed by one
 // of four compute warps, which run both contractions on warp-level tensor-
 // core MMAs (mma.sync m16n8k16): S^T = K Q^T over the groups of 8 pairs still
-// kept in the block, then O^T += V^T P^T.  K is loaded only from the block's
-// first kept group on: in 32-byte sector columns of each half of the head
-// dim for the [B, L, Hkv, D] cache, or in 1 KB slabs for the pair-major
-// cache; a paged cache moves whole rows.  A second kernel merges the key
-// ranges by their log-sum-exp.
+// kept in the block, then O^T += V^T P^T.  With the pair-major K cache only
+// the slabs of the block's kept groups are loaded (1 KB each).  In the
+// [B, L, Hkv, D] layout (contiguous or paged) whole K rows are loaded: each
+// 128-byte half of a row holds one half of every pair, DRAM moves whole half
+// rows whatever part of them is asked for (measured with 32-byte column
+// copies: the same DRAM bytes as whole rows), and the kept slice reaches
+// into both halves at every distance.  A second kernel merges the key ranges
+// by their log-sum-exp.
 #pragma once
 
 #include "device_util.cuh"
@@ -54,13 +57,9 @@ struct DecodeParams {
   double theta[64];
 };
 
-// Shared-memory ring of the split kernel: blocks of KB keys of K and V, plus
-// the query heads, the thresholds and each warp's p row.  V (and K of a
-// paged cache) is in the 128-byte-swizzled layout TMA writes (64-dim panels,
-// row = key).  K of a [B, L, Hkv, D] cache is in sector columns: column c of
-// half h (dims h * D/2 + 16c .. + 16, one 32-byte DRAM sector of each row)
-// of the block's keys at (2c + h) * KB * 32, key r at 32 r; a group g of 8
-// pairs is the 16 bytes at (g & 1) * 16 of column g / 2 in both halves.
+// Shared-memory ring of the split kernel: blocks of KB keys of K and V in
+// the 128-byte-swizzled layout TMA writes (64-dim panels, row = key), plus
+// the query heads, the thresholds and each warp's p row.
 constexpr int kDecodeComputeWarps = 4;
 
 template <int D>
@@ -144,7 +143,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   const int nblk = j_end > j_begin ? (j_end - j_begin + KB - 1) / KB : 0;
   const int qpos = p.q_pos[b];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool paged = !PM && p.block_table != nullptr;  // K in swizzled rows, not sector columns
+  const bool paged = !PM && p.block_table != nullptr;
   // first group of 8 pairs kept for some key of the block starting at j0:
   // groups whose largest threshold is below the block's smallest distance
   // (that of its last real key) are pruned for every key of the block
@@ -228,10 +227,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       nsub = (min(j0 + KB, j_end) - j0 + R - 1) / R;
     };
     if (paged && nblk > 0) plan_block(0);
-    // first kept group of the next block, found while its stage drains (with
-    // explicit key positions it is only known once the keys are: load them all)
-    auto first_loaded_group = [&](int j0) -> int { return p.k_pos ? 0 : first_kept_group(j0); };
-    int g0_next = nblk > 0 ? first_loaded_group(j_begin) : 0;
+    // pair-major: first slab of the next block, found while its stage drains
+    int g0_next = (PM && nblk > 0) ? first_kept_group(j_begin) : 0;
     int issued = 0;           // blocks whose copies were issued
     bool ok_prod = true;
     for (int i = 0; i < nblk; ++i) {
@@ -265,22 +262,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           mbar_arrive_expect_tx(full(s), (NG - g0) * KB * 32 + L::TILE);
           for (int g = g0; g < NG; ++g)
             tma_load_4d(sbase + L::OFF_K + s * L::TILE + g * KB * 32, &tmK, full(s), 0, j0, kvh * NG + g, b);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(sbase + L::OFF_V + s * L::TILE + c * L::PANEL, &tmV, full(s), 64 * c, j0, kvh, b);
         } else {
-          // the 32-byte sector columns of both halves from the one holding group g0
-          constexpr int NC = P / 16;
-          const int c0 = g0 >> 1;
-          mbar_arrive_expect_tx(full(s), 2 * (NC - c0) * KB * 32 + L::TILE);
-          for (int c = c0; c < NC; ++c)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
-              tma_load_4d(sbase + L::OFF_K + s * L::TILE + (2 * c + hf) * KB * 32, &tmK, full(s),
-                          hf * P + 16 * c, j0, kvh, b);
+          mbar_arrive_expect_tx(full(s), 2 * L::TILE);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_4d(sbase + L::OFF_K + s * L::TILE + c * L::PANEL, &tmK, full(s), 64 * c, j0, kvh, b);
+            tma_load_4d(sbase + L::OFF_V + s * L::TILE + c * L::PANEL, &tmV, full(s), 64 * c, j0, kvh, b);
+          }
         }
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sbase + L::OFF_V + s * L::TILE + c * L::PANEL, &tmV, full(s), 64 * c, j0, kvh, b);
       }
       issued = i + 1;
-      if (i + 1 < nblk) g0_next = first_loaded_group(j0 + KB);
+      if (PM && i + 1 < nblk) g0_next = first_kept_group(j0 + KB);
     }
     if (!ok_prod) {
       // A wait ran out: copies issued into the ring may still be landing.
@@ -372,11 +365,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           uint32_t addr;
           if (PM) {
             addr = smem_u32(kt) + g * KB * 32 + key * 32 + lhalf * 16;
-          } else if (paged) {
+          } else {
             const int ch = lhalf ? NG + g : g;
             addr = smem_u32(kt) + (ch >> 3) * L::PANEL + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
-          } else {  // sector column g / 2 of half lhalf, group g's 16 bytes in it
-            addr = smem_u32(kt) + (2 * (g >> 1) + lhalf) * KB * 32 + key * 32 + (g & 1) * 16;
           }
           uint32_t a0, a1, a2, a3;
           ldsm_x4(addr, a0, a1, a2, a3);

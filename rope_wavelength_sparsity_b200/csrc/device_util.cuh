@@ -76,6 +76,27 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   return true;
 }
 
+// Non-blocking test of a phase: on a phase that has already completed it
+// answers in ~20 cycles, against ~50 for a try with a suspend-time hint.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait for the few hand-off points where the phase has often completed
+// already: a cheap test first.  (Used sparingly: every inlined site of the
+// test grows the code more than the hinted try does.)
+__device__ __forceinline__ bool mbar_wait_handoff(uint32_t bar, uint32_t parity) {
+  return mbar_test(bar, parity) || mbar_wait(bar, parity);
+}
+
 // ---------------------------------------------------------------- TMA loads
 // Four 8x8 b16 matrices from shared memory: lane t gives the address of row
 // t % 8 of matrix t / 8 (16 bytes each); register m receives, for matrix m,

@@ -484,7 +484,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const bool do_qk = ok && next && in_n;
           const int ps_n = do_qk ? plan_qk(t, kt_n, (j + 1) % NS) : 0;
           if (ok && in_j) {
-            if (!mbar_wait(p_full(t), cnt[t] & 1)) { ok = false; }
+            if (!mbar_wait_handoff(p_full(t), cnt[t] & 1)) { ok = false; }
             if (ok) {
               tc_fence_after();
 #pragma unroll
@@ -617,7 +617,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (lane == 0) mbar_arrive(k_empty(s));
       }
 
-      if (!__all_sync(FULL, mbar_wait(s_full(t), cnt & 1))) { ok = false; break; }
+      if (!__all_sync(FULL, mbar_wait_handoff(s_full(t), cnt & 1))) { ok = false; break; }
       tc_fence_after();
       if (corr && G8) {
         const uint8_t* kb = smem + L::OFF_K + s * L::KTILE;
@@ -840,6 +840,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
       for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(tS + 32 * cc, &sc[32 * cc]);
       tmem_ld_wait();
+      // the loaded values are only defined after the wait: keep every use of
+      // them below it (an empty asm that takes each register as an operand)
+#pragma unroll
+      for (int c = 0; c < BN; ++c) asm volatile("" : "+f"(sc[c]));
 
       if (all_pruned) {
 #pragma unroll

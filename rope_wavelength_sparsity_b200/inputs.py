@@ -65,6 +65,8 @@ WORKLOADS = {
                                    5e5, 1.0, 1),
     "llama3.2-3b-decode-32k": Workload("llama3.2-3b-decode-32k", "decode", 4, 24, 8, 128, 1,
                                        32768, 5e5, 1.0, 1),
+    "qwen2.5-7b-64k-chunk": Workload("qwen2.5-7b-64k-chunk", "prefill", 1, 28, 4, 128, 16384,
+                                     65536, 1e7, 1.0, 8, q_pos0=65536 - 16384),
 }
 
 

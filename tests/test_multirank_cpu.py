@@ -165,3 +165,30 @@ def test_shard_keys_bounds():
     assert wd.shard_keys([100, 30, 0], 0, 40) == ([0, 0, 0], [40, 30, 0])
     assert wd.shard_keys([100, 30, 0], 1, 40) == ([40, 40, 40], [40, 0, 0])
     assert wd.shard_keys([100, 30, 0], 2, 40) == ([80, 80, 80], [20, 0, 0])
+
+
+def test_reference_arm_loads_no_product_library():
+    """The oracle arm (``--impl reference``) counts its work with the oracle and loads
+    nothing from the library: run it in a fresh process and read that process's
+    mapped files."""
+    import json
+    import subprocess
+    code = (
+        "import json, sys\n"
+        f"sys.path.insert(0, {ROOT!r})\n"
+        "import bench\n"
+        "class A:\n"
+        "    workload, steps, warmup, ref_seconds = 'tiny', 1, 1, 0.5\n"
+        "rank, res = bench.reference_arm(A())\n"
+        "maps = open('/proc/self/maps').read()\n"
+        "print(json.dumps({'res': res, 'wpattn': 'libwpattn' in maps,\n"
+        "                  'oracle': 'liboracle' in maps}))\n")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         timeout=600, env={**os.environ, "WORLD_SIZE": "1", "RANK": "0"})
+    assert out.returncode == 0, out.stderr[-2000:]
+    got = json.loads(out.stdout.strip().splitlines()[-1])
+    assert got["oracle"] and not got["wpattn"]
+    res = got["res"]
+    assert res["impl"] == "reference" and res["value"] > 0
+    assert res["config"]["workload"] == "tiny" and res["config"]["Nk"] == 256
+    assert res["cpu_baseline"]["cores"] >= 1 and res["cpu_baseline"]["kind"] == "oracle"

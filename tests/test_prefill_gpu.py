@@ -57,6 +57,34 @@ def test_prefill_cases_all_rows(cuda_dev, case):
                    k_pos0=k0, what=str(case))
 
 
+# More edges of the D = 64, g = 8 shape: large logits (the running max jumps,
+# so O is rescaled), a chunk at the end of the keys, the window off, a CTA whose
+# second query tile is empty, rows that see no key, group edges inside tiles.
+G8_EDGE_CASES = [
+    # D, g, alpha, base, B, Hq, Hkv, Nq, Nk, q0, k0, input scale
+    (64, 8, 1.0, 1e6, 1, 2, 1, 1000, 1000, 0, 0, 3.0),     # large logits: the lazy O rescale
+    (64, 8, 1.0, 1e6, 1, 3, 1, 300, 1500, 1200, 0, 3.0),   # chunk at the end of the keys
+    (64, 8, float("inf"), 1e6, 1, 2, 2, 700, 700, 0, 0, 1.0),  # window off
+    (64, 8, 1.0, 1e4, 1, 2, 1, 100, 900, 800, 0, 1.0),     # second query tile empty
+    (64, 8, 1.0, 1e4, 1, 2, 1, 200, 200, 0, 60, 2.0),      # first rows see no key
+    (64, 8, 0.05, 1e4, 2, 4, 2, 513, 513, 0, 0, 3.0),      # group edges inside tiles, batch 2
+]
+
+
+@pytest.mark.parametrize("case", G8_EDGE_CASES, ids=[str(i) for i in range(len(G8_EDGE_CASES))])
+def test_prefill_g8_edges_all_rows(cuda_dev, case):
+    D, g, alpha, base, B, Hq, Hkv, Nq, Nk, q0, k0, amp = case
+    q, k, v = _qkv(B, Nq, Nk, Hq, Hkv, D, seed=len(str(case)) + 500)
+    # q and k scaled up: large logits, so the running max jumps and O is rescaled;
+    # v scaled down by the same factor: with near one-hot rows the bf16 rounding of
+    # P (relative 2^-8) times max |v| must stay inside the output tolerance
+    q = (q.float() * amp).to(torch.bfloat16)
+    k = (k.float() * amp).to(torch.bfloat16)
+    v = (v.float() / amp).to(torch.bfloat16)
+    prefill_parity(q, k, v, Hq=Hq, Hkv=Hkv, D=D, base=base, alpha=alpha, g=g, q_pos0=q0,
+                   k_pos0=k0, what=str(case))
+
+
 def test_planted_key_small(cuda_dev):
     w = inputs.Workload("plant", "prefill", 1, 8, 2, 128, 1500, 1500, 5e5, 1.0, 1, plant_key=True)
     q, k, v, planted = inputs.prefill_inputs(w, seed=3)
