@@ -329,32 +329,6 @@ __device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// 2^x for a pair, on the FMA and integer pipes instead of the MUFU unit.
-// Range reduction x = n + f with n = round(x), f in [-1/2, 1/2]: adding
-// 1.5 * 2^23 leaves n in the low mantissa bits of y, so n is exact, and
-// ((bits(y) + 127) << 23) is the float 2^n (0.0 when n = -127).  2^f is a
-// degree-3 polynomial fitted for minimum maximum relative error on
-// [-1/2, 1/2] (Lawson's iteratively reweighted least squares, our own fit);
-// with fp32 Horner evaluation its relative error stays below 8e-5.  Inputs
-// are clamped to -127, so -inf (a masked score) gives exactly 0.
-__device__ __forceinline__ void exp2_poly2(float& r0, float& r1, float x0, float x1) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261117f, c3 = 0.05517166f;
-  x0 = fmaxf(x0, -127.f);
-  x1 = fmaxf(x1, -127.f);
-  float y0, y1, n0, n1, f0, f1;
-  add2(y0, y1, x0, x1, kShift, kShift);
-  add2(n0, n1, y0, y1, -kShift, -kShift);
-  add2(f0, f1, x0, x1, -n0, -n1);
-  float p0, p1;
-  fma2(p0, p1, c3, c3, f0, f1, c2, c2);
-  fma2(p0, p1, p0, p1, f0, f1, c1, c1);
-  fma2(p0, p1, p0, p1, f0, f1, c0, c0);
-  const float s0 = __uint_as_float((__float_as_uint(y0) + 127u) << 23);
-  const float s1 = __uint_as_float((__float_as_uint(y1) + 127u) << 23);
-  mul2(r0, r1, p0, p1, s0, s1);
-}
-
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) {
   return __uint_as_float(v & 0xFFFF0000u);

@@ -95,7 +95,6 @@ template <int D>
 struct PrefillSmem {
   static constexpr int QT = PrefillShape<D>::QT, BN = PrefillShape<D>::BN;
   static constexpr int NS = (D == 64 && QT > 1) ? 4 : 2;  // K/V ring depth
-  static constexpr int NPOLY = 0;                    // of every 8 column pairs, exp2 on the FMA pipe
   static constexpr int QTILE = kBM * D * 2;          // one Q tile in bytes
   static constexpr int KTILE = BN * D * 2;           // one K or V tile in bytes
   static constexpr int PANEL_Q = kBM * 16;           // one 8-dim panel of a Q tile
@@ -902,12 +901,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const int c = 2 * i;
           float x0, x1, e0, e1;
           fma2(x0, x1, sc[c], sc[c + 1], sl, sl, nm, nm);
-          if ((i & 7) >= 8 - L::NPOLY) {
-            exp2_poly2(e0, e1, x0, x1);
-          } else {
-            e0 = ex2_approx(x0);
-            e1 = ex2_approx(x1);
-          }
+          e0 = ex2_approx(x0);
+          e1 = ex2_approx(x1);
           add2(acc[2 * (i & 3)], acc[2 * (i & 3) + 1], acc[2 * (i & 3)], acc[2 * (i & 3) + 1], e0, e1);
           pk[i] = pack_bf16x2(e0, e1);
           if constexpr (BN == 96) {
