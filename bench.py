@@ -58,12 +58,14 @@ FLUSH_BYTES = 512 << 20
 # ncu capture, keyed by workload and by a hash of that kernel's sources at
 # capture time: a changed kernel reports null until it is captured again.
 NCU_TRAFFIC = {
-    # prefill_kernel<64, g8> on the Qwen2.5-0.5B 32K workload: 76.266496 MB read + 26.896128 MB
-    # written
-    ("qwen2.5-0.5b-32k", "08e5772bb4e2955c"): 76266496 + 26896128,
-    # decode_split_kernel<128, 3, 0> on the reduced B=4, L=32768 Llama decode: 536.940032 MB read
-    # + 3.973632 MB written, scaled by the 16x keys x heads of the B=16, L=131072 call
-    ("llama3.2-3b-decode-128k", "bdf11727c8e434b8"): 16 * (536940032 + 3973632),
+    # prefill_kernel<128, 1, 0, 0> on the full 1M-key chunk (one pass): 54.71 GB read + 131.40 MB
+    # written; K and V (2.15 GB) come from DRAM about 24 times, at 4 % of the HBM bandwidth
+    ("qwen2.5-7b-1m-prefill", "4507275ab3553a09"): 54710000000 + 131400000,
+    # prefill_kernel<64, 1, 0, 0> on the Qwen2.5-0.5B 32K prefill (one pass): 76.28 MB + 23.42 MB
+    ("qwen2.5-0.5b-32k", "4507275ab3553a09"): 76280000 + 23420000,
+    # decode_split_kernel<128, 3, 0> on the full B=16, L=131072 Llama decode (one pass):
+    # 8.59 GB read + 3.85 MB written (all of K and V: whole rows of the [B, L, Hkv, D] cache)
+    ("llama3.2-3b-decode-128k", "7808fd5285038f87"): 8590000000 + 3850000,
 }
 
 KERNEL_SOURCES = {"prefill": ("prefill_kernel.cuh", "device_util.cuh"),

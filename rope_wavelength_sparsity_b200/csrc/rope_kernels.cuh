@@ -49,11 +49,14 @@ struct RopeParams {
 // One thread per (token, chunk of 8 pairs): the eight angles of the chunk are
 // turned into cosines and sines once and reused for every head of the token;
 // per head two 16-byte loads (dims 8c..8c+7 and D/2+8c..D/2+8c+7) and two
-// 16-byte stores.  Grid-stride over the (token, chunk) items; every element
-// is read before the same thread writes it, so out may alias x.
+// 16-byte stores.  Heads go four at a time, all four heads' loads issued
+// before any of their stores, so that each thread keeps 128 bytes in flight
+// instead of waiting a memory round trip per head.  Every element is read
+// before the same thread writes it (and a thread's heads are disjoint), so
+// out may alias x.  Grid-stride over the (token, chunk) items.
 template <int D>
 __global__ void __launch_bounds__(256) rope_kernel(const __grid_constant__ RopeParams p) {
-  constexpr int P = D / 2, NC = P / 8;
+  constexpr int P = D / 2, NC = P / 8, HB = 4;
   const uint64_t n = static_cast<uint64_t>(p.B) * p.N * NC;
   for (uint64_t idx = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < n;
        idx += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
@@ -64,11 +67,8 @@ __global__ void __launch_bounds__(256) rope_kernel(const __grid_constant__ RopeP
     float cs[8], sn[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) rope_cos_sin(pos, p.theta[8 * c + e], cs[e], sn[e]);
-    for (int h = 0; h < p.H; ++h) {
-      const uint64_t th = token * static_cast<uint64_t>(p.H) + h;
-      const uint16_t* row = p.x + th * D;
-      const uint4 lo = *reinterpret_cast<const uint4*>(row + 8 * c);
-      const uint4 hi = *reinterpret_cast<const uint4*>(row + P + 8 * c);
+    // rotate one head's two 16-byte chunks and store them
+    auto rotate_store = [&](uint64_t th, const uint4& lo, const uint4& hi) {
       const uint32_t a[4] = {lo.x, lo.y, lo.z, lo.w};
       const uint32_t b[4] = {hi.x, hi.y, hi.z, hi.w};
       uint32_t ra[4], rb[4];
@@ -83,6 +83,25 @@ __global__ void __launch_bounds__(256) rope_kernel(const __grid_constant__ RopeP
       uint16_t* orow = p.out + th * D;
       *reinterpret_cast<uint4*>(orow + 8 * c) = make_uint4(ra[0], ra[1], ra[2], ra[3]);
       *reinterpret_cast<uint4*>(orow + P + 8 * c) = make_uint4(rb[0], rb[1], rb[2], rb[3]);
+    };
+    const uint64_t th0 = token * static_cast<uint64_t>(p.H);
+    int h = 0;
+    for (; h + HB <= p.H; h += HB) {
+      uint4 lo[HB], hi[HB];
+#pragma unroll
+      for (int u = 0; u < HB; ++u) {
+        const uint16_t* row = p.x + (th0 + h + u) * D;
+        lo[u] = *reinterpret_cast<const uint4*>(row + 8 * c);
+        hi[u] = *reinterpret_cast<const uint4*>(row + P + 8 * c);
+      }
+#pragma unroll
+      for (int u = 0; u < HB; ++u) rotate_store(th0 + h + u, lo[u], hi[u]);
+    }
+    for (; h < p.H; ++h) {
+      const uint16_t* row = p.x + (th0 + h) * D;
+      const uint4 lo = *reinterpret_cast<const uint4*>(row + 8 * c);
+      const uint4 hi = *reinterpret_cast<const uint4*>(row + P + 8 * c);
+      rotate_store(th0 + h, lo, hi);
     }
   }
 }
