@@ -21,7 +21,9 @@ step; decode: algorithmic GB/s = K bytes of the kept pairs + all V bytes
 (+ q and out) over the decode call's device time.
 
 Timing: CUDA events on the launching stream around every step, an L2 flush
-(a 512 MiB write) between steps outside the events, W warm-up steps, barrier
+(a 512 MiB write, then a read of 256 MiB of it, so that the flush's own dirty
+lines are written back before the step rather than inside it) between steps
+outside the events, W warm-up steps, barrier
 + synchronize around the timed region, max over ranks.  Multi-GPU: every rank
 runs its own independent problem (weak scaling, no data-path collective).
 
@@ -53,6 +55,8 @@ NESTED_DECODE = ("llama3.2-3b-decode-128k", "qwen2.5-7b-1m-decode")
 # the block-mask, pre-RoPE and explicit-positions variants run on this one
 VARIANTS_WORKLOAD = "qwen2.5-0.5b-32k"
 FLUSH_BYTES = 512 << 20
+FLUSH_NOTE = ("flushed between steps (512 MiB write, then a 256 MiB read of it: no dirty "
+              "line of the flush is written back inside a step)")
 
 # DRAM bytes (read + write) per launch of a workload's dominant kernel from one
 # ncu capture, keyed by workload and by a hash of that kernel's sources at
@@ -64,8 +68,8 @@ NCU_TRAFFIC = {
     # prefill_kernel<64, 1, 0, 0> on the Qwen2.5-0.5B 32K prefill (one pass): 76.28 MB + 23.42 MB
     ("qwen2.5-0.5b-32k", "4507275ab3553a09"): 76280000 + 23420000,
     # decode_split_kernel<128, 3, 0> on the full B=16, L=131072 Llama decode (one pass):
-    # 8.59 GB read + 3.85 MB written (all of K and V: whole rows of the [B, L, Hkv, D] cache)
-    ("llama3.2-3b-decode-128k", "7808fd5285038f87"): 8590000000 + 3850000,
+    # 8.59 GB read + 3.66 MB written (all of K and V: whole rows of the [B, L, Hkv, D] cache)
+    ("llama3.2-3b-decode-128k", "668b26ccc741d486"): 8590000000 + 3660000,
 }
 
 KERNEL_SOURCES = {"prefill": ("prefill_kernel.cuh", "device_util.cuh"),
@@ -100,12 +104,12 @@ def workload_config(w, world: int) -> dict:
                 "Nq": w.Nq, "Nk": w.Nk, "q_pos0": w.q_pos0, "rope_base": w.base,
                 "alpha": w.alpha, "group_pairs": w.g, "global_batch": w.B * world,
                 "seq_len": w.Nk, "parallelism": f"independent problem per GPU x{world}",
-                "l2": "flushed between steps (512 MiB write)"}
+                "l2": FLUSH_NOTE}
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.Nk,
             "rope_base": w.base, "alpha": w.alpha, "group_pairs": w.g,
             "global_batch": w.B * world, "seq_len": w.Nk,
             "parallelism": f"independent problem per GPU x{world}",
-            "l2": "flushed between steps (512 MiB write)"}
+            "l2": FLUSH_NOTE}
 
 
 # ----------------------------------------------------------- work accounting
@@ -324,13 +328,25 @@ def bench_prefill(w, args, world, rank, dev, flush, peaks, variants=False):
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
     eff, off_flops = prefill_flops(w, win, wp)
+    # the library's key-range split plan for this grid, its workspace made once
+    main_items, split_items, parts = wp.prefill_split_plan(w.B, w.Nq, w.Nk, w.Hq, w.q_pos0, w.k_pos0)
+    S = 0 if split_items else 1
+    nws = wp.prefill_split_workspace_size(w.B, w.Nq, w.Nk, w.Hq, w.D, w.q_pos0, w.k_pos0, 0)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev) if split_items else None
+    # the prefill kernel; with a split, the split items' kernel and their merge
+    launches = (1 if main_items else 0) + (2 if split_items else 0)
 
     def step():
-        wp.prefill(q, k, v, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale, out=out, lse=lse)
+        wp.prefill(q, k, v, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale, out=out, lse=lse,
+                   kv_splits=S, workspace=ws)
 
     def step_off():
         wp.prefill(q, k, v, win_off, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale, out=out,
-                   lse=lse)
+                   lse=lse, kv_splits=S, workspace=ws)
+
+    def step_unsplit():
+        wp.prefill(q, k, v, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale, out=out, lse=lse,
+                   kv_splits=1)
 
     clocks = ClockSampler(dev.index) if rank == 0 else None
     total_ms, per, clk = time_steps(step, args.warmup, args.steps, flush, world, clocks)
@@ -340,6 +356,12 @@ def bench_prefill(w, args, world, rank, dev, flush, peaks, variants=False):
     _check_status(wp, w.name + " window off")
     ms_step = total_ms / args.steps
     off_ms_step = off_ms / n_off
+    unsplit = None
+    if split_items:
+        un_ms, _, _ = time_steps(step_unsplit, 1, n_off, flush, world)
+        _check_status(wp, w.name + " unsplit")
+        unsplit = {"ms_per_step": round(un_ms / n_off, 4),
+                   "speedup_of_split": round((un_ms / n_off) / ms_step, 3)}
     kernel_ms = statistics.mean(per)
     achieved = eff / (kernel_ms * 1e-3) / 1e12
     peak_t, peak_label = _tensor_peak(peaks, clk, total_ms)
@@ -357,10 +379,14 @@ def bench_prefill(w, args, world, rank, dev, flush, peaks, variants=False):
         "work": {"effective_tflop_per_step": round(world * eff / 1e12, 4),
                  "window_off_tflop_per_step": round(world * off_flops / 1e12, 4),
                  "pruned_fraction": wp.pruned_fraction(win, w.Nq, w.Nk, w.q_pos0, w.k_pos0)[2]},
-        "gpu_launches": args.steps,
+        "split_plan": {"unsplit_items": main_items, "split_items": split_items,
+                       "parts_per_split_item": parts},
+        "gpu_launches": launches * args.steps,
         "clocks": clk,
         "config": workload_config(w, world),
     }
+    if unsplit:
+        res["unsplit"] = unsplit
     if variants:
         res.update(_prefill_variants(w, args, world, rank, dev, flush, peaks, q, k, v, out, lse,
                                      win, eff, ms_step))
@@ -375,7 +401,7 @@ def bench_prefill(w, args, world, rank, dev, flush, peaks, variants=False):
         kd = k.copy_(kh, non_blocking=True)
         vd = v.copy_(vh, non_blocking=True)
         o, _ = wp.prefill(qd, kd, vd, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale,
-                          out=out, lse=lse)
+                          out=out, lse=lse, kv_splits=S, workspace=ws)
         oh.copy_(o, non_blocking=True)
 
     n_e2e = max(5, args.steps // 4)
@@ -384,7 +410,7 @@ def bench_prefill(w, args, world, rank, dev, flush, peaks, variants=False):
     res["e2e"] = {"value": round(world * eff / (e2e_ms / n_e2e * 1e-3) / 1e12, 2),
                   "unit": "TFLOP/s", "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * 2,
                   "d2h_bytes_per_step": out.numel() * 2}
-    del q, k, v, out, lse, qh, kh, vh, oh
+    del q, k, v, out, lse, qh, kh, vh, oh, ws
     torch.cuda.empty_cache()
     return res
 
@@ -437,8 +463,7 @@ def _prefill_variants(w, args, world, rank, dev, flush, peaks, q, k, v, out, lse
                         lse=lse, workspace=ws_r)
 
     def step_rope_only():
-        wp.rope(q, base=w.base, pos0=w.q_pos0, out=qr_buf)
-        wp.rope(k, base=w.base, pos0=w.k_pos0, out=kr_buf)
+        wp.rope_qk(q, k, base=w.base, q_pos0=w.q_pos0, k_pos0=w.k_pos0, q_out=qr_buf, k_out=kr_buf)
 
     rp_ms, _, _ = time_steps(step_rope_prefill, args.warmup, n_v, flush, world)
     ro_ms, ro_per, _ = time_steps(step_rope_only, args.warmup, n_v, flush, world)
@@ -450,13 +475,13 @@ def _prefill_variants(w, args, world, rank, dev, flush, peaks, q, k, v, out, lse
                                  "value": round(weak_scaling_value(eff, world, rp_ms / n_v) / 1e12, 2),
                                  "unit": "TFLOP/s",
                                  "overhead_vs_prefill": round((rp_ms / n_v) / ms_step - 1.0, 4),
-                                 "gpu_launches": 3 * n_v},
+                                 "gpu_launches": 2 * n_v},
         "rotation_kernels": {"ms_per_step": round(ro_ms / n_v, 4),
                              "roofline": {"bound": "hbm", "achieved": round(ro_gbs, 1),
                                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                           "frac": round(ro_gbs / peaks["hbm_gbs"], 4),
                                           "traffic": None},
-                             "bytes_per_step": rope_bytes, "gpu_launches": 2 * n_v},
+                             "bytes_per_step": rope_bytes, "gpu_launches": n_v},
     }
     del ws_r, qr_buf, kr_buf
     # the same prefill through the explicit-positions kernel, given the workload's own
@@ -640,8 +665,14 @@ def gpu_arm(args):
     w = inputs.WORKLOADS[args.workload]
     flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
+    flush_words = flush_buf[: FLUSH_BYTES // 2].view(torch.int32)
+
     def flush():
+        # the write evicts every line of the step's inputs; the read then
+        # replaces the write's dirty lines with clean ones, so their write-back
+        # is not charged to the next step
         flush_buf.fill_(1)
+        flush_words.sum()
 
     result = _run_workload(args.workload, args, world, rank, dev, flush, peaks)
     if args.workload == DEFAULT_WORKLOAD and not args.only_primary:

@@ -117,6 +117,60 @@ WPATTN_API int wpattn_prefill(const wpattn_window *w,
                    void *cuda_stream);
 
 /*
+ * Prefill with the key ranges of some work items split into parts (flash-
+ * decoding's split along the keys, applied to prefill CTAs).  A work item is
+ * one 256-row query block of one head of one sequence: one CTA of
+ * wpattn_prefill's grid.  A split item runs as P CTAs, one per range of
+ * ceil(nkt / P) key tiles of 128 keys (a range past the last key tile is
+ * dropped); each writes its rows' fp32 result, normalised over its own keys,
+ * and the log2-sum-exp of its scores into the workspace, and a merge kernel
+ * combines the parts (weights 2^(l_s - max l)) into out and lse.  The items
+ * that are not split run in wpattn_prefill's kernel, unchanged.
+ *   kv_splits = 0: the library's plan (wpattn_prefill_split_plan) on the
+ *                  current device; it splits only the items of the grid's last
+ *                  partial wave, and only when every item does the same work;
+ *   kv_splits = 1: nothing is split (wpattn_prefill);
+ *   kv_splits = 2 .. 64: every item in kv_splits parts.
+ * Same arguments and results as wpattn_prefill (equal to it up to float
+ * rounding order), plus:
+ *   workspace: device, 256-byte aligned, at least
+ *              wpattn_prefill_split_workspace_size(...) bytes when the plan
+ *              splits anything (else WPATTN_EWORKSPACE; WPATTN_EINVAL when
+ *              NULL or misaligned); unused otherwise.
+ * kv_splits outside 0 .. 64: WPATTN_EINVAL.
+ */
+WPATTN_API int wpattn_prefill_split(const wpattn_window *w,
+                   const void *q, const void *k, const void *v,
+                   void *out, float *lse,
+                   int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
+                   int64_t q_pos0, int64_t k_pos0, float softmax_scale,
+                   int32_t kv_splits, void *workspace, size_t workspace_bytes,
+                   void *cuda_stream);
+
+/*
+ * The split plan of wpattn_prefill_split on a device with num_sms SMs
+ * (num_sms <= 0: the current device).  Host only.  Outputs (any may be NULL):
+ * the items run unsplit (the first main_items in grid order), the items split
+ * after them, and the parts of each split item (1 when none is split).
+ * kv_splits = 0 plans as follows: when the last query sees at most 10% more
+ * keys than the first (a chunk far into a long context), every item takes the
+ * same time, and with one CTA per SM a grid of W full waves plus r < num_sms
+ * items leaves most SMs idle while the last r run.  Those r items are split
+ * into min(8, num_sms / r) parts of at least 64 key tiles, so they take a
+ * fraction of a wave; nothing is split when r = 0 or fewer than 2 parts fit.
+ */
+WPATTN_API int wpattn_prefill_split_plan(int32_t B, int32_t Nq, int32_t Nk, int32_t Hq,
+                   int64_t q_pos0, int64_t k_pos0, int32_t kv_splits, int32_t num_sms,
+                   int64_t *main_items, int32_t *split_items, int32_t *parts);
+
+/* Workspace bytes of wpattn_prefill_split for that plan: parts * split items *
+ * 256 * (head_dim + 1) * 4; 0 when nothing is split or on bad sizes.  Host
+ * only (num_sms <= 0: the current device). */
+WPATTN_API size_t wpattn_prefill_split_workspace_size(int32_t B, int32_t Nq, int32_t Nk,
+                   int32_t Hq, int32_t head_dim, int64_t q_pos0, int64_t k_pos0,
+                   int32_t kv_splits, int32_t num_sms);
+
+/*
  * Prefill with a block mask stacked on the window (token-level block
  * sparsity of the MInference kind; ATFlash Abstract: the window is orthogonal
  * to token selection and composes with it).  Same arguments and results as
@@ -347,10 +401,25 @@ WPATTN_API int wpattn_rope(const void *x, void *out, int32_t B, int32_t N, int32
                   void *cuda_stream);
 
 /*
+ * The RoPE rotation of a prefill's queries and keys in one launch: q
+ * [B, Nq, Hq, head_dim] at positions q_pos0 + t into q_out, and k
+ * [B, Nk, Hkv, head_dim] at k_pos0 + j into k_out, each exactly as
+ * wpattn_rope would turn it (same rounding, same result bit for bit).
+ *   q, q_out, k, k_out: bf16 device, 16-byte aligned; q_out may be q and
+ *                       k_out may be k.  Nk = 0 turns q alone (k, k_out unused).
+ *   0 <= q_pos0, k_pos0 <= 2^40.
+ * head_dim in {64, 128} (else WPATTN_EUNSUPPORTED); rope_base > 1.
+ */
+WPATTN_API int wpattn_rope_qk(const void *q, void *q_out, const void *k, void *k_out,
+                  int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
+                  int32_t head_dim, int64_t q_pos0, int64_t k_pos0, double rope_base,
+                  void *cuda_stream);
+
+/*
  * Prefill from queries and keys that arrive before their RoPE rotation
  * (v is never rotated).  Arguments and results as for wpattn_prefill; q and
  * k are rotated with w->rope_base at their positions q_pos0 + t and
- * k_pos0 + j (wpattn_rope), into the workspace, then attended.  The rotation
+ * k_pos0 + j (wpattn_rope_qk, one launch), into the workspace, then attended.  The rotation
  * is a pre-pass rather than part of the attention kernel's producer: there
  * each key tile would be turned again by every query block that reads it,
  * on the special-function pipe the attention's exponentials already fill.

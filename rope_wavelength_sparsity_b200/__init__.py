@@ -77,12 +77,22 @@ def lib() -> ctypes.CDLL:
                                              ctypes.POINTER(ctypes.c_double)]
         L.wpattn_prefill.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64, i64,
                                      f32, vp]
+        L.wpattn_prefill_split.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64,
+                                           i64, f32, i32, vp, ctypes.c_size_t, vp]
+        L.wpattn_prefill_split_workspace_size.restype = ctypes.c_size_t
+        L.wpattn_prefill_split_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64, i64, i32, i32]
+        L.wpattn_prefill_split_plan.argtypes = [i32, i32, i32, i32, i64, i64, i32, i32,
+                                                ctypes.POINTER(ctypes.c_int64),
+                                                ctypes.POINTER(ctypes.c_int32),
+                                                ctypes.POINTER(ctypes.c_int32)]
         L.wpattn_prefill_masked.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64,
                                             i64, f32, vp, i32, vp]
         L.wpattn_pack_block_mask.argtypes = [vp, vp, i64, i32, i32, vp]
         L.wpattn_prefill_positions.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp,
                                                i64, vp, i64, f32, vp]
         L.wpattn_rope.argtypes = [vp, vp, i32, i32, i32, i32, i64, vp, ctypes.c_double, vp]
+        L.wpattn_rope_qk.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64,
+                                     ctypes.c_double, vp]
         L.wpattn_prefill_rope.argtypes = [wp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64, i64,
                                           f32, vp, ctypes.c_size_t, vp]
         L.wpattn_prefill_rope_workspace_size.restype = ctypes.c_size_t
@@ -200,13 +210,35 @@ def _prefill_shapes(q, k, v, w, out, lse):
     return B, Nq, Hq, D, Nk, Hkv
 
 
+def prefill_split_plan(B: int, Nq: int, Nk: int, Hq: int, q_pos0: int = 0, k_pos0: int = 0,
+                       kv_splits: int = 0, num_sms: int = 0):
+    """(main_items, split_items, parts) of ``prefill``'s key-range split: the work items
+    (256-row query blocks x heads x sequences) run unsplit, those split after them, and
+    the parts of each.  kv_splits 0 = the library's plan; num_sms 0 = this device."""
+    m, n, s = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().wpattn_prefill_split_plan(B, Nq, Nk, Hq, q_pos0, k_pos0, kv_splits, num_sms,
+                                           ctypes.byref(m), ctypes.byref(n), ctypes.byref(s)),
+           "wpattn_prefill_split_plan")
+    return m.value, n.value, s.value
+
+
+def prefill_split_workspace_size(B: int, Nq: int, Nk: int, Hq: int, D: int, q_pos0: int = 0,
+                                 k_pos0: int = 0, kv_splits: int = 0, num_sms: int = 0) -> int:
+    return int(lib().wpattn_prefill_split_workspace_size(B, Nq, Nk, Hq, D, q_pos0, k_pos0,
+                                                         kv_splits, num_sms))
+
+
 def prefill(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0, scale: float | None = None,
-            out=None, lse=None, want_lse: bool = True, stream=None, check: bool = False):
+            out=None, lse=None, want_lse: bool = True, stream=None, check: bool = False,
+            kv_splits: int | None = None, workspace=None):
     """Windowed causal prefill.  q [B,Nq,Hq,D], k/v [B,Nk,Hkv,D] bf16 CUDA tensors.
 
-    Returns (out [B,Nq,Hq,D] bf16, lse [B,Hq,Nq] fp32 or None).  The call is
-    asynchronous; a kernel that gave up a bounded wait is reported only by
-    ``device_status()``, unless ``check`` (synchronise and raise).
+    Returns (out [B,Nq,Hq,D] bf16, lse [B,Hq,Nq] fp32 or None).  ``kv_splits``
+    splits work items' key ranges into parts merged by their log-sum-exp
+    (None or 0: the library's plan, ``prefill_split_plan``; 1: no split; 2..64:
+    every item); a split needs ``workspace`` (uint8 CUDA, allocated here if None).
+    The call is asynchronous; a kernel that gave up a bounded wait is reported
+    only by ``device_status()``, unless ``check`` (synchronise and raise).
     """
     import torch
     B, Nq, Hq, D, Nk, Hkv = _prefill_shapes(q, k, v, w, out, lse)
@@ -214,12 +246,27 @@ def prefill(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0, scale: floa
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
-    rc = lib().wpattn_prefill(ctypes.byref(w._c()), _dev_tensor(q, "q"), _dev_tensor(k, "k"),
-                              _dev_tensor(v, "v"), _dev_tensor(out, "out"),
-                              ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
-                              B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0,
-                              float(scale) if scale else 0.0, _stream_ptr(stream))
-    _check(rc, "wpattn_prefill")
+    kv_splits = 0 if kv_splits is None else int(kv_splits)
+    lse_p = ctypes.c_void_p(lse.data_ptr()) if lse is not None else None
+    need = (prefill_split_workspace_size(B, Nq, Nk, Hq, D, q_pos0, k_pos0, kv_splits)
+            if kv_splits != 1 and B and Nq and Nk else 0)
+    if need > 0 or not 0 <= kv_splits <= 64:
+        if workspace is None and need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        rc = lib().wpattn_prefill_split(ctypes.byref(w._c()), _dev_tensor(q, "q"), _dev_tensor(k, "k"),
+                                        _dev_tensor(v, "v"), _dev_tensor(out, "out"), lse_p,
+                                        B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0,
+                                        float(scale) if scale else 0.0, kv_splits,
+                                        ctypes.c_void_p(workspace.data_ptr()) if workspace is not None
+                                        else None, workspace.numel() if workspace is not None else 0,
+                                        _stream_ptr(stream))
+        _check(rc, "wpattn_prefill_split")
+    else:
+        rc = lib().wpattn_prefill(ctypes.byref(w._c()), _dev_tensor(q, "q"), _dev_tensor(k, "k"),
+                                  _dev_tensor(v, "v"), _dev_tensor(out, "out"), lse_p,
+                                  B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0,
+                                  float(scale) if scale else 0.0, _stream_ptr(stream))
+        _check(rc, "wpattn_prefill")
     if check:
         _check(device_status(stream), "wpattn_prefill (device status)")
     return out, lse
@@ -291,6 +338,25 @@ def rope(x, *, base: float, pos0: int = 0, positions=None, out=None, stream=None
                              _int32_dev(positions, "positions") if positions is not None else None,
                              float(base), _stream_ptr(stream)), "wpattn_rope")
     return out
+
+
+def rope_qk(q, k, *, base: float, q_pos0: int = 0, k_pos0: int = 0, q_out=None, k_out=None,
+            stream=None):
+    """RoPE of a prefill's q [B, Nq, Hq, D] at q_pos0 + t and k [B, Nk, Hkv, D] at
+    k_pos0 + j in one launch, each as ``rope`` would turn it.  Returns (q_out, k_out)."""
+    import torch
+    B, Nq, Hq, D = q.shape
+    if k.dim() != 4 or k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("k must be [B, Nk, Hkv, D] with q's B and D")
+    Nk, Hkv = k.shape[1], k.shape[2]
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    if tuple(q_out.shape) != tuple(q.shape) or tuple(k_out.shape) != tuple(k.shape):
+        raise ValueError("q_out / k_out must have the shapes of q / k")
+    _check(lib().wpattn_rope_qk(_dev_tensor(q, "q"), _dev_tensor(q_out, "q_out"), _dev_tensor(k, "k"),
+                                _dev_tensor(k_out, "k_out"), B, Nq, Nk, Hq, Hkv, D, q_pos0, k_pos0,
+                                float(base), _stream_ptr(stream)), "wpattn_rope_qk")
+    return q_out, k_out
 
 
 def prefill_rope(q, k, v, w: Window, *, q_pos0: int = 0, k_pos0: int = 0,

@@ -51,7 +51,7 @@ struct DeviceInfo {
   int decode_slots = 0;  // decode CTAs resident on the whole GPU at once
   // shared-memory attribute set, per prefill instantiation: (D 64, 128) x (g 1, 8) x
   // (plain, block mask, positions); atomic because host threads may launch concurrently
-  std::atomic<bool> prefill_attr[12] = {};
+  std::atomic<bool> prefill_attr[16] = {};
   void* static_scratch = nullptr;  // device address of g_decode_static_scratch
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -133,28 +133,34 @@ void rope_thetas(double base, int D, double* theta) {
     theta[p] = p < D / 2 ? std::pow(base, -static_cast<double>(2 * p) / static_cast<double>(D)) : 0.0;
 }
 
-int launch_rope(const void* x, void* out, int64_t B, int64_t N, int H, int D, int64_t pos0,
-                const int32_t* pos, double base, int num_sms, cudaStream_t st) {
+// Rotation of one tensor, or of two in one launch (x1 null for one).  Every
+// tensor has B sequences and the same head dim D.
+int launch_rope(const void* x0, void* out0, int64_t N0, int H0, int64_t pos0_0, const int32_t* pos,
+                const void* x1, void* out1, int64_t N1, int H1, int64_t pos0_1, int64_t B, int D,
+                double base, int num_sms, cudaStream_t st) {
   RopeParams rp;
   std::memset(&rp, 0, sizeof rp);
-  rp.x = static_cast<const uint16_t*>(x);
-  rp.out = static_cast<uint16_t*>(out);
-  rp.pos = pos;
-  rp.pos0 = pos0;
-  rp.B = B;
-  rp.N = N;
-  rp.H = H;
+  rp.seg[0] = RopeSegment{static_cast<const uint16_t*>(x0), static_cast<uint16_t*>(out0), pos, pos0_0,
+                          N0, H0};
+  rp.nseg = 1;
+  if (x1 && N1 > 0) {
+    rp.seg[1] = RopeSegment{static_cast<const uint16_t*>(x1), static_cast<uint16_t*>(out1), nullptr,
+                            pos0_1, N1, H1};
+    rp.nseg = 2;
+  }
   rope_thetas(base, D, rp.theta);
-  const uint64_t n = static_cast<uint64_t>(B) * N * (D / 16);  // (token, 8-pair chunk) items
-  if (n == 0) return WPATTN_OK;
-  const uint64_t want = (n + 255) / 256;
+  // (token, 8-pair chunk) items
+  rp.items0 = static_cast<uint64_t>(B) * N0 * (D / 16);
+  rp.items = rp.items0 + (rp.nseg == 2 ? static_cast<uint64_t>(B) * N1 * (D / 16) : 0);
+  if (rp.items == 0) return WPATTN_OK;
+  const uint64_t want = (rp.items + 255) / 256;
   const unsigned grid = static_cast<unsigned>(std::min<uint64_t>(want, static_cast<uint64_t>(num_sms) * 8));
   if (D == 64) rope_kernel<64><<<grid, 256, 0, st>>>(rp);
   else rope_kernel<128><<<grid, 256, 0, st>>>(rp);
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
-template <int D, bool G8, bool MASK, bool POS>
+template <int D, bool G8, bool MASK, bool POS, bool SPLIT = false>
 int launch_prefill(const void* q, const void* k, const void* v, PrefillParams prm,
                    DeviceInfo* dev, cudaStream_t st) {
   using Shape = PrefillShape<D>;
@@ -169,31 +175,49 @@ int launch_prefill(const void* q, const void* k, const void* v, PrefillParams pr
   if ((rc = encode_bf16_4d(&tk, k, D, nk, hk, prm.B, 8, Shape::BN, false)) != WPATTN_OK) return rc;
   if ((rc = encode_bf16_4d(&tv, v, D, nk, hk, prm.B, 64, Shape::BN, true)) != WPATTN_OK) return rc;
   constexpr int smem = PrefillSmem<D>::ALLOC;
-  const int slot = (D == 64 ? 0 : 6) + (G8 ? 3 : 0) + (MASK ? 1 : 0) + (POS ? 2 : 0);
+  const int slot = SPLIT ? 12 + (D == 64 ? 0 : 2) + (G8 ? 1 : 0)
+                         : (D == 64 ? 0 : 6) + (G8 ? 3 : 0) + (MASK ? 1 : 0) + (POS ? 2 : 0);
   // a mask bit covers one 128-row query tile x one 128-key tile
   if (MASK && (Shape::BN != 128 || kBM != 128)) return WPATTN_EUNSUPPORTED;
   if (!dev->prefill_attr[slot].load(std::memory_order_acquire)) {
-    if (cudaFuncSetAttribute(prefill_kernel<D, G8, MASK, POS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(prefill_kernel<D, G8, MASK, POS, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
       return WPATTN_ECUDA;
     dev->prefill_attr[slot].store(true, std::memory_order_release);
   }
-  dim3 grid(prm.num_ctas_q, prm.Hq, prm.B);
-  prefill_kernel<D, G8, MASK, POS><<<grid, Shape::THREADS, smem, st>>>(tq, tk, tv, prm);
+  if constexpr (SPLIT) {
+    // the split items' parts, then their merge
+    const dim3 grid(static_cast<unsigned>(prm.split_items) * prm.kv_splits);
+    prefill_kernel<D, G8, MASK, POS, true><<<grid, Shape::THREADS, smem, st>>>(tq, tk, tv, prm);
+    if (cudaGetLastError() != cudaSuccess) return WPATTN_ECUDA;
+    prefill_combine_kernel<D><<<static_cast<unsigned>(prm.split_items) * Shape::QT * kBM, D, 0, st>>>(prm);
+  } else {
+    const dim3 grid(prm.num_ctas_q, prm.Hq, prm.B);
+    prefill_kernel<D, G8, MASK, POS, false><<<grid, Shape::THREADS, smem, st>>>(tq, tk, tv, prm);
+  }
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
 }
 
-template <int D, bool MASK, bool POS>
+template <int D, bool MASK, bool POS, bool SPLIT = false>
 int launch_prefill_g(const void* q, const void* k, const void* v, const PrefillParams& prm,
                      DeviceInfo* dev, cudaStream_t st) {
-  return prm.g8 ? launch_prefill<D, true, MASK, POS>(q, k, v, prm, dev, st)
-                : launch_prefill<D, false, MASK, POS>(q, k, v, prm, dev, st);
+  return prm.g8 ? launch_prefill<D, true, MASK, POS, SPLIT>(q, k, v, prm, dev, st)
+                : launch_prefill<D, false, MASK, POS, SPLIT>(q, k, v, prm, dev, st);
 }
 
 template <int D>
 int launch_prefill_mode(const void* q, const void* k, const void* v, const PrefillParams& prm,
                         DeviceInfo* dev, cudaStream_t st) {
   if (prm.block_mask && prm.q_pos) return WPATTN_EUNSUPPORTED;
+  if (prm.kv_splits > 1) {
+    // the unsplit kernel takes the items below item_end (full waves), the split
+    // kernel the rest
+    if (prm.block_mask || prm.q_pos) return WPATTN_EUNSUPPORTED;
+    int rc = WPATTN_OK;
+    if (prm.item_end > 0) rc = launch_prefill_g<D, false, false, false>(q, k, v, prm, dev, st);
+    if (rc != WPATTN_OK) return rc;
+    return launch_prefill_g<D, false, false, true>(q, k, v, prm, dev, st);
+  }
   if (prm.block_mask) return launch_prefill_g<D, true, false>(q, k, v, prm, dev, st);
   if (prm.q_pos) return launch_prefill_g<D, false, true>(q, k, v, prm, dev, st);
   return launch_prefill_g<D, false, false>(q, k, v, prm, dev, st);
@@ -357,13 +381,68 @@ int wpattn_pruned_fraction(const wpattn_window* w, int64_t Nq, int64_t Nk, int64
 }  // extern "C"
 
 namespace {
+constexpr int kPrefillBN = 128;  // keys per key tile of the prefill kernel (both head dims)
+static_assert(PrefillShape<64>::BN == kPrefillBN && PrefillShape<128>::BN == kPrefillBN,
+              "the split plan counts key tiles of 128 keys");
+
+constexpr int kItemRows = 256;   // query rows of one work item (two 128-row tiles)
+
+// Which work items (CTAs of the unsplit grid) run with their key range split,
+// and into how many parts: main_items run unsplit, the split_items after
+// them as parts of per key tiles each.
+struct SplitPlan {
+  int64_t items = 0, main_items = 0;
+  int split_items = 0, parts = 1, per = 0;
+  size_t bytes(int D) const {   // fp32 O parts, then the parts' log2-sum-exps
+    return split_items > 0 ? static_cast<size_t>(parts) * split_items * kItemRows * (D + 1) * sizeof(float)
+                           : 0;
+  }
+};
+
+// kv_splits >= 2: every item in kv_splits parts.  kv_splits == 0: when every
+// item does about the same work (the last query sees at most 10% more keys
+// than the first, as for a chunk far into a long context), the items of the
+// grid's last partial wave (one CTA per SM) are split into min(8, num_sms /
+// their count) parts of at least 64 key tiles, so that they finish in a
+// fraction of a wave.  Otherwise (and for kv_splits == 1) nothing is split.
+SplitPlan make_split_plan(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t qk_off,
+                          int kv_splits, int num_sms) {
+  SplitPlan sp;
+  sp.items = (Nq + kItemRows - 1) / kItemRows * Hq * B;
+  sp.main_items = sp.items;
+  if (B <= 0 || Nq <= 0 || Nk <= 0 || Hq <= 0 || kv_splits == 1) return sp;
+  const int64_t nkt = (Nk + kPrefillBN - 1) / kPrefillBN;
+  int S = kv_splits;
+  int64_t first_split = 0;
+  if (kv_splits == 0) {
+    const int64_t first = std::min<int64_t>(std::max<int64_t>(qk_off + 1, 0), Nk);
+    const int64_t last = std::min<int64_t>(std::max<int64_t>(qk_off + Nq, 0), Nk);
+    if (num_sms <= 0 || last <= 0 || first * 10 < last * 9) return sp;
+    const int64_t r = sp.items % num_sms;
+    if (r == 0) return sp;
+    S = static_cast<int>(std::min<int64_t>(8, num_sms / r));
+    S = static_cast<int>(std::min<int64_t>(S, ((last + kPrefillBN - 1) / kPrefillBN) / 64));
+    if (S < 2) return sp;
+    first_split = sp.items - r;
+  }
+  const int64_t per = (nkt + S - 1) / S;
+  S = static_cast<int>((nkt + per - 1) / per);   // no part past the last key tile
+  if (S < 2) return sp;
+  sp.main_items = first_split;
+  sp.split_items = static_cast<int>(sp.items - first_split);
+  sp.parts = S;
+  sp.per = static_cast<int>(per);
+  return sp;
+}
+
 // wpattn_prefill and wpattn_prefill_masked: block_mask null = no mask
 int prefill_impl(const wpattn_window* w, const void* q, const void* k, const void* v, void* out,
                  float* lse, int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int32_t Hkv,
                  int64_t q_pos0, int64_t k_pos0, float softmax_scale, const uint32_t* block_mask,
                  int32_t mask_words, void* cuda_stream, const int32_t* q_pos = nullptr,
                  int64_t q_pos_stride = 0, const int32_t* k_pos = nullptr,
-                 int64_t k_pos_stride = 0) {
+                 int64_t k_pos_stride = 0, int32_t kv_splits = 1, void* workspace = nullptr,
+                 size_t workspace_bytes = 0) {
   WindowPlan plan;
   int rc = make_window_plan(w, &plan);
   if (rc != WPATTN_OK) return rc;
@@ -415,6 +494,24 @@ int prefill_impl(const wpattn_window* w, const void* q, const void* k, const voi
     prm.mask_words = mask_words;
   }
   for (int p = 0; p < 64; ++p) prm.T[p] = plan.T[p] > INT32_MAX ? INT32_MAX : static_cast<int>(plan.T[p]);
+  prm.item_end = INT64_MAX;
+  if (kv_splits != 1) {
+    const SplitPlan sp = make_split_plan(B, Nq, Nk, Hq, qk_off, kv_splits, dev->num_sms);
+    if (sp.split_items > 0) {
+      if (sp.items > 0x7FFFFFFFLL ||
+          static_cast<int64_t>(sp.split_items) * std::max(sp.parts, kItemRows) > 0x7FFFFFFFLL)
+        return WPATTN_EUNSUPPORTED;
+      if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return WPATTN_EINVAL;
+      if (workspace_bytes < sp.bytes(plan.D)) return WPATTN_EWORKSPACE;
+      prm.item_end = sp.main_items;
+      prm.split_item0 = static_cast<int>(sp.main_items);
+      prm.split_items = sp.split_items;
+      prm.kv_splits = sp.parts;
+      prm.split_tiles = sp.per;
+      prm.part_o = static_cast<float*>(workspace);
+      prm.part_l = prm.part_o + static_cast<size_t>(sp.parts) * sp.split_items * kItemRows * plan.D;
+    }
+  }
   const void* kk = Nk > 0 ? k : q;
   const void* vv = Nk > 0 ? v : q;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
@@ -432,6 +529,47 @@ int wpattn_prefill(const wpattn_window* w, const void* q, const void* k, const v
                    int64_t q_pos0, int64_t k_pos0, float softmax_scale, void* cuda_stream) {
   return prefill_impl(w, q, k, v, out, lse, B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0, softmax_scale,
                       nullptr, 0, cuda_stream);
+}
+
+int wpattn_prefill_split_plan(int32_t B, int32_t Nq, int32_t Nk, int32_t Hq, int64_t q_pos0,
+                              int64_t k_pos0, int32_t kv_splits, int32_t num_sms, int64_t* main_items,
+                              int32_t* split_items, int32_t* parts) {
+  if (B < 0 || Nq < 0 || Nk < 0 || Hq <= 0 || kv_splits < 0 || kv_splits > 64) return WPATTN_EINVAL;
+  if (num_sms <= 0) {
+    DeviceInfo* dev = nullptr;
+    const int rc = device_info(&dev);
+    if (rc != WPATTN_OK) return rc;
+    num_sms = dev->num_sms;
+  }
+  const SplitPlan sp = make_split_plan(B, Nq, Nk, Hq, q_pos0 - k_pos0, kv_splits, num_sms);
+  if (main_items) *main_items = sp.main_items;
+  if (split_items) *split_items = sp.split_items;
+  if (parts) *parts = sp.split_items > 0 ? sp.parts : 1;
+  return WPATTN_OK;
+}
+
+size_t wpattn_prefill_split_workspace_size(int32_t B, int32_t Nq, int32_t Nk, int32_t Hq,
+                                           int32_t head_dim, int64_t q_pos0, int64_t k_pos0,
+                                           int32_t kv_splits, int32_t num_sms) {
+  if (B <= 0 || Nq <= 0 || Nk <= 0 || Hq <= 0 || (head_dim != 64 && head_dim != 128) ||
+      kv_splits < 0 || kv_splits > 64)
+    return 0;
+  if (num_sms <= 0) {
+    DeviceInfo* dev = nullptr;
+    if (device_info(&dev) != WPATTN_OK) return 0;
+    num_sms = dev->num_sms;
+  }
+  return make_split_plan(B, Nq, Nk, Hq, q_pos0 - k_pos0, kv_splits, num_sms).bytes(head_dim);
+}
+
+int wpattn_prefill_split(const wpattn_window* w, const void* q, const void* k, const void* v,
+                         void* out, float* lse, int32_t B, int32_t Nq, int32_t Nk, int32_t Hq,
+                         int32_t Hkv, int64_t q_pos0, int64_t k_pos0, float softmax_scale,
+                         int32_t kv_splits, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  if (kv_splits < 0 || kv_splits > 64) return WPATTN_EINVAL;
+  return prefill_impl(w, q, k, v, out, lse, B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0, softmax_scale,
+                      nullptr, 0, cuda_stream, nullptr, 0, nullptr, 0, kv_splits, workspace,
+                      workspace_bytes);
 }
 
 int wpattn_prefill_masked(const wpattn_window* w, const void* q, const void* k, const void* v,
@@ -481,8 +619,30 @@ int wpattn_rope(const void* x, void* out, int32_t B, int32_t N, int32_t H, int32
   DeviceInfo* dev = nullptr;
   int rc;
   if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
-  return launch_rope(x, out, B, N, H, head_dim, pos0, positions, rope_base, dev->num_sms,
-                     static_cast<cudaStream_t>(cuda_stream));
+  return launch_rope(x, out, N, H, pos0, positions, nullptr, nullptr, 0, 0, 0, B, head_dim, rope_base,
+                     dev->num_sms, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int wpattn_rope_qk(const void* q, void* q_out, const void* k, void* k_out, int32_t B, int32_t Nq,
+                   int32_t Nk, int32_t Hq, int32_t Hkv, int32_t head_dim, int64_t q_pos0, int64_t k_pos0,
+                   double rope_base, void* cuda_stream) {
+  if (B < 0 || Nq < 0 || Nk < 0 || Hq <= 0 || Hkv <= 0) return WPATTN_EINVAL;
+  if (!(rope_base > 1.0) || std::isinf(rope_base)) return WPATTN_EINVAL;
+  if (head_dim != 64 && head_dim != 128) return WPATTN_EUNSUPPORTED;
+  if (q_pos0 < 0 || k_pos0 < 0 || q_pos0 > (int64_t(1) << 40) || k_pos0 > (int64_t(1) << 40))
+    return WPATTN_EINVAL;
+  if (B == 0 || (Nq == 0 && Nk == 0)) return WPATTN_OK;
+  if (Nq > 0 && (!q || !q_out || !aligned16(q) || !aligned16(q_out))) return WPATTN_EINVAL;
+  if (Nk > 0 && (!k || !k_out || !aligned16(k) || !aligned16(k_out))) return WPATTN_EINVAL;
+  DeviceInfo* dev = nullptr;
+  int rc;
+  if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (Nq == 0)
+    return launch_rope(k, k_out, Nk, Hkv, k_pos0, nullptr, nullptr, nullptr, 0, 0, 0, B, head_dim,
+                       rope_base, dev->num_sms, st);
+  return launch_rope(q, q_out, Nq, Hq, q_pos0, nullptr, Nk > 0 ? k : nullptr, k_out, Nk, Hkv, k_pos0, B,
+                     head_dim, rope_base, dev->num_sms, st);
 }
 
 size_t wpattn_prefill_rope_workspace_size(int32_t B, int32_t Nq, int32_t Nk, int32_t Hq,
@@ -512,17 +672,11 @@ int wpattn_prefill_rope(const wpattn_window* w, const void* q, const void* k, co
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* qr = ws;
   void* kr = ws + ((static_cast<size_t>(B) * Nq * Hq * plan.D * 2 + 255) / 256) * 256;
-  DeviceInfo* dev = nullptr;
-  if ((rc = device_info(&dev)) != WPATTN_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   // the rotations are a pre-pass: each key row is turned once, not once per
-  // query block that reads it, and off the MUFU pipe the attention needs
-  if ((rc = launch_rope(q, qr, B, Nq, Hq, plan.D, q_pos0, nullptr, w->rope_base, dev->num_sms, st)) !=
-      WPATTN_OK)
-    return rc;
-  if (Nk > 0 &&
-      (rc = launch_rope(k, kr, B, Nk, Hkv, plan.D, k_pos0, nullptr, w->rope_base, dev->num_sms, st)) !=
-          WPATTN_OK)
+  // query block that reads it, and off the MUFU pipe the attention needs;
+  // q and k go in one launch
+  if ((rc = wpattn_rope_qk(q, qr, k, kr, B, Nq, Nk, Hq, Hkv, plan.D, q_pos0, k_pos0, w->rope_base,
+                           cuda_stream)) != WPATTN_OK)
     return rc;
   return prefill_impl(w, qr, kr, v, out, lse, B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0, softmax_scale,
                       nullptr, 0, cuda_stream);

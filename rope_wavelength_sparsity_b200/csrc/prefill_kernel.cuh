@@ -89,6 +89,21 @@ struct PrefillParams {
   const int32_t* q_pos;
   const int32_t* k_pos;
   int64_t q_pos_stride, k_pos_stride;
+  // Work items: the CTA of query block bx (longest rows first) of head h and
+  // sequence b is item (b * Hq + h) * num_ctas_q + bx, its linear block index
+  // in the unsplit grid.  The unsplit kernel runs items below item_end.
+  int64_t item_end;
+  // The split kernel runs items split_item0 .. split_item0 + split_items - 1,
+  // each as kv_splits CTAs (block x = local item * kv_splits + s): part s
+  // attends only key tiles [s * split_tiles, (s + 1) * split_tiles) and writes
+  // its rows' result, normalised over that range's keys, to part_o
+  // [kv_splits][split_items * 256][D] fp32 and the log2-sum-exp of its scores
+  // (-inf when it has none) to part_l [kv_splits][split_items * 256], at row
+  // (s * split_items + local item) * 256 + the row's index within the item.
+  int split_item0, split_items;
+  int kv_splits, split_tiles;
+  float* part_o;
+  float* part_l;
 };
 
 template <int D>
@@ -130,8 +145,10 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 // mask selects the key tiles (compile-time too, so that the plain causal walk
 // keeps its registers).  POS: explicit, non-decreasing positions per token;
 // every column range that the contiguous kernel derives from a distance is
-// found by a binary search over the key tile's positions instead.
-template <int D, bool G8, bool MASK, bool POS>
+// found by a binary search over the key tile's positions instead.  SPLIT: the
+// key range is split into p.kv_splits parts (a compile-time switch too: the
+// unsplit kernel keeps its registers).
+template <int D, bool G8, bool MASK, bool POS, bool SPLIT>
 __global__ void __launch_bounds__(PrefillShape<D>::THREADS, PrefillShape<D>::CTAS_PER_SM)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ PrefillParams p) {
@@ -174,10 +191,27 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cq = p.num_ctas_q - 1 - blockIdx.x;  // longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
+  int cq, h, b, part = 0, local_item = 0;
+  if constexpr (SPLIT) {
+    local_item = static_cast<int>(blockIdx.x) / p.kv_splits;
+    part = static_cast<int>(blockIdx.x) % p.kv_splits;
+    const int item = p.split_item0 + local_item;
+    const int hb = item / p.num_ctas_q;
+    cq = p.num_ctas_q - 1 - (item % p.num_ctas_q);
+    h = hb % p.Hq;
+    b = hb / p.Hq;
+  } else {
+    if ((static_cast<int64_t>(blockIdx.z) * p.Hq + blockIdx.y) * p.num_ctas_q + blockIdx.x >= p.item_end)
+      return;  // an item the split kernel runs
+    cq = p.num_ctas_q - 1 - blockIdx.x;  // longest rows first
+    h = blockIdx.y;
+    b = blockIdx.z;
+  }
   const int kvh = h / p.G;
   const int nkt = (p.Nk + BN - 1) / BN;
+  // the key tiles this CTA may attend: all of them, or its part's range
+  const int kt_lo = SPLIT ? part * p.split_tiles : 0;
+  const int kt_hi = SPLIT ? min(kt_lo + p.split_tiles, nkt) - 1 : nkt - 1;
 
   // Positions.  Without POS query i sits at qk_off + i and key j at j
   // (relative to the first key); with POS they are read from the arrays.
@@ -220,19 +254,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   };
   int kt_last[QT];
 #pragma unroll
-  for (int t = 0; t < QT; ++t) kt_last[t] = last_key_tile(t);
+  for (int t = 0; t < QT; ++t) kt_last[t] = SPLIT ? min(last_key_tile(t), kt_hi) : last_key_tile(t);
   // Key tiles query tile t attends: at most its causal limit lim, and with a
   // block mask only those whose bit is set.  Largest such tile <= kt, or -1.
   const int nqt = (p.Nq + kBM - 1) / kBM;
   auto attended_below = [&](int t, int kt, int lim) -> int {
     kt = min(kt, lim);
-    if (kt < 0) return -1;
+    if (kt < kt_lo) return -1;
     if constexpr (!MASK) return kt;
     const uint32_t* row =
         p.block_mask + ((size_t)(b * p.Hq + h) * nqt + (QT * cq + t)) * p.mask_words;
-    while (kt >= 0) {
+    while (kt >= kt_lo) {
       const uint32_t w = __ldg(row + (kt >> 5)) & (0xFFFFFFFFu >> (31 - (kt & 31)));
-      if (w) return (kt & ~31) + 31 - __clz(w);
+      if (w) {
+        const int u = (kt & ~31) + 31 - __clz(w);
+        return u >= kt_lo ? u : -1;
+      }
       kt = (kt & ~31) - 1;
     }
     return -1;
@@ -248,9 +285,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int u = min(kt, top);
       uint32_t bits = 0;
 #pragma unroll
-      for (int t = 0; t < QT; ++t) bits |= (u >= 0 && u <= kt_last[t]) ? (1u << t) : 0u;
+      for (int t = 0; t < QT; ++t) bits |= (u >= kt_lo && u <= kt_last[t]) ? (1u << t) : 0u;
       *mem = bits;
-      return u < 0 ? -1 : u;
+      return u < kt_lo ? -1 : u;
     }
     int a[QT], u = -1;
 #pragma unroll
@@ -262,10 +299,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     return u;
   };
   uint32_t mem_top;
-  const int kt_top = stream_below(nkt - 1, &mem_top);  // first step of the stream, -1 if none
+  const int kt_top = stream_below(kt_hi, &mem_top);  // first step of the stream, -1 if none
   // the step after key tile kt (for the roles that do not need the bits)
   auto stream_next = [&](int kt) -> int {
-    if constexpr (!MASK) return kt - 1;
+    if constexpr (!MASK) return kt > kt_lo ? kt - 1 : -1;
     uint32_t unused;
     return stream_below(kt - 1, &unused);
   };
@@ -471,7 +508,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint32_t mem_n = 0;
         int kt_n;
         if constexpr (MASK) kt_n = stream_below(kt - 1, &mem_n);
-        else kt_n = kt - 1;
+        else kt_n = kt > kt_lo ? kt - 1 : -1;
         const bool next = kt_n >= 0;
         if (next && !mbar_wait(k_full((j + 1) % NS), ((j + 1) / NS) & 1)) { ok = false; break; }
         if (!mbar_wait(v_full(j % NS), (j / NS) & 1)) { ok = false; break; }
@@ -521,7 +558,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint8_t* smem_q = smem + L::OFF_Q + t * L::QTILE;
     uint8_t* smem_qm = smem + L::OFF_QM + t * 2 * PANEL_Q;
     const int i_tile0 = q_first(t);           // position of the tile's first row
-    const int my_kt_last = last_key_tile(t);
+    const int my_kt_last = SPLIT ? min(last_key_tile(t), kt_hi) : last_key_tile(t);
     int my_next = attended_below(t, my_kt_last, my_kt_last);  // this tile's next key tile, -1 when done
     float m_ref = -INFINITY;   // exponent reference of O and l (log2 units)
     float l_run = 0.f;
@@ -586,7 +623,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int plo = plo_next, ps = ps_next;
       const bool all_pruned = plo >= P;
       if constexpr (MASK) my_next = attended_below(t, kt - 1, my_kt_last);
-      else my_next = kt - 1;  // below the first attended tile, every tile is attended
+      else my_next = kt > kt_lo ? kt - 1 : -1;  // below the first attended tile, every tile is attended
       if (my_next >= 0) {
         advance_plo(t, my_next, plo_next);
         ps_next = split_pair(t, my_next, plo_next, psr);
@@ -940,7 +977,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tmem_st32u(tS + 32, &pk[32]);
       }
       // the next tile's masked Q step, before P is released to the MMA warp
-      if (MASK ? my_next >= 0 : kt > 0) write_masked_q(ps_next);
+      if (MASK ? my_next >= 0 : kt > kt_lo) write_masked_q(ps_next);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -950,12 +987,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     // epilogue: O / l
     const bool row_ok = row < p.Nq;
-    uint16_t* orow = p.out + (((size_t)b * p.Nq + (row_ok ? row : 0)) * p.Hq + h) * D;
+    const size_t out_row = ((size_t)b * p.Nq + (row_ok ? row : 0)) * p.Hq + h;
+    uint16_t* orow = p.out + out_row * D;
     if (cnt > 0) {
       ok = __all_sync(FULL, mbar_wait(o_final(t), 0)) && ok;
       tc_fence_after();
     }
     const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+    // a split's part: fp32 O / l over its keys and the log2-sum-exp of its scores
+    const size_t part_row =
+        SPLIT ? ((size_t)part * p.split_items + local_item) * (QT * kBM) + t * kBM + r : 0;
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
       float o[32];
@@ -965,6 +1006,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
 #pragma unroll
       for (int e = 0; e < 32; ++e) o[e] = (cnt > 0) ? o[e] * inv : 0.f;
+      if constexpr (SPLIT) {
+        if (row_ok) {
+          float4* prow = reinterpret_cast<float4*>(p.part_o + part_row * D + 32 * cc);
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            prow[v4] = make_float4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
+        }
+        continue;
+      }
       if (row_ok) {
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4) {
@@ -977,7 +1027,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
       }
     }
-    if (row_ok && p.lse)
+    if (SPLIT && row_ok)
+      p.part_l[part_row] = (cnt > 0 && l_run > 0.f) ? m_ref + __log2f(l_run) : -INFINITY;
+    else if (row_ok && p.lse)
       p.lse[((size_t)b * p.Hq + h) * p.Nq + row] =
           (l_run > 0.f) ? (m_ref + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
   }
@@ -1006,6 +1058,43 @@ pack_block_mask_kernel(const uint8_t* __restrict__ mask, uint32_t* __restrict__ 
     if (kb < nkb && src[kb]) w |= 1u << i;
   }
   words[idx] = w;
+}
+
+// Merge of the parts of the split kernel's items (one block per row of an
+// item, one thread per head dim): with w_s = 2^(l_s - max l), out = sum_s
+// w_s o_s / sum_s w_s and lse = ln 2 * (max l + log2 sum_s w_s); a row none
+// of whose parts has a key gets 0 and -inf.
+template <int D>
+__global__ void __launch_bounds__(D)
+prefill_combine_kernel(const __grid_constant__ PrefillParams p) {
+  constexpr int ROWS = PrefillShape<D>::QT * kBM;   // query rows of an item
+  const int local_item = static_cast<int>(blockIdx.x) / ROWS;
+  const int lr = static_cast<int>(blockIdx.x) % ROWS;
+  const int item = p.split_item0 + local_item;
+  const int hb = item / p.num_ctas_q;
+  const int cq = p.num_ctas_q - 1 - (item % p.num_ctas_q);
+  const int h = hb % p.Hq, b = hb / p.Hq;
+  const int t = cq * ROWS + lr;
+  if (t >= p.Nq) return;
+  const int e = threadIdx.x;
+  const size_t prow = (size_t)local_item * ROWS + lr;
+  const size_t pstride = (size_t)p.split_items * ROWS;   // rows of one part
+  float M = -INFINITY;
+  for (int s = 0; s < p.kv_splits; ++s) M = fmaxf(M, p.part_l[s * pstride + prow]);
+  float W = 0.f, acc = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < p.kv_splits; ++s) {
+      const float ls = p.part_l[s * pstride + prow];
+      const float w = ls == -INFINITY ? 0.f : ex2_approx(ls - M);
+      W += w;
+      acc = fmaf(w, p.part_o[(s * pstride + prow) * D + e], acc);
+    }
+  }
+  const float val = W > 0.f ? acc / W : 0.f;
+  p.out[(((size_t)b * p.Nq + t) * p.Hq + h) * D + e] = static_cast<uint16_t>(pack_bf16x2(val, 0.f) & 0xFFFFu);
+  if (p.lse && e == 0)
+    p.lse[((size_t)b * p.Hq + h) * p.Nq + t] =
+        W > 0.f ? (M + __log2f(W)) * 0.69314718055994530942f : -INFINITY;
 }
 
 }  // namespace wpattn

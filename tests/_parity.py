@@ -48,14 +48,15 @@ def check_rows(o_gpu, l_gpu, o_ref, l_ref, what):
 
 
 def prefill_parity(q, k, v, *, Hq, Hkv, D, base, alpha, g, q_pos0=0, k_pos0=0, rows=None,
-                   scale=None, what=""):
-    """q, k, v: bf16 tensors (any device).  Returns (max dout, max dlse)."""
+                   scale=None, what="", kv_splits=None):
+    """q, k, v: bf16 tensors (any device).  Returns (max dout, max dlse).
+    kv_splits: passed to wp.prefill (None = the library's choice)."""
     dev = torch.device("cuda:0")
     B, Nq = q.shape[0], q.shape[1]
     scale = scale or 1.0 / math.sqrt(D)
     win = wp.Window(D, base, alpha, g)
     out, lse = wp.prefill(q.to(dev), k.to(dev), v.to(dev), win, q_pos0=q_pos0, k_pos0=k_pos0,
-                          scale=scale)
+                          scale=scale, kv_splits=kv_splits)
     assert wp.device_status() == wp.OK
     if rows is None:
         rows = [(b, h, t) for b in range(B) for h in range(Hq) for t in range(Nq)]

@@ -117,7 +117,52 @@ def test_argument_errors_are_status_codes():
     assert L.wpattn_decode(ctypes.byref(w._c()), ctypes.c_void_p(16), ctypes.c_void_p(16),
                            ctypes.c_void_p(16), kvl, 8, 1, 2, 2, 0.0, ctypes.c_void_p(16), None,
                            None, 0, None) == wp.EINVAL   # kv_len 0
+    # the fused q and k rotation: bad sizes, base, head dim and positions are
+    # refused before any launch; nothing to rotate is a no-op
+    v16 = ctypes.c_void_p(16)
+    assert L.wpattn_rope_qk(v16, v16, v16, v16, -1, 4, 4, 2, 2, 64, 0, 0, 1e4, None) == wp.EINVAL
+    assert L.wpattn_rope_qk(v16, v16, v16, v16, 1, 4, 4, 2, 2, 64, 0, 0, 1.0, None) == wp.EINVAL
+    assert L.wpattn_rope_qk(v16, v16, v16, v16, 1, 4, 4, 2, 2, 96, 0, 0, 1e4, None) == wp.EUNSUPPORTED
+    assert L.wpattn_rope_qk(v16, v16, v16, v16, 1, 4, 4, 2, 2, 64, -1, 0, 1e4, None) == wp.EINVAL
+    assert L.wpattn_rope_qk(v16, v16, v16, v16, 1, 4, 4, 2, 2, 64, 0, 2**41, 1e4, None) == wp.EINVAL
+    assert L.wpattn_rope_qk(None, None, None, None, 1, 4, 0, 2, 2, 64, 0, 0, 1e4, None) == wp.EINVAL
+    assert L.wpattn_rope_qk(None, None, None, None, 1, 0, 0, 2, 2, 64, 0, 0, 1e4, None) == wp.OK
     assert wp.lib().wpattn_strerror(wp.EWORKSPACE).decode() != "unknown status code"
+
+
+def test_prefill_split_plan():
+    """The library's key-range split: only for items of equal work (a chunk far into a
+    long context), and only the items of the grid's last partial wave."""
+    plan = wp.prefill_split_plan
+    # 1M-key chunk, 28 heads: 1792 items = 12 waves of 148 + 16; the 16 go in 8 parts
+    assert plan(1, 16384, 1048576, 28, 1032192, 0, 0, 148) == (1776, 16, 8)
+    # causal self-attention (unequal items), or a grid of whole waves: nothing split
+    assert plan(1, 131072, 131072, 24, 0, 0, 0, 148) == (12288, 0, 1)
+    assert plan(1, 32768, 32768, 14, 0, 0, 0, 148) == (1792, 0, 1)
+    assert plan(1, 256, 1048576, 148, 1048320, 0, 0, 148) == (148, 0, 1)
+    # 20 items on 148 SMs: all of them in 7 parts
+    assert plan(1, 256, 65536, 20, 65280, 0, 0, 148) == (0, 20, 7)
+    # parts of at least 64 key tiles: 16K keys allow 2
+    assert plan(1, 256, 16384, 20, 16128, 0, 0, 148) == (0, 20, 2)
+    assert plan(1, 256, 8192, 20, 7936, 0, 0, 148) == (20, 0, 1)
+    # more than half a wave left over: splitting it gains nothing
+    assert plan(1, 256, 65536, 100, 65280, 0, 0, 148) == (100, 0, 1)
+    # explicit parts: every item; parts past the last key tile are dropped
+    assert plan(2, 300, 1000, 3, 700, 0, 5, 148) == (0, 12, 4)
+    assert plan(1, 300, 1000, 3, 700, 0, 1, 148) == (6, 0, 1)
+    # workspace: parts * split items * 256 rows * (D + 1) fp32
+    ws = wp.prefill_split_workspace_size
+    assert ws(1, 16384, 1048576, 28, 128, 1032192, 0, 0, 148) == 8 * 16 * 256 * 129 * 4
+    assert ws(2, 300, 1000, 3, 64, 700, 0, 5, 148) == 4 * 12 * 256 * 65 * 4
+    assert ws(1, 131072, 131072, 24, 128, 0, 0, 0, 148) == 0
+    assert ws(1, 300, 1000, 3, 96, 700, 0, 5, 148) == 0
+    w = wp.Window(64, 1e4, 1.0, 1)
+    L = wp.lib()
+    for S in (-1, 65):
+        assert L.wpattn_prefill_split(ctypes.byref(w._c()), None, None, None, None, None, 1, 4, 4, 2,
+                                      2, 0, 0, 0.0, S, None, 0, None) == wp.EINVAL
+    with pytest.raises(wp.WpattnError):
+        plan(1, 256, 1024, 2, 0, 0, 65, 148)
 
 
 def test_decode_workspace_size_bounds_every_split_plan():

@@ -81,6 +81,41 @@ def test_rope_kernel_explicit_positions_and_in_place(cuda_dev, D):
         _compare_rotation(inputs.bits(y.cpu()[b]), xb[b], pos[b].numpy(), 5e5, f"D={D} b={b}")
 
 
+QK_CASES = [
+    # D, base, B, Nq, Nk, Hq, Hkv, q_pos0, k_pos0
+    (64, 1e6, 2, 300, 300, 14, 2, 0, 0),        # head counts past and below the 4-head batch
+    (128, 1e7, 1, 100, 700, 7, 1, 600, 0),      # chunked prefill: q at the end of k's range
+    (128, 5e5, 3, 65, 33, 5, 3, 1032192, 77),
+    (64, 1e4, 1, 129, 0, 4, 2, 5, 0),           # Nk = 0: q alone
+]
+
+
+@pytest.mark.parametrize("case", QK_CASES, ids=[str(i) for i in range(len(QK_CASES))])
+def test_rope_qk_one_launch(cuda_dev, case):
+    """The fused q and k rotation equals two separate rotations bit for bit, in
+    place too, and each tensor is within the rotation bound of the oracle."""
+    D, base, B, Nq, Nk, Hq, Hkv, q0, k0 = case
+    s = len(str(case))
+    q = inputs.randn_bf16((B, Nq, Hq, D), 50 * s + 1)
+    k = inputs.randn_bf16((B, Nk, Hkv, D), 50 * s + 2)
+    qd, kd = q.cuda(), k.cuda()
+    qr, kr = wp.rope_qk(qd, kd, base=base, q_pos0=q0, k_pos0=k0)
+    q1 = wp.rope(qd, base=base, pos0=q0)
+    qi, ki = qd.clone(), kd.clone()
+    wp.rope_qk(qi, ki, base=base, q_pos0=q0, k_pos0=k0, q_out=qi, k_out=ki)
+    torch.cuda.synchronize()
+    assert torch.equal(qr, q1) and torch.equal(qi, qr)
+    if Nk > 0:
+        k1 = wp.rope(kd, base=base, pos0=k0)
+        torch.cuda.synchronize()
+        assert torch.equal(kr, k1) and torch.equal(ki, kr)
+    qb, kb = inputs.bits(q), inputs.bits(k)
+    for b in range(B):
+        _compare_rotation(inputs.bits(qr.cpu()[b]), qb[b], q0 + np.arange(Nq), base, f"q b={b}")
+        if Nk > 0:
+            _compare_rotation(inputs.bits(kr.cpu()[b]), kb[b], k0 + np.arange(Nk), base, f"k b={b}")
+
+
 DEC_CASES = [
     # D, g, alpha, base, B, Hq, Hkv, L, kv_len
     (128, 1, 1.0, 5e5, 3, 24, 8, 1000, [1000, 1, 517]),
@@ -171,6 +206,16 @@ def test_rope_rejects_bad_args(cuda_dev):
     with pytest.raises(wp.WpattnError) as e:
         wp.rope(x, base=1e4)
     assert e.value.code == wp.EUNSUPPORTED
+    with pytest.raises(wp.WpattnError) as e:
+        wp.rope_qk(x, x, base=1e4)
+    assert e.value.code == wp.EUNSUPPORTED
+    y = torch.zeros((1, 4, 1, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(wp.WpattnError) as e:
+        wp.rope_qk(y, y, base=1.0)
+    assert e.value.code == wp.EINVAL
+    with pytest.raises(wp.WpattnError) as e:
+        wp.rope_qk(y, y, base=1e4, q_pos0=-1)
+    assert e.value.code == wp.EINVAL
     q = torch.zeros((1, 256, 2, 64), dtype=torch.bfloat16, device="cuda")
     ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
     with pytest.raises(wp.WpattnError) as e:
