@@ -62,11 +62,10 @@ FLUSH_NOTE = ("flushed between steps (512 MiB write, then a 256 MiB read of it: 
 # ncu capture, keyed by workload and by a hash of that kernel's sources at
 # capture time: a changed kernel reports null until it is captured again.
 NCU_TRAFFIC = {
-    # prefill_kernel<128, 1, 0, 0> on the full 1M-key chunk (one pass): 54.71 GB read + 131.40 MB
-    # written; K and V (2.15 GB) come from DRAM about 24 times, at 4 % of the HBM bandwidth
-    ("qwen2.5-7b-1m-prefill", "4507275ab3553a09"): 54710000000 + 131400000,
-    # prefill_kernel<64, 1, 0, 0> on the Qwen2.5-0.5B 32K prefill (one pass): 76.28 MB + 23.42 MB
-    ("qwen2.5-0.5b-32k", "4507275ab3553a09"): 76280000 + 23420000,
+    # prefill_kernel<128, 1, 0, 0, 0> on the full 1M-key chunk, its 1,776 unsplit items (one
+    # pass): 43.46 GB read + 129.93 MB written; K and V (2.15 GB) come from DRAM about 20 times,
+    # at 3 % of the HBM bandwidth
+    ("qwen2.5-7b-1m-prefill", "caed9ad913f38822"): 43460000000 + 129930000,
     # decode_split_kernel<128, 3, 0> on the full B=16, L=131072 Llama decode (one pass):
     # 8.59 GB read + 3.66 MB written (all of K and V: whole rows of the [B, L, Hkv, D] cache)
     ("llama3.2-3b-decode-128k", "668b26ccc741d486"): 8590000000 + 3660000,
