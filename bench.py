@@ -309,6 +309,27 @@ def _tensor_peak(peaks, clk, timed_ms):
     return peaks["bf16_tflops"], f"{peaks['source']} bf16 dense (burst)"
 
 
+# ex2.approx issue rate of one SM (4 per clock per sub-partition; measured with a probe
+# of independent chains, 8 cycles per warp instruction at 1, 2 and 4 warps per SP)
+EXP_PER_CLK_SM = 16
+
+
+def exp_roof(w, off_flops, kernel_ms, clk, dev):
+    """Second roof of a prefill step: every causal (query, key) score needs one exponential
+    on the special-function unit, whatever the window prunes.  Its peak comes from the unit
+    count and the maximum SM clock; floor_ms is the step time at that rate."""
+    import torch
+    exps = off_flops // (4 * w.D)        # window-off FLOPs = 4 D per causal pair and head
+    mhz = (clk or {}).get("sm_max_mhz") or 1965.0
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    peak = EXP_PER_CLK_SM * sms * mhz * 1e6
+    floor_ms = exps / peak * 1e3
+    return {"bound": "mufu", "exps_per_step": int(exps), "peak": peak, "unit": "exp/s",
+            "achieved": round(exps / (kernel_ms * 1e-3), 1), "floor_ms": round(floor_ms, 3),
+            "frac": round(floor_ms / kernel_ms, 4),
+            "peak_source": f"{EXP_PER_CLK_SM}/clk/SM x {sms} SMs x {mhz:.0f} MHz"}
+
+
 def _check_status(wp, what):
     if wp.device_status() != wp.OK:
         raise RuntimeError(f"{what}: kernel status not ok")
@@ -386,6 +407,7 @@ def bench_prefill(w, args, world, rank, dev, flush, peaks, variants=False):
     }
     if unsplit:
         res["unsplit"] = unsplit
+    res["exp_roof"] = exp_roof(w, off_flops, kernel_ms, clk, dev)
     if variants:
         res.update(_prefill_variants(w, args, world, rank, dev, flush, peaks, q, k, v, out, lse,
                                      win, eff, ms_step))
