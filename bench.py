@@ -430,7 +430,37 @@ def bench_prefill(w, args, world, rank, dev, flush, peaks, variants=False):
     _check_status(wp, w.name + " end to end")
     res["e2e"] = {"value": round(world * eff / (e2e_ms / n_e2e * 1e-3) / 1e12, 2),
                   "unit": "TFLOP/s", "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * 2,
-                  "d2h_bytes_per_step": out.numel() * 2}
+                  "d2h_bytes_per_step": out.numel() * 2,
+                  "inputs": "all of q, k and v copied every step"}
+    # A chunk far into a context (keys before the chunk's first query): the earlier keys'
+    # K and V were written by the earlier chunks and stay resident, as a decode's KV cache
+    # does; each step copies the chunk's q and its own k and v rows.
+    new0 = max(0, w.q_pos0 - w.k_pos0)
+    if 0 < new0 < w.Nk:
+        kd_new = [k[b, new0:] for b in range(w.B)]
+        vd_new = [v[b, new0:] for b in range(w.B)]
+        kh_new = [kh[b, new0:] for b in range(w.B)]
+        vh_new = [vh[b, new0:] for b in range(w.B)]
+
+        def step_e2e_chunk():
+            q.copy_(qh, non_blocking=True)
+            for b in range(w.B):
+                kd_new[b].copy_(kh_new[b], non_blocking=True)
+                vd_new[b].copy_(vh_new[b], non_blocking=True)
+            o, _ = wp.prefill(q, k, v, win, q_pos0=w.q_pos0, k_pos0=w.k_pos0, scale=w.scale,
+                              out=out, lse=lse, kv_splits=S, workspace=ws)
+            oh.copy_(o, non_blocking=True)
+
+        c_ms, _, _ = time_steps(step_e2e_chunk, 2, n_e2e, flush, world)
+        _check_status(wp, w.name + " end to end, chunk inputs")
+        new_rows = w.Nk - new0
+        res["e2e_chunk_inputs"] = {
+            "value": round(world * eff / (c_ms / n_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": (q.numel() + 2 * w.B * new_rows * w.Hkv * w.D) * 2,
+            "d2h_bytes_per_step": out.numel() * 2,
+            "inputs": f"q and the chunk's own {new_rows} k and v rows per sequence; the "
+                      f"{new0} earlier keys' K and V resident on the device"}
+        del kd_new, vd_new, kh_new, vh_new
     del q, k, v, out, lse, qh, kh, vh, oh, ws
     torch.cuda.empty_cache()
     return res
