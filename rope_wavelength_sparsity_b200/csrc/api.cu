@@ -192,7 +192,7 @@ int launch_prefill(const void* q, const void* k, const void* v, PrefillParams pr
     if (cudaGetLastError() != cudaSuccess) return WPATTN_ECUDA;
     prefill_combine_kernel<D><<<static_cast<unsigned>(prm.split_items) * Shape::QT * kBM, D, 0, st>>>(prm);
   } else {
-    const dim3 grid(prm.num_ctas_q, prm.Hq, prm.B);
+    const dim3 grid = prm.heads_fast ? dim3(prm.Hq, prm.B, prm.num_ctas_q) : dim3(prm.num_ctas_q, prm.Hq, prm.B);
     prefill_kernel<D, G8, MASK, POS, false><<<grid, Shape::THREADS, smem, st>>>(tq, tk, tv, prm);
   }
   return cudaGetLastError() == cudaSuccess ? WPATTN_OK : WPATTN_ECUDA;
@@ -511,6 +511,15 @@ int prefill_impl(const wpattn_window* w, const void* q, const void* k, const voi
       prm.part_o = static_cast<float*>(workspace);
       prm.part_l = prm.part_o + static_cast<size_t>(sp.parts) * sp.split_items * kItemRows * plan.D;
     }
+  }
+  // Heaviest query blocks of every head first when the whole K and V stay in L2
+  // (concurrent CTAs of many heads then share no L2 working set they would
+  // thrash); otherwise one head's blocks after another, so that concurrent CTAs
+  // walk the same K and V.
+  {
+    const int64_t nq_ctas = (static_cast<int64_t>(Nq) + 255) / 256;
+    const int64_t kv_bytes = static_cast<int64_t>(B) * Nk * Hkv * plan.D * 4;
+    prm.heads_fast = (prm.item_end == INT64_MAX && nq_ctas <= 65535 && kv_bytes <= (int64_t(48) << 20)) ? 1 : 0;
   }
   const void* kk = Nk > 0 ? k : q;
   const void* vv = Nk > 0 ? v : q;

@@ -101,6 +101,9 @@ struct PrefillParams {
   // (-inf when it has none) to part_l [kv_splits][split_items * 256], at row
   // (s * split_items + local item) * 256 + the row's index within the item.
   int split_item0, split_items;
+  // unsplit grid (Hq, B, num_ctas_q) instead of (num_ctas_q, Hq, B): every head's
+  // heaviest query blocks are dispatched before any head's lighter ones
+  int heads_fast;
   int kv_splits, split_tiles;
   float* part_o;
   float* part_l;
@@ -200,6 +203,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     cq = p.num_ctas_q - 1 - (item % p.num_ctas_q);
     h = hb % p.Hq;
     b = hb / p.Hq;
+  } else if (p.heads_fast) {
+    cq = p.num_ctas_q - 1 - blockIdx.z;  // longest rows first, across all heads
+    h = blockIdx.x;
+    b = blockIdx.y;
   } else {
     if ((static_cast<int64_t>(blockIdx.z) * p.Hq + blockIdx.y) * p.num_ctas_q + blockIdx.x >= p.item_end)
       return;  // an item the split kernel runs
