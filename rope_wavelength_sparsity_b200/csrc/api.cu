@@ -519,7 +519,8 @@ int prefill_impl(const wpattn_window* w, const void* q, const void* k, const voi
   {
     const int64_t nq_ctas = (static_cast<int64_t>(Nq) + 255) / 256;
     const int64_t kv_bytes = static_cast<int64_t>(B) * Nk * Hkv * plan.D * 4;
-    prm.heads_fast = (prm.item_end == INT64_MAX && nq_ctas <= 65535 && kv_bytes <= (int64_t(48) << 20)) ? 1 : 0;
+    prm.heads_fast = (prm.g8 && prm.item_end == INT64_MAX && nq_ctas <= 65535 &&
+                      kv_bytes <= (int64_t(48) << 20)) ? 1 : 0;
   }
   const void* kk = Nk > 0 ? k : q;
   const void* vv = Nk > 0 ? v : q;

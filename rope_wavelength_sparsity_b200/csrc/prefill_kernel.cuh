@@ -102,7 +102,7 @@ struct PrefillParams {
   // (s * split_items + local item) * 256 + the row's index within the item.
   int split_item0, split_items;
   // unsplit grid (Hq, B, num_ctas_q) instead of (num_ctas_q, Hq, B): every head's
-  // heaviest query blocks are dispatched before any head's lighter ones
+  // heaviest query blocks are dispatched before any head's lighter ones (g = 8 only)
   int heads_fast;
   int kv_splits, split_tiles;
   float* part_o;
@@ -203,7 +203,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     cq = p.num_ctas_q - 1 - (item % p.num_ctas_q);
     h = hb % p.Hq;
     b = hb / p.Hq;
-  } else if (p.heads_fast) {
+  } else if (G8 && p.heads_fast) {
     cq = p.num_ctas_q - 1 - blockIdx.z;  // longest rows first, across all heads
     h = blockIdx.x;
     b = blockIdx.y;
