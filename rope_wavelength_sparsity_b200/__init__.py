@@ -8,11 +8,12 @@ fallback path: if the shared library is missing or a call fails, an
 exception is raised.
 
 Entry points (same names as the C ABI, without the ``wpattn_`` prefix):
-``prefill``, ``decode``, ``decode_pairmajor``, ``kcache_to_pairmajor``,
-``decode_positions``, ``decode_paged``, ``prefill_masked``, ``pack_block_mask``, ``rope``,
-``prefill_rope``, ``decode_rope``, ``prefill_positions``, ``decode_shard``, ``merge_lse``,
-``decode_workspace_size``, ``decode_noalloc``, ``pruned_fraction``,
-``thresholds``, ``device_status``.
+``prefill`` (with the key-range split of ``prefill_split`` when its plan splits anything;
+``prefill_split_plan``, ``prefill_split_workspace_size``), ``decode``, ``decode_pairmajor``,
+``kcache_to_pairmajor``, ``decode_positions``, ``decode_paged``, ``prefill_masked``,
+``pack_block_mask``, ``rope``, ``rope_qk``, ``prefill_rope``, ``decode_rope``,
+``prefill_positions``, ``decode_shard``, ``merge_lse``, ``decode_workspace_size``,
+``decode_noalloc``, ``pruned_fraction``, ``thresholds``, ``device_status``.
 
 Calls are asynchronous on the given stream (torch's current stream by
 default).  Every wait inside a kernel is bounded; when one runs out, the
