@@ -179,6 +179,18 @@ def decode_row_bytes_oracle(w, L):
     return ((total - pruned) * 4 + L * w.D * 2) / (w.Hq // w.Hkv)
 
 
+def full_step_work_oracle(w, kv_len=None):
+    """Effective FLOPs (prefill) or algorithmic bytes (decode, sequences of kv_len keys) of
+    one whole step of workload w, counted with the oracle's own pair-term count."""
+    import oracle
+    P = w.D // 2
+    if w.kind == "prefill":
+        pruned, total = oracle.count_rows(w.D, w.base, w.alpha, w.g, w.Nq, w.Nk, w.q_pos0,
+                                          w.k_pos0)
+        return w.B * w.Hq * (4 * (total - pruned) + 2 * w.D * (total // P))
+    return sum(w.Hq * decode_row_bytes_oracle(w, int(L)) for L in (kv_len or [w.Nk] * w.B))
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -869,11 +881,15 @@ def reference_arm(args):
             vals.append(val)
             rows_done += n
     value = statistics.mean(vals) if vals else 0.0
+    # the whole workload's step at that rate (its work counted with the oracle's own count)
+    full = full_step_work_oracle(w, getattr(job, "kv_len", None))
+    ms_step = full / (value * job.scale) * 1e3 if value > 0 else None
     sample = (f"each step: rows of {w.name} on {cores} threads for {per_step:.1f} s "
               f"({rows_done} rows over the timed steps); work counted with the oracle's own "
-              "pair-term count")
+              "pair-term count; ms_per_step is the whole workload's step at the measured rate")
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": job.unit,
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(ms_step, 3) if ms_step else None,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic", "config": workload_config(w, world),
            "cpu_baseline": {"value": value, "unit": job.unit, "cores": cores, "kind": "oracle",

@@ -192,3 +192,8 @@ def test_reference_arm_loads_no_product_library():
     assert res["impl"] == "reference" and res["value"] > 0
     assert res["config"]["workload"] == "tiny" and res["config"]["Nk"] == 256
     assert res["cpu_baseline"]["cores"] >= 1 and res["cpu_baseline"]["kind"] == "oracle"
+    # the whole tiny step at the measured rate, its work counted with the oracle
+    import bench
+    from rope_wavelength_sparsity_b200 import inputs
+    full = bench.full_step_work_oracle(inputs.WORKLOADS["tiny"])
+    assert res["ms_per_step"] == pytest.approx(full / (res["value"] * 1e12) * 1e3, rel=1e-3)
