@@ -574,9 +574,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     // Copy of Q's first contracted k-step for a key tile whose split pair is
     // ps, with the pairs below ps zeroed (the MMA reads it instead of Q).
+    // (g = 1) the split pair whose masked copy the buffer holds: the split pair only
+    // moves forward along the walk, and far from the diagonal it stays put for dozens
+    // of key tiles, so the copy and its proxy fence are skipped while it does
+    int qm_ps = -1;
     auto write_masked_q = [&](int ps) {
       const int rz = ps & 7;
       if (rz == 0 || (ps >> 3) >= KS) return;
+      if constexpr (!G8) {
+        if (ps == qm_ps) return;
+        qm_ps = ps;
+      }
       uint4 lo = *reinterpret_cast<const uint4*>(smem_q + (ps >> 3) * PANEL_Q + r * 16);
       uint4 hi = *reinterpret_cast<const uint4*>(smem_q + (P / 8 + (ps >> 3)) * PANEL_Q + r * 16);
       const uint32_t m0 = (rz > 0 ? 0u : 0xFFFFu) | (rz > 1 ? 0u : 0xFFFF0000u);
