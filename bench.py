@@ -63,14 +63,14 @@ FLUSH_NOTE = ("flushed between steps (512 MiB write, then a 256 MiB read of it: 
 # capture time: a changed kernel reports null until it is captured again.
 NCU_TRAFFIC = {
     # prefill_kernel<128, 1, 0, 0, 0> on the full 1M-key chunk, its 1,776 unsplit items (one
-    # pass): 59.81 GB read + 130.62 MB written; K and V (2.15 GB) come from DRAM about 28 times,
-    # at 5 % of the HBM bandwidth (43.5 to 59.8 GB over captures of this grid: the CTAs' drift
+    # pass): 57.86 GB read + 128.71 MB written; K and V (2.15 GB) come from DRAM about 27 times,
+    # at 4-5 % of the HBM bandwidth (43.5 to 59.8 GB over captures of this grid: the CTAs' drift
     # along their walks decides how much an L2 line is shared)
-    ("qwen2.5-7b-1m-prefill", "4b772376e7acd0ff"): 59810000000 + 130620000,
-    # prefill_kernel<64, 1, 0, 0, 0> on the Qwen2.5-0.5B 32K prefill (one pass): 75.71 MB read +
-    # 20.22 MB written, against 75.5 MB of inputs and 60.5 MB of outputs (part of the output is
+    ("qwen2.5-7b-1m-prefill", "e9a4244609de9f9f"): 57860000000 + 128710000,
+    # prefill_kernel<64, 1, 0, 0, 0> on the Qwen2.5-0.5B 32K prefill (one pass): 75.60 MB read +
+    # 21.47 MB written, against 75.5 MB of inputs and 60.5 MB of outputs (part of the output is
     # still in L2 when the kernel ends)
-    ("qwen2.5-0.5b-32k", "4b772376e7acd0ff"): 75710000 + 20220000,
+    ("qwen2.5-0.5b-32k", "e9a4244609de9f9f"): 75600000 + 21470000,
     # decode_split_kernel<128, 3, 0> on the full B=16, L=131072 Llama decode (one pass):
     # 8.59 GB read + 3.66 MB written (all of K and V: whole rows of the [B, L, Hkv, D] cache)
     ("llama3.2-3b-decode-128k", "668b26ccc741d486"): 8590000000 + 3660000,
