@@ -91,6 +91,28 @@ def test_prefill_split_library_plan_last_wave(cuda_dev):
                    what="library plan, last wave")
 
 
+def test_prefill_split_unsplit_items_bitwise(cuda_dev):
+    """Under the library's last-wave plan the unsplit items run the plain kernel: their rows
+    equal an unsplit call bit for bit; the split items' rows agree within the bar."""
+    B, Hq, Hkv, D, Nq, Nk = 1, 150, 2, 64, 256, 65536
+    q0 = Nk - Nq
+    main, n_split, parts = wp.prefill_split_plan(B, Nq, Nk, Hq, q0, 0)
+    if n_split == 0:
+        pytest.skip("this device's plan splits nothing for the shape")
+    q, k, v = _qkv(B, Nq, Nk, Hq, Hkv, D, seed=46)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    win = wp.Window(D, 1e6, 1.0, 8)
+    o_s, l_s = wp.prefill(qd, kd, vd, win, q_pos0=q0)
+    o_1, l_1 = wp.prefill(qd, kd, vd, win, q_pos0=q0, kv_splits=1)
+    torch.cuda.synchronize()
+    assert wp.device_status() == wp.OK
+    # with one query block per head (Nq = 256) item i is head i
+    assert torch.equal(o_s[:, :, :main], o_1[:, :, :main])
+    assert torch.equal(l_s[:, :main], l_1[:, :main])
+    assert (o_s[:, :, main:].float() - o_1[:, :, main:].float()).abs().max().item() <= 1e-2
+    assert (l_s[:, main:] - l_1[:, main:]).abs().max().item() <= 1e-4
+
+
 def test_prefill_split_workspace_checks(cuda_dev):
     q, k, v = _qkv(1, 256, 1024, 2, 1, 64, seed=45)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
