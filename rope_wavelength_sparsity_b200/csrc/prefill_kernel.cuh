@@ -35,6 +35,14 @@
 // [256, 256+D), O_1 at [256+D, 256+2D).  P_t (bf16 pairs) overwrites the
 // first 64 columns of S_t; the next QK of tile t is issued after PV_t, and
 // tcgen05 MMAs of one thread run in issue order.
+//
+// Grid.  One CTA per work item (a 256-row query block of one head of one
+// sequence), heaviest query blocks first: one head after another, or, for
+// g = 8 when K and V fit in L2, every head's heaviest blocks before any
+// head's lighter ones.  The SPLIT instantiation runs work items as several
+// CTAs over disjoint key ranges, each writing a partial result that
+// prefill_combine_kernel merges; the host uses it for the items of a grid's
+// last partial wave when all items do the same work.
 #pragma once
 
 #include "device_util.cuh"

@@ -123,3 +123,15 @@ def test_masked_flops_equal_enumeration():
     # every block attended: the unmasked count
     ones = torch.ones((w.B, w.Hq, nqb, nkb), dtype=torch.bool)
     assert bench.masked_flops(w, win, wp, ones) == bench.prefill_flops(w, win, wp)[0]
+
+
+def test_kernel_hash_ignores_comments_not_code():
+    """The traffic table's key: a comment or layout change keeps the hash, a code change
+    does not."""
+    import bench
+    a = "int f(int x) {  // twice\n  return 2 * x; /* doubled */\n}\n"
+    b = "// the same function\nint f(int x) {\n    return 2 * x;\n}"
+    c = "int f(int x) { return 3 * x; }"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    assert len(bench.kernel_source_hash("prefill")) == 16
